@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark: one Muon step (momentum, Gram Newton-Schulz x5, update) over a
+projection-matrix set, on N GPUs of one node.
+
+A "step" is one dmuon_step call over the whole set (224 bf16 matrices of the
+Llama-7B projection shapes by default).  Inputs are resident in HBM when the
+timed region starts; they total far more than the 126 MB L2 per step, so no
+L2 flush is done between steps.  Per-kernel times come from CUDA events that
+the library records around each of its launches on the launching stream,
+inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 oracle on the host cores
+
+Multi-GPU (torchrun): every rank runs its own replica of the set (weak
+scaling, no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "Muon steps/sec (matrices/s) and NS TFLOP/s as % of B200 BF16 peak, 1 GPU"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama_7b_bf16")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-budget-s", type=float, default=30.0,
+                    help="bound on the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------- peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it still matches the source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(f"{kernel}@{workload}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "newton_schulz_grad_b200", "csrc", ent.get("source", ""))
+    try:
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if digest != ent.get("sha256"):
+        return None  # the kernel changed since the counters were taken
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def _gpu_id(self) -> str:
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = getattr(p, "pci_bus_id", None)
+            dom = getattr(p, "pci_domain_id", 0)
+            devid = getattr(p, "pci_device_id", 0)
+            if bus is not None:
+                return f"{dom:08X}:{bus:02X}:{devid:02X}.0"
+        except Exception:
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[self.dev].strip()
+        return str(self.dev)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self._gpu_id(), f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                if len(r) >= len(self.FIELDS):
+                    rows.append([c.strip() for c in r])
+        os.unlink(self.path)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for k, nm in enumerate(names):
+                if r[5 + k].lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def reduce_max(value: float, device) -> float:
+    """Max over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(count_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job matrices/s: all ranks' matrices over the slowest rank's time."""
+    return world * count_per_rank / (ms_max / 1e3)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def class_samples(w):
+    """One matrix index per launch class (oriented shape), with class sizes."""
+    classes = {}
+    for i, (r, c) in enumerate(w.shapes):
+        key = (min(r, c), max(r, c))
+        classes.setdefault(key, []).append(i)
+    return [(key, idx[0], len(idx)) for key, idx in classes.items()]
+
+
+def oracle_matrix_seconds(w, idx: int) -> float:
+    """Time the oracle's Muon step on matrix idx of w (host fp64)."""
+    from oracle import muon as om
+    p, g, b = workloads.make_matrix(w, idx, "cpu", workloads.skewed_indices(w))
+    p64, g64, b64 = (t.to(torch.float64).numpy() for t in (p, g, b))
+    t0 = time.perf_counter()
+    om.muon_step([p64], [g64], [b64], w.lr, w.momentum, w.nesterov, w.ns_steps, None, w.wd)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s: float):
+    """Oracle matrices/s extrapolated from one timed matrix per launch class."""
+    per_class = []
+    spent = 0.0
+    for key, idx, cnt in sorted(class_samples(w), key=lambda e: e[0][0] ** 2 * e[0][1]):
+        if spent > budget_s and per_class:
+            # out of budget: extrapolate by flops from the cheapest measured class
+            (k0, t0, _) = per_class[0]
+            f0 = 3 * k0[0] ** 2 * k0[1] + k0[0] ** 3
+            f = 3 * key[0] ** 2 * key[1] + key[0] ** 3
+            per_class.append((key, t0 * f / f0, cnt))
+            continue
+        t = oracle_matrix_seconds(w, idx)
+        spent += t
+        per_class.append((key, t, cnt))
+    total = sum(t * cnt for _, t, cnt in per_class)
+    sample = "; ".join(f"1 x {k[0]}x{k[1]} ({t:.2f} s, class of {c})" for k, t, c in per_class)
+    return {"value": w.count / total, "unit": "matrices/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle, one matrix per launch class, extrapolated to the "
+                      f"{w.count}-matrix set by class counts: {sample}"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import newton_schulz_grad_b200 as nsg
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+        pg = dist
+    w = workloads.get(args.workload)
+    ps, gs, bs = workloads.make_all(w, dev)
+    code = 1 if w.dtype == "bf16" else 0
+    shapes = [(r, c, code) for r, c in w.shapes]
+    pp = [t.data_ptr() for t in ps]
+    gp = [t.data_ptr() for t in gs]
+    bp = [t.data_ptr() for t in bs]
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = nsg.dmuon_step_launches(shapes, w.ns_steps)
+
+    def step():
+        nsg.dmuon_step_ptrs(pp, gp, bp, shapes, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
+                            ns_steps=w.ns_steps, wd=w.wd, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    st = nsg.dmuon_stream_status(stream)
+    if st != nsg.DMUON_OK:
+        raise RuntimeError(f"warm-up failed: {nsg.STATUS_NAMES[st]} {nsg.dmuon_get_last_error()}")
+
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    nsg.dmuon_profile_start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    kstats = nsg.dmuon_profile_stop()
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    clk = clocks.stop()
+    st = nsg.dmuon_stream_status(stream)
+    if st != nsg.DMUON_OK:
+        raise RuntimeError(f"timed steps failed: {nsg.STATUS_NAMES[st]}")
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = reduce_max(ms_local, dev)
+    value = aggregate_value(w.count, world, ms)
+
+    peaks, peak_src = load_peaks()
+    chain = {k: v for k, v in kstats.items() if k.endswith("_tc") or k.endswith("_ffma")}
+    chain_ms = sum(v["total_ms"] for v in chain.values()) / args.steps
+    ns_flops = w.ns_flops()
+    ns_tflops_step = ns_flops / (ms / 1e3) / 1e12
+    ns_tflops_chain = ns_flops / (chain_ms / 1e3) / 1e12 if chain_ms > 0 else None
+    # dominant kernel: largest share of the timed region
+    dom = max(kstats.items(), key=lambda kv: kv[1]["total_ms"])
+    dname, d = dom
+    avg_ms = d["total_ms"] / d["launches"]
+    if d["flops"] > 0:
+        achieved = (d["flops"] / d["launches"]) / (avg_ms / 1e3) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        bound, unit = "tensor", "TFLOP/s"
+    else:
+        achieved = (d["bytes"] / d["launches"]) / (avg_ms / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        bound, unit = "hbm", "GB/s"
+    elem = {}
+    for k in ("momentum", "update"):
+        if k in kstats:
+            v = kstats[k]
+            elem[k] = {"GB/s": round(v["bytes"] / (v["total_ms"] / 1e3) / 1e9, 1),
+                       "frac_of_hbm": round(v["bytes"] / (v["total_ms"] / 1e3) / 1e9 /
+                                            float(peaks["hbm_gbs"]), 3),
+                       "ms_per_step": round(v["total_ms"] / args.steps, 3)}
+    kernels = {k: {"launches_per_step": v["launches"] // args.steps,
+                   "ms_per_step": round(v["total_ms"] / args.steps, 3),
+                   "share": round(v["total_ms"] / sum(x["total_ms"] for x in kstats.values()), 4)}
+               for k, v in kstats.items()}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, ps, gs, bs, shapes, stream, dev, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_budget_s)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "matrices/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded low-rank + noise gradients, random-init parameters)",
+        "config": {"workload": w.name, "matrices": w.count,
+                   "shapes": sorted({f"{r}x{c}" for r, c in w.shapes}),
+                   "ns_steps": w.ns_steps, "nesterov": w.nesterov, "lr": w.lr, "wd": w.wd,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"no flush: each step touches {w.elements() * 2 * 7 / 1e9:.1f} GB "
+                         f"(inputs alone {w.elements() * 2 * 3 / 1e9:.1f} GB) >> 126 MB L2"},
+        "ns_tflops": round(ns_tflops_step, 1),
+        "ns_frac_of_peak": round(ns_tflops_step / float(peaks.get("bf16_tflops_sustained",
+                                                               peaks["bf16_tflops"])), 4),
+        "ns_chain_tflops": round(ns_tflops_chain, 1) if ns_tflops_chain else None,
+        "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+        "roofline": {"kernel": dname, "bound": bound, "achieved": round(achieved, 1), "peak": peak,
+                     "unit": unit, "frac": round(achieved / peak, 4),
+                     "traffic": traffic_record(dname, w.name),
+                     "per_launch": {"flops": d["flops"] / d["launches"],
+                                    "bytes": d["bytes"] / d["launches"], "avg_ms": avg_ms}},
+        "elementwise": elem,
+        "kernels": kernels,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+def run_e2e(args, w, ps, gs, bs, shapes, stream, dev, world):
+    """Same metric through the public API with host buffers: every step copies
+    the gradients host->device (pinned) and reads the updated parameters back."""
+    import newton_schulz_grad_b200 as nsg
+    try:
+        g_host = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in gs]
+        p_host = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in ps]
+    except RuntimeError as exc:
+        return {"value": None, "unit": "matrices/s", "unavailable": f"pinned allocation failed: {exc}"}
+    for gh, g in zip(g_host, gs):
+        gh.copy_(g)
+    h2d = sum(g.numel() * g.element_size() for g in gs)
+    d2h = sum(p.numel() * p.element_size() for p in ps)
+
+    def e2e_step():
+        for g, gh in zip(gs, g_host):
+            g.copy_(gh, non_blocking=True)
+        nsg.dmuon_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
+                       ns_steps=w.ns_steps, wd=w.wd, stream=stream)
+        for ph, p in zip(p_host, ps):
+            ph.copy_(p, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(max(1, args.e2e_steps)):
+        e2e_step()
+    e1.record(stream)
+    e1.synchronize()
+    wall = (time.perf_counter() - t0) / max(1, args.e2e_steps)
+    ms = reduce_max(e0.elapsed_time(e1) / max(1, args.e2e_steps), dev)
+    return {"value": round(aggregate_value(w.count, world, ms), 3), "unit": "matrices/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "wall_ms_per_step": round(wall * 1e3, 3), "steps": max(1, args.e2e_steps),
+            "api": "newton_schulz_grad_b200.dmuon_step (C ABI dmuon_step), pinned host buffers"}
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args):
+    """The fp64 oracle on the host cores: each step one sampled matrix, the
+    samples rotating through the launch classes; extrapolated to the set."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = workloads.get(args.workload)
+    samples = class_samples(w)
+    for i in range(max(args.warmup, 0)):
+        oracle_matrix_seconds(w, samples[i % len(samples)][1])
+    times = {}
+    for i in range(args.steps):
+        key, idx, cnt = samples[i % len(samples)]
+        times.setdefault(key, []).append(oracle_matrix_seconds(w, idx))
+    # classes not reached in K steps: extrapolate by flops from the measured ones
+    rate = statistics.mean(t / (3 * k[0] ** 2 * k[1] + k[0] ** 3)
+                           for k, ts in times.items() for t in ts)
+    total = 0.0
+    for key, idx, cnt in samples:
+        t = statistics.mean(times[key]) if key in times else rate * (3 * key[0] ** 2 * key[1] + key[0] ** 3)
+        total += t * cnt
+    value = w.count / total
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "matrices/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "matrices": w.count, "ns_steps": w.ns_steps},
+            "cpu_baseline": {"value": round(value, 5), "unit": "matrices/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": "each step one matrix, rotating over the launch classes; "
+                                       f"extrapolated to the {w.count}-matrix set by class counts"},
+            "e2e": {"value": round(value, 5), "unit": "matrices/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

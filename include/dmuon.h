@@ -1,0 +1,247 @@
+/*
+ * dmuon.h - C ABI of the B200 (sm_100a) Muon-step library.
+ *
+ * One Muon optimizer step over a list of 2D matrices, on one GPU:
+ *   momentum -> Nesterov input -> Frobenius normalisation -> ns_steps quintic
+ *   Gram Newton-Schulz iterations -> decoupled weight decay + shape-scaled update.
+ *
+ * The method is the per-owner step of DMuon (DMuon Training Guide, "Step 4:
+ * Create Optimizer" and its "Hyperparameter Guide" table; DMuon FAQ, "Why isn't
+ * DMuon just ZeRO-1?" - Newton-Schulz needs the whole (m, n) gradient - and
+ * "What related work should I cite?" - the default "gram" backend follows Gram
+ * Newton-Schulz).  Per matrix of shape R x C, with m = min(R,C), n = max(R,C):
+ *
+ *   buf' = mu*buf + g
+ *   x0   = g + mu*buf'  (nesterov)   |   buf'  (otherwise)
+ *   X    = orient(x0) / (||x0||_F + 1e-7)      orient = transpose when R > C
+ *   repeat ns_steps:  G = X X^T ;  X = a X + (b G + c G G) X
+ *   O    = orient^-1(X)
+ *   p'   = p (1 - lr wd) - lr * 0.2 * sqrt(n) * O
+ *
+ * Conventions common to every call:
+ *  - Pointers named "device" are CUDA device pointers owned by the caller; the
+ *    library never frees them.  Matrices are row-major and contiguous unless a
+ *    leading dimension is given.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Nothing synchronises the host except
+ *    dmuon_stream_status().
+ *  - Arguments are validated on the host before anything is launched; on an
+ *    error nothing is modified and the status says why (dmuon_get_last_error()
+ *    holds a message, per host thread).
+ *  - Device waits inside the kernels are bounded; a wait that runs out sets a
+ *    per-device status word read by dmuon_stream_status() (DMUON_ERR_TIMEOUT).
+ *  - Results do not depend on how matrices are batched: a matrix gives the
+ *    same bits alone, inside its group, or in a permuted list.
+ */
+#ifndef DMUON_H
+#define DMUON_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DMUON_API __attribute__((visibility("default")))
+#else
+#define DMUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* dmuon_stream_t;
+
+typedef enum {
+    DMUON_OK = 0,
+    DMUON_ERR_INVALID_ARG = 1, /* bad pointer, size, dtype, alignment or count */
+    DMUON_ERR_UNSUPPORTED = 2, /* no sm_100 device, or a size beyond a limit  */
+    DMUON_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed             */
+    DMUON_ERR_OOM = 4,         /* workspace allocation failed                   */
+    DMUON_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out            */
+} dmuon_status_t;
+
+typedef enum {
+    DMUON_F32 = 0,  /* fp32 storage; FFMA Newton-Schulz (fp32 X, G, p(G))            */
+    DMUON_BF16 = 1  /* bf16 storage; tcgen05 tensor-core chain with fp32 accumulation */
+} dmuon_dtype_t;
+
+/* Shape of one matrix of a Muon step. */
+typedef struct {
+    int64_t rows;
+    int64_t cols;
+    int32_t dtype;     /* dmuon_dtype_t of param, grad and momentum buffer */
+    int32_t reserved;  /* must be 0 */
+} dmuon_shape_t;
+
+/* Default quintic coefficients used when `coeffs` is NULL (the pages print
+ * none; this is the widely used Muon triple). */
+#define DMUON_DEFAULT_A 3.4445f
+#define DMUON_DEFAULT_B (-4.7750f)
+#define DMUON_DEFAULT_C 2.0315f
+#define DMUON_NORM_EPS 1e-7f
+
+/* ------------------------------------------------------------------------ */
+/* Whole-path calls                                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * dmuon_ns - orthogonalise one bf16 matrix with the Gram Newton-Schulz
+ * iteration (DMuon Training Guide, Hyperparameter Guide: ns_steps and the
+ * "gram" ns_backend rows).
+ *   X      device, rows x cols bf16, row-major contiguous (read only)
+ *   out    device, rows x cols bf16; may not overlap X
+ *   rows, cols  > 0; rows*cols < 2^31
+ *   steps  >= 0; steps == 0 gives out = X / (||X||_F + eps)
+ *   coeffs HOST array of 3*steps floats (a_k, b_k, c_k for iteration k), or
+ *          NULL for the default triple at every iteration
+ * Works over the smaller side (transposes internally when rows > cols).
+ * Uses the library's cached workspace for this (device, stream).
+ */
+DMUON_API dmuon_status_t dmuon_ns(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,
+                        const float* coeffs, dmuon_stream_t stream);
+
+/* dmuon_ns with an explicit dtype (DMUON_F32 selects the fp32 FFMA path). */
+DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,
+                           const float* coeffs, int32_t dtype, dmuon_stream_t stream);
+
+/*
+ * dmuon_step - one Muon step over `count` matrices (DMuon Training Guide,
+ * "Step 4": group 0, "momentum + NS + update").
+ *   params, grads, mom_bufs  HOST arrays of `count` DEVICE pointers; matrix i
+ *          is shapes[i].rows x shapes[i].cols, row-major contiguous, in
+ *          shapes[i].dtype.  params and mom_bufs are updated in place; grads
+ *          are read only.  No two matrices may overlap.
+ *   shapes HOST array of `count` shapes (reserved fields 0)
+ *   count  >= 0 (0 is a no-op)
+ *   lr     Muon learning rate; the update uses lr * 0.2 * sqrt(max(R, C))
+ *          (Hyperparameter Guide, lr row), the decay uses lr
+ *   momentum  mu (default 0.95 on the pages); nesterov 0/1 (default 1)
+ *   ns_steps  >= 0 (default 5); coeffs as for dmuon_ns
+ *   wd     decoupled weight decay: p <- p (1 - lr wd) - ...
+ * Matrices are grouped by shape (dmuon_plan_groups) and each group runs as
+ * batched launches.
+ */
+DMUON_API dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
+                          const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
+                          int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
+                          dmuon_stream_t stream);
+
+/*
+ * dmuon_plan_groups - the shape grouping dmuon_step uses (host only, no GPU).
+ * Matrices with equal (rows, cols, dtype) form a group; group ids follow
+ * first appearance; `order` lists the groups one after another, members in
+ * ascending index.
+ *   shapes    HOST array of `count` shapes
+ *   group_of  HOST out, `count` ints (group id of matrix i)
+ *   order     HOST out, `count` ints (execution order)
+ *   num_groups HOST out, 1 int
+ */
+DMUON_API dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int32_t* group_of,
+                                 int32_t* order, int32_t* num_groups);
+
+/* ------------------------------------------------------------------------ */
+/* Stage calls: the individual kernels of the path, over `batch` matrices    */
+/* stored one after another (matrix b starts at b * rows * ld elements).     */
+/* dtype DMUON_BF16 runs the tcgen05 tensor-core kernels (bf16 in and out,   */
+/* fp32 accumulation; ld a multiple of 8, pointers 16-byte aligned);         */
+/* DMUON_F32 runs the FFMA kernels (fp32 in and out).                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * dmuon_gram - G = alpha * X X^T (the Gram matrix of one Gram Newton-Schulz
+ * iteration, over the smaller side).  Only one triangle is computed; the
+ * other is written as its mirror, so G is exactly symmetric.
+ *   X  device, batch x m x n (leading dimension ldx >= n)
+ *   G  device, batch x m x m (leading dimension ldg >= m); may not overlap X
+ */
+DMUON_API dmuon_status_t dmuon_gram(const void* X, void* G, int64_t batch, int64_t m, int64_t n,
+                          int64_t ldx, int64_t ldg, float alpha, int32_t dtype,
+                          dmuon_stream_t stream);
+
+/*
+ * dmuon_gram_poly - P = b G + c G G for a symmetric G (so that
+ * p(G) = a I + P).  One triangle computed, the other mirrored.
+ *   G  device, batch x m x m (ldg); P device, batch x m x m (ldp), no overlap
+ */
+DMUON_API dmuon_status_t dmuon_gram_poly(const void* G, void* P, int64_t batch, int64_t m, int64_t ldg,
+                               int64_t ldp, float b, float c, int32_t dtype,
+                               dmuon_stream_t stream);
+
+/*
+ * dmuon_poly_apply - Y = alpha * (a X + P X)  ( = alpha * p(G) X ).
+ *   P  device, batch x m x m (ldp);  X device, batch x m x n (ldx)
+ *   Y  device, batch x m x n (ldy); may not overlap X or P
+ */
+DMUON_API dmuon_status_t dmuon_poly_apply(const void* P, const void* X, void* Y, int64_t batch, int64_t m,
+                                int64_t n, int64_t ldp, int64_t ldx, int64_t ldy, float a,
+                                float alpha, int32_t dtype, dmuon_stream_t stream);
+
+/*
+ * dmuon_momentum - the momentum stage for one matrix, in place on `buf`:
+ *   buf' = mu*buf + g ;  x0 = g + mu*buf' (nesterov) or buf'
+ * in fp32 with each operation rounded (no fused multiply-add), stored in
+ * `dtype` (bf16 round-to-nearest-even).  x0 uses the unrounded fp32 buf'.
+ *   buf, grad, x0  device, rows x cols, row-major contiguous
+ *   sumsq  device, 1 double, or NULL: receives sum of squares of stored x0
+ */
+DMUON_API dmuon_status_t dmuon_momentum(void* buf, const void* grad, void* x0, int64_t rows, int64_t cols,
+                              float momentum, int32_t nesterov, int32_t dtype, double* sumsq,
+                              dmuon_stream_t stream);
+
+/*
+ * dmuon_update - the update stage for one matrix, in place on `param`:
+ *   p' = fl(p * fl(1 - lr*wd)) - fl(s * O),  s = fl32(lr * 0.2 * sqrt(max(rows,cols)))
+ *   param, O  device, rows x cols in dtype, row-major contiguous
+ */
+DMUON_API dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, int64_t cols, float lr,
+                            float wd, int32_t dtype, dmuon_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Status, workspace, build information                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Message for the last non-OK status returned on this host thread. */
+DMUON_API const char* dmuon_get_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: DMUON_ERR_TIMEOUT if a device-side wait ran out since the
+ * last call, DMUON_ERR_CUDA if the stream reports an error, else DMUON_OK. */
+DMUON_API dmuon_status_t dmuon_stream_status(dmuon_stream_t stream);
+
+/* Frees every cached workspace of the calling thread's current device after
+ * synchronising the device.  Safe to call at any time between calls. */
+DMUON_API void dmuon_release_workspace(void);
+
+/* Bytes of workspace dmuon_step would use for these shapes (host only). */
+DMUON_API int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps);
+
+/* Number of kernels dmuon_step launches for these shapes (host only). */
+DMUON_API int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps);
+
+/*
+ * Per-kernel timing.  Between dmuon_profile_start() and dmuon_profile_stop()
+ * every kernel that the calling host thread's calls enqueue is bracketed by
+ * two CUDA events on its stream.  dmuon_profile_stop() waits for the last
+ * event, then fills up to max_stats entries (one per kernel kind) and returns
+ * how many kinds were seen (or -1 on a CUDA error).  "flops" and "bytes" are
+ * the algorithmic work of the launches: gram m^2 n, poly m^3, apply 2 m^2 n
+ * flops per matrix; momentum 4, update 3 element accesses per element.
+ */
+typedef struct {
+    char name[32];
+    int64_t launches;
+    double total_ms;
+    double flops;
+    double bytes;
+} dmuon_kernel_stat_t;
+
+DMUON_API dmuon_status_t dmuon_profile_start(void);
+DMUON_API int32_t dmuon_profile_stop(dmuon_kernel_stat_t* stats, int32_t max_stats);
+
+/* Static string: version, target architecture, tile configuration. */
+DMUON_API const char* dmuon_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DMUON_H */

@@ -1,0 +1,339 @@
+"""Python binding of the B200 Muon-step library (``libdmuon_b200.so``).
+
+Argument marshalling only: every function below takes torch tensors (for
+device memory) and an optional CUDA stream, turns them into the plain
+pointers and sizes of the C ABI declared in ``include/dmuon.h`` and calls the
+function of the same name.  All computation happens in the library's CUDA
+kernels; there is no CPU or PyTorch fallback.  If the shared library is
+missing this module raises on import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdmuon_b200.so")
+
+DMUON_OK = 0
+DMUON_ERR_INVALID_ARG = 1
+DMUON_ERR_UNSUPPORTED = 2
+DMUON_ERR_CUDA = 3
+DMUON_ERR_OOM = 4
+DMUON_ERR_TIMEOUT = 5
+STATUS_NAMES = {0: "DMUON_OK", 1: "DMUON_ERR_INVALID_ARG", 2: "DMUON_ERR_UNSUPPORTED",
+                3: "DMUON_ERR_CUDA", 4: "DMUON_ERR_OOM", 5: "DMUON_ERR_TIMEOUT"}
+DMUON_F32 = 0
+DMUON_BF16 = 1
+DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
+
+EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon_gram",
+            "dmuon_gram_poly", "dmuon_poly_apply", "dmuon_momentum", "dmuon_update",
+            "dmuon_get_last_error", "dmuon_stream_status", "dmuon_release_workspace",
+            "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
+            "dmuon_profile_start", "dmuon_profile_stop")
+
+
+class DmuonError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python newton_schulz_grad_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+    fp = ctypes.POINTER(ctypes.c_float)
+    sig = {
+        "dmuon_ns": ([vp, vp, i64, i64, i32, fp, vp], i32),
+        "dmuon_ns_ex": ([vp, vp, i64, i64, i32, fp, i32, vp], i32),
+        "dmuon_step": ([ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                        ctypes.POINTER(Shape), i32, f32, f32, i32, i32, fp, f32, vp], i32),
+        "dmuon_plan_groups": ([ctypes.POINTER(Shape), i32, ctypes.POINTER(i32),
+                               ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
+        "dmuon_gram": ([vp, vp, i64, i64, i64, i64, i64, f32, i32, vp], i32),
+        "dmuon_gram_poly": ([vp, vp, i64, i64, i64, i64, f32, f32, i32, vp], i32),
+        "dmuon_poly_apply": ([vp, vp, vp, i64, i64, i64, i64, i64, i64, f32, f32, i32, vp], i32),
+        "dmuon_momentum": ([vp, vp, vp, i64, i64, f32, i32, i32, vp, vp], i32),
+        "dmuon_update": ([vp, vp, i64, i64, f32, f32, i32, vp], i32),
+        "dmuon_get_last_error": ([], ctypes.c_char_p),
+        "dmuon_stream_status": ([vp], i32),
+        "dmuon_release_workspace": ([], None),
+        "dmuon_workspace_bytes": ([ctypes.POINTER(Shape), i32, i32], i64),
+        "dmuon_step_launches": ([ctypes.POINTER(Shape), i32, i32], i64),
+        "dmuon_build_info": ([], ctypes.c_char_p),
+        "dmuon_profile_start": ([], i32),
+        "dmuon_profile_stop": ([ctypes.POINTER(KernelStat), i32], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+# ------------------------------------------------------------------ helpers
+def _check(status: int) -> None:
+    if status != DMUON_OK:
+        raise DmuonError(status, _lib.dmuon_get_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DMUON_BF16
+    if t.dtype == torch.float32:
+        return DMUON_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+
+
+def _coeffs(steps: int, coeffs):
+    """None -> NULL (library default); one triple -> repeated; else 3*steps floats."""
+    if coeffs is None or steps == 0:
+        return None
+    flat = [float(v) for trip in (coeffs if isinstance(coeffs[0], (tuple, list)) else [coeffs])
+            for v in trip]
+    if len(flat) == 3 and steps != 1:
+        flat = flat * steps
+    if len(flat) != 3 * steps:
+        raise ValueError("coeffs must hold one triple or one triple per step")
+    arr = (ctypes.c_float * max(1, len(flat)))(*flat)
+    return arr
+
+
+def _shape_array(shapes: Sequence[Tuple[int, int, int]]):
+    arr = (Shape * max(1, len(shapes)))()
+    for i, (r, c, d) in enumerate(shapes):
+        arr[i].rows, arr[i].cols, arr[i].dtype, arr[i].reserved = int(r), int(c), int(d), 0
+    return arr
+
+
+def _rows_ld(t: torch.Tensor):
+    """(batch, rows, cols, ld) of a 2D or 3D tensor with unit column stride."""
+    if t.dim() == 2:
+        t3 = t.unsqueeze(0)
+    elif t.dim() == 3:
+        t3 = t
+    else:
+        raise ValueError("expected a 2D or 3D tensor")
+    b, r, c = t3.shape
+    if t3.stride(2) != 1:
+        raise ValueError("last dimension must be contiguous")
+    ld = t3.stride(1)
+    if b > 1 and t3.stride(0) != r * ld:
+        raise ValueError("matrices of a batch must follow one another (stride rows*ld)")
+    return b, r, c, ld
+
+
+# ------------------------------------------------------------- whole path
+def dmuon_ns(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=None, stream=None) -> None:
+    """out = Gram Newton-Schulz(X / (||X|| + eps)); bf16 or fp32 (``dmuon_ns_ex``)."""
+    _need_cuda(X, out)
+    if X.shape != out.shape or X.dim() != 2 or X.dtype != out.dtype:
+        raise ValueError("X and out must be 2D tensors of equal shape and dtype")
+    if not (X.is_contiguous() and out.is_contiguous()):
+        raise ValueError("X and out must be contiguous")
+    c = _coeffs(steps, coeffs)
+    _check(_lib.dmuon_ns_ex(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps, c,
+                            _dtype_code(X), _stream(stream)))
+
+
+def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+               mom_bufs: Sequence[torch.Tensor], lr: float = 0.02, momentum: float = 0.95,
+               nesterov: bool = True, ns_steps: int = 5, coeffs=None, wd: float = 0.0,
+               stream=None) -> None:
+    """One Muon step over lists of 2D tensors; params and mom_bufs updated in place."""
+    n = len(params)
+    if len(grads) != n or len(mom_bufs) != n:
+        raise ValueError("params, grads and mom_bufs must have the same length")
+    shapes = []
+    for p, g, b in zip(params, grads, mom_bufs):
+        _need_cuda(p, g, b)
+        if p.dim() != 2 or p.shape != g.shape or p.shape != b.shape:
+            raise ValueError("each param, grad and buffer must be 2D with one shape")
+        if not (p.dtype == g.dtype == b.dtype):
+            raise ValueError("param, grad and buffer must share a dtype")
+        if not (p.is_contiguous() and g.is_contiguous() and b.is_contiguous()):
+            raise ValueError("tensors must be contiguous")
+        shapes.append((p.shape[0], p.shape[1], _dtype_code(p)))
+    vp = ctypes.c_void_p
+    pa = (vp * max(1, n))(*[t.data_ptr() for t in params])
+    ga = (vp * max(1, n))(*[t.data_ptr() for t in grads])
+    ba = (vp * max(1, n))(*[t.data_ptr() for t in mom_bufs])
+    c = _coeffs(ns_steps, coeffs)
+    _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
+                           ns_steps, c, wd, _stream(stream)))
+
+
+def dmuon_step_ptrs(params: Sequence[int], grads: Sequence[int], mom_bufs: Sequence[int],
+                    shapes: Sequence[Tuple[int, int, int]], lr: float = 0.02,
+                    momentum: float = 0.95, nesterov: bool = True, ns_steps: int = 5,
+                    coeffs=None, wd: float = 0.0, stream=None) -> None:
+    """dmuon_step on raw device addresses (no per-tensor checks on the Python side)."""
+    n = len(params)
+    vp = ctypes.c_void_p
+    pa = (vp * max(1, n))(*params)
+    ga = (vp * max(1, n))(*grads)
+    ba = (vp * max(1, n))(*mom_bufs)
+    _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
+                           ns_steps, _coeffs(ns_steps, coeffs), wd, _stream(stream)))
+
+
+def dmuon_plan_groups(shapes: Sequence[Tuple[int, int, int]]):
+    """(group_of, order, num_groups) for (rows, cols, dtype_code) shapes (host only)."""
+    n = len(shapes)
+    g = (ctypes.c_int32 * max(1, n))()
+    o = (ctypes.c_int32 * max(1, n))()
+    k = ctypes.c_int32(0)
+    _check(_lib.dmuon_plan_groups(_shape_array(shapes), n, g, o, ctypes.byref(k)))
+    return list(g)[:n], list(o)[:n], k.value
+
+
+def dmuon_workspace_bytes(shapes, ns_steps: int = 5) -> int:
+    return int(_lib.dmuon_workspace_bytes(_shape_array(shapes), len(shapes), ns_steps))
+
+
+def dmuon_step_launches(shapes, ns_steps: int = 5) -> int:
+    return int(_lib.dmuon_step_launches(_shape_array(shapes), len(shapes), ns_steps))
+
+
+# ------------------------------------------------------------- stage calls
+def dmuon_gram(X: torch.Tensor, G: torch.Tensor, alpha: float = 1.0, stream=None) -> None:
+    """G = alpha X X^T over a batch ([B,] m x n -> [B,] m x m)."""
+    _need_cuda(X, G)
+    b, m, n, ldx = _rows_ld(X)
+    b2, m2, m3, ldg = _rows_ld(G)
+    if (b2, m2, m3) != (b, m, m) or X.dtype != G.dtype:
+        raise ValueError("G must be [B,] m x m with X's dtype")
+    _check(_lib.dmuon_gram(_ptr(X), _ptr(G), b, m, n, ldx, ldg, alpha, _dtype_code(X),
+                           _stream(stream)))
+
+
+def dmuon_gram_poly(G: torch.Tensor, P: torch.Tensor, b: float, c: float, stream=None) -> None:
+    """P = b G + c G G for symmetric G ([B,] m x m)."""
+    _need_cuda(G, P)
+    bb, m, m2, ldg = _rows_ld(G)
+    b2, p1, p2, ldp = _rows_ld(P)
+    if m != m2 or (b2, p1, p2) != (bb, m, m) or G.dtype != P.dtype:
+        raise ValueError("G and P must be [B,] m x m of one dtype")
+    _check(_lib.dmuon_gram_poly(_ptr(G), _ptr(P), bb, m, ldg, ldp, b, c, _dtype_code(G),
+                                _stream(stream)))
+
+
+def dmuon_poly_apply(P: torch.Tensor, X: torch.Tensor, Y: torch.Tensor, a: float,
+                     alpha: float = 1.0, stream=None) -> None:
+    """Y = alpha (a X + P X) ([B,] m x m, [B,] m x n -> [B,] m x n)."""
+    _need_cuda(P, X, Y)
+    bp, m, m2, ldp = _rows_ld(P)
+    bx, mx, n, ldx = _rows_ld(X)
+    by, my, ny, ldy = _rows_ld(Y)
+    if not (bp == bx == by and m == m2 == mx == my and n == ny) or not (P.dtype == X.dtype == Y.dtype):
+        raise ValueError("shape or dtype mismatch")
+    _check(_lib.dmuon_poly_apply(_ptr(P), _ptr(X), _ptr(Y), bx, m, n, ldp, ldx, ldy, a, alpha,
+                                 _dtype_code(X), _stream(stream)))
+
+
+def dmuon_momentum(buf: torch.Tensor, grad: torch.Tensor, x0: torch.Tensor, momentum: float = 0.95,
+                   nesterov: bool = True, sumsq: Optional[torch.Tensor] = None, stream=None) -> None:
+    """buf <- mu buf + g ; x0 = g + mu buf (or buf); optional fp64 sum of squares of x0."""
+    _need_cuda(buf, grad, x0)
+    if not (buf.shape == grad.shape == x0.shape) or buf.dim() != 2:
+        raise ValueError("buf, grad and x0 must be 2D of one shape")
+    if sumsq is not None and (sumsq.dtype != torch.float64 or not sumsq.is_cuda):
+        raise ValueError("sumsq must be a CUDA float64 tensor")
+    _check(_lib.dmuon_momentum(_ptr(buf), _ptr(grad), _ptr(x0), buf.shape[0], buf.shape[1],
+                               momentum, int(bool(nesterov)), _dtype_code(buf), _ptr(sumsq),
+                               _stream(stream)))
+
+
+def dmuon_update(param: torch.Tensor, O: torch.Tensor, lr: float, wd: float = 0.0,
+                 stream=None) -> None:
+    """param <- param (1 - lr wd) - lr 0.2 sqrt(max(m,n)) O."""
+    _need_cuda(param, O)
+    if param.shape != O.shape or param.dim() != 2 or param.dtype != O.dtype:
+        raise ValueError("param and O must be 2D of one shape and dtype")
+    _check(_lib.dmuon_update(_ptr(param), _ptr(O), param.shape[0], param.shape[1], lr, wd,
+                             _dtype_code(param), _stream(stream)))
+
+
+# ---------------------------------------------------------- status / misc
+def dmuon_stream_status(stream=None) -> int:
+    """Synchronise the stream and return (without raising) the library status."""
+    return int(_lib.dmuon_stream_status(_stream(stream)))
+
+
+def dmuon_get_last_error() -> str:
+    return _lib.dmuon_get_last_error().decode()
+
+
+def dmuon_release_workspace() -> None:
+    _lib.dmuon_release_workspace()
+
+
+def dmuon_profile_start() -> None:
+    _check(_lib.dmuon_profile_start())
+
+
+def dmuon_profile_stop() -> dict:
+    """{kind: {launches, total_ms, flops, bytes}} for the launches since start."""
+    arr = (KernelStat * 32)()
+    n = _lib.dmuon_profile_stop(arr, 32)
+    if n < 0:
+        raise DmuonError(DMUON_ERR_CUDA, dmuon_get_last_error())
+    return {arr[i].name.decode(): {"launches": int(arr[i].launches), "total_ms": arr[i].total_ms,
+                                   "flops": arr[i].flops, "bytes": arr[i].bytes}
+            for i in range(min(n, 32))}
+
+
+def dmuon_build_info() -> str:
+    return _lib.dmuon_build_info().decode()
+
+
+def coeff_list(steps: int, coeffs=None) -> List[Tuple[float, float, float]]:
+    """The per-iteration coefficient triples the library will use."""
+    if coeffs is None:
+        return [DEFAULT_COEFFS] * steps
+    if not isinstance(coeffs[0], (tuple, list)):
+        return [tuple(coeffs)] * steps
+    return [tuple(c) for c in coeffs]

@@ -1,0 +1,658 @@
+// C ABI of the Muon-step library: argument validation, device state,
+// workspace cache and the orchestration of one step.
+//
+// dmuon_step (DMuon Training Guide, "Step 4": momentum + NS + update for the
+// dedicated parameters) runs, per launch class (same oriented shape and
+// dtype) and per chunk of at most 256 matrices that fits the workspace cap:
+//   momentum+norm partials -> norm finalise -> ns_steps x (gram, poly, apply)
+//   -> update
+// all enqueued on the caller's stream with no host synchronisation.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "internal.h"
+
+namespace dmuon {
+namespace {
+
+thread_local std::string g_last_error;
+
+dmuon_status_t fail(dmuon_status_t s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+dmuon_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(DMUON_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+struct DeviceState {
+  int sm_count = 0;
+  int major = 0, minor = 0;
+  int* status_word = nullptr;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceState> g_devices;
+std::map<std::pair<int, uintptr_t>, std::pair<void*, size_t>> g_workspace;
+
+dmuon_status_t device_state(DeviceState* out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_devices.find(dev);
+  if (it == g_devices.end()) {
+    DeviceState ds;
+    e = cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ds.major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ds.minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    if (ds.major != 10)
+      return fail(DMUON_ERR_UNSUPPORTED, "device is sm_" + std::to_string(ds.major) +
+                                             std::to_string(ds.minor) + "; this library is built for sm_100a");
+    e = cudaMalloc(&ds.status_word, sizeof(int));
+    if (e != cudaSuccess) return fail(DMUON_ERR_OOM, "status word allocation failed");
+    e = cudaMemset(ds.status_word, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset");
+    it = g_devices.emplace(dev, ds).first;
+  }
+  *out = it->second;
+  return DMUON_OK;
+}
+
+bool fault_injected(const char* what) {
+  const char* e = std::getenv("DMUON_FAULT_INJECT");
+  return e && std::strcmp(e, what) == 0;
+}
+
+// Stream-ordered, grow-only workspace per (device, stream).
+dmuon_status_t get_workspace(size_t bytes, cudaStream_t st, void** out) {
+  if (fault_injected("alloc")) return fail(DMUON_ERR_OOM, "workspace allocation failed (injected)");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto key = std::make_pair(dev, reinterpret_cast<uintptr_t>(st));
+  auto& slot = g_workspace[key];
+  if (slot.first && slot.second >= bytes) {
+    *out = slot.first;
+    return DMUON_OK;
+  }
+  if (slot.first) {
+    cudaFreeAsync(slot.first, st);
+    slot = {nullptr, 0};
+  }
+  void* p = nullptr;
+  e = cudaMallocAsync(&p, bytes, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(DMUON_ERR_OOM, "workspace allocation of " + std::to_string(bytes) + " bytes failed: " +
+                                   cudaGetErrorString(e));
+  }
+  slot = {p, bytes};
+  *out = p;
+  return DMUON_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t esize(int32_t dtype) { return dtype == DMUON_BF16 ? 2 : 4; }
+bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
+
+// ------------------------------------------------------------ kernel timing
+enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
+            kLoad, kCopyOut, kNumKinds };
+const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
+                                           "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
+                                           "copy_out"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+thread_local bool g_prof_on = false;
+thread_local std::vector<ProfRec> g_prof;
+
+// Brackets one kernel launch with events when profiling is on.
+struct Prof {
+  bool on;
+  ProfRec r;
+  Prof(int kind, cudaStream_t st, double flops, double bytes) : on(g_prof_on) {
+    if (!on) return;
+    r = ProfRec{kind, nullptr, nullptr, flops, bytes};
+    if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
+      on = false;
+      return;
+    }
+    cudaEventRecord(r.a, st);
+  }
+  void done(cudaStream_t st) {
+    if (!on) return;
+    cudaEventRecord(r.b, st);
+    g_prof.push_back(r);
+    on = false;
+  }
+};
+
+constexpr int64_t kMaxSide = int64_t(1) << 20;
+constexpr int64_t kMaxElems = (int64_t(1) << 31) - 1;
+
+dmuon_status_t check_shape(int64_t rows, int64_t cols, const char* what) {
+  if (rows <= 0 || cols <= 0 || rows > kMaxSide || cols > kMaxSide || rows * cols > kMaxElems)
+    return fail(DMUON_ERR_INVALID_ARG, std::string(what) + ": shape " + std::to_string(rows) + "x" +
+                                           std::to_string(cols) + " out of range (sides 1..2^20, < 2^31 elements)");
+  return DMUON_OK;
+}
+
+dmuon_status_t coeff_schedule(int32_t steps, const float* coeffs, std::vector<float>& out) {
+  out.resize(3 * (size_t)steps);
+  for (int32_t k = 0; k < steps; ++k) {
+    if (coeffs) {
+      out[3 * k] = coeffs[3 * k];
+      out[3 * k + 1] = coeffs[3 * k + 1];
+      out[3 * k + 2] = coeffs[3 * k + 2];
+    } else {
+      out[3 * k] = DMUON_DEFAULT_A;
+      out[3 * k + 1] = DMUON_DEFAULT_B;
+      out[3 * k + 2] = DMUON_DEFAULT_C;
+    }
+  }
+  return DMUON_OK;
+}
+
+struct Interval {
+  uintptr_t lo, hi;
+  int who;
+};
+
+// True if any two intervals overlap.
+bool any_overlap(std::vector<Interval>& v) {
+  std::sort(v.begin(), v.end(), [](const Interval& a, const Interval& b) { return a.lo < b.lo; });
+  for (size_t i = 1; i < v.size(); ++i)
+    if (v[i].lo < v[i - 1].hi) return true;
+  return false;
+}
+
+// The Newton-Schulz chain over a chunk of `b` oriented m x n matrices in the
+// workspace; returns the buffer that holds the result.
+dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char* ws,
+                         const ChunkOffsets& off, int32_t steps, const std::vector<float>& sched,
+                         const DeviceState& ds, cudaStream_t st, void** result) {
+  void* cur = ws + off.x0;
+  void* nxt = ws + off.x1;
+  void* G = ws + off.g;
+  void* P = ws + off.p;
+  const float* scale = reinterpret_cast<const float*>(ws + off.scale);
+  const bool tc = L.path == Path::kTensorBf16;
+  const bool xbf16 = L.path == Path::kSmallBf16;
+  const double fm = (double)m, fn = (double)n, fb = (double)b;
+  for (int32_t k = 0; k < steps; ++k) {
+    const float a = sched[3 * k], bb = sched[3 * k + 1], c = sched[3 * k + 2];
+    const float* sc = k == 0 ? scale : nullptr;
+    cudaError_t e;
+    {
+      Prof p(tc ? kGramTc : kGramFfma, st, fb * fm * fm * fn, 0.0);
+      e = tc ? tc_gram(cur, G, b, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, ds.status_word, ds.sm_count, st)
+             : simt_gram(cur, G, b, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, xbf16, st);
+      p.done(st);
+    }
+    if (e == cudaSuccess) {
+      Prof p(tc ? kPolyTc : kPolyFfma, st, fb * fm * fm * fm, 0.0);
+      e = tc ? tc_poly(G, P, b, (int)m, L.ldm, L.ldm, bb, c, ds.status_word, ds.sm_count, st)
+             : simt_poly(G, P, b, (int)m, L.ldm, L.ldm, bb, c, st);
+      p.done(st);
+    }
+    if (e == cudaSuccess) {
+      Prof p(tc ? kApplyTc : kApplyFfma, st, 2.0 * fb * fm * fm * fn, 0.0);
+      e = tc ? tc_apply(P, cur, nxt, b, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, ds.status_word,
+                        ds.sm_count, st)
+             : simt_apply(P, cur, nxt, b, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st);
+      p.done(st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
+    std::swap(cur, nxt);
+  }
+  *result = cur;
+  return DMUON_OK;
+}
+
+int64_t chunk_launches(int32_t steps) { return 3 + 3 * (int64_t)steps; }
+
+}  // namespace
+}  // namespace dmuon
+
+using namespace dmuon;
+
+extern "C" {
+
+const char* dmuon_get_last_error(void) { return g_last_error.c_str(); }
+
+const char* dmuon_build_info(void) {
+  static std::string s = std::string("dmuon-b200 0.1.0; sm_100a; ") + tc_config_string() +
+                         "; FFMA chain for fp32 and min side <= 64; elementwise 64x64 tiles";
+  return s.c_str();
+}
+
+dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int32_t* group_of,
+                                 int32_t* order, int32_t* num_groups) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
+  if (!num_groups || (count > 0 && (!shapes || !group_of || !order)))
+    return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  std::vector<Group> groups = plan_groups(shapes, count);
+  int32_t pos = 0;
+  for (size_t g = 0; g < groups.size(); ++g)
+    for (int32_t i : groups[g].members) {
+      group_of[i] = (int32_t)g;
+      order[pos++] = i;
+    }
+  *num_groups = (int32_t)groups.size();
+  return DMUON_OK;
+}
+
+int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
+  (void)ns_steps;
+  if (count <= 0 || !shapes) return 0;
+  int64_t best = 0;
+  for (const LaunchClass& c : plan_classes(plan_groups(shapes, count))) {
+    ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
+    best = std::max(best, chunk_offsets(L, chunk_size(L, (int64_t)c.members.size())).total);
+  }
+  return best;
+}
+
+int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
+  if (count <= 0 || !shapes) return 0;
+  int64_t n = 0;
+  for (const LaunchClass& c : plan_classes(plan_groups(shapes, count))) {
+    ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
+    const int64_t cs = chunk_size(L, (int64_t)c.members.size());
+    const int64_t chunks = ((int64_t)c.members.size() + cs - 1) / cs;
+    n += chunks * chunk_launches(ns_steps);
+  }
+  return n;
+}
+
+dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
+                          const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
+                          int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
+                          dmuon_stream_t stream) {
+  // ---------------------------------------------------------- validation
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
+  if (ns_steps < 0 || ns_steps > 1000) return fail(DMUON_ERR_INVALID_ARG, "ns_steps must be in 0..1000");
+  if (nesterov != 0 && nesterov != 1) return fail(DMUON_ERR_INVALID_ARG, "nesterov must be 0 or 1");
+  if (!std::isfinite(lr) || !std::isfinite(momentum) || !std::isfinite(wd))
+    return fail(DMUON_ERR_INVALID_ARG, "lr, momentum and wd must be finite");
+  if (count == 0) return DMUON_OK;
+  if (!params || !grads || !mom_bufs || !shapes) return fail(DMUON_ERR_INVALID_ARG, "null array argument");
+  std::vector<Interval> iv;
+  iv.reserve(3 * (size_t)count);
+  for (int32_t i = 0; i < count; ++i) {
+    const dmuon_shape_t& s = shapes[i];
+    dmuon_status_t st = check_shape(s.rows, s.cols, "dmuon_step");
+    if (st != DMUON_OK) return st;
+    if (!dtype_ok(s.dtype)) return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": bad dtype");
+    if (s.reserved != 0) return fail(DMUON_ERR_INVALID_ARG, "reserved shape field must be 0");
+    if (!params[i] || !grads[i] || !mom_bufs[i])
+      return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": null pointer");
+    const uintptr_t bytes = (uintptr_t)(s.rows * s.cols) * esize(s.dtype);
+    iv.push_back({(uintptr_t)params[i], (uintptr_t)params[i] + bytes, i});
+    iv.push_back({(uintptr_t)grads[i], (uintptr_t)grads[i] + bytes, i});
+    iv.push_back({(uintptr_t)mom_bufs[i], (uintptr_t)mom_bufs[i] + bytes, i});
+  }
+  if (any_overlap(iv)) return fail(DMUON_ERR_INVALID_ARG, "params, grads and momentum buffers must not overlap");
+  std::vector<float> sched;
+  coeff_schedule(ns_steps, coeffs, sched);
+
+  // ------------------------------------------------------------- planning
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceState ds;
+  dmuon_status_t rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  std::vector<LaunchClass> classes = plan_classes(plan_groups(shapes, count));
+  int64_t ws_bytes = 0;
+  for (const LaunchClass& c : classes) {
+    ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
+    ws_bytes = std::max(ws_bytes, chunk_offsets(L, chunk_size(L, (int64_t)c.members.size())).total);
+  }
+  void* wsv = nullptr;
+  rc = get_workspace((size_t)ws_bytes, st, &wsv);
+  if (rc != DMUON_OK) return rc;
+  char* ws = static_cast<char*>(wsv);
+  std::unique_ptr<ElemTable> tab(new ElemTable());
+
+  // ------------------------------------------------------------ execution
+  for (const LaunchClass& c : classes) {
+    const ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
+    const int64_t cs = chunk_size(L, (int64_t)c.members.size());
+    const size_t es = esize(c.dtype);
+    for (size_t start = 0; start < c.members.size(); start += (size_t)cs) {
+      const int b = (int)std::min<int64_t>(cs, (int64_t)(c.members.size() - start));
+      const ChunkOffsets off = chunk_offsets(L, b);
+      tab->m = c.m;
+      tab->n = c.n;
+      tab->ldn = L.ldn;
+      tab->count = b;
+      tab->tiles_per_mat = (int32_t)L.tiles_per_mat;
+      for (int j = 0; j < b; ++j) {
+        const int32_t i = c.members[start + j];
+        MatEntry& e = tab->e[j];
+        e.src = grads[i];
+        e.buf = mom_bufs[i];
+        e.dst = params[i];
+        e.transposed = shapes[i].rows > shapes[i].cols ? 1 : 0;
+        const bool row16 = ((int64_t)shapes[i].cols * (int64_t)es) % 16 == 0;
+        e.pad = ((row16 && aligned16(grads[i]) && aligned16(mom_bufs[i])) ? 1 : 0) |
+                ((row16 && aligned16(params[i])) ? 2 : 0);
+      }
+      float* partials = reinterpret_cast<float*>(ws + off.partials);
+      float* scale = reinterpret_cast<float*>(ws + off.scale);
+      const double elems = (double)b * (double)c.m * (double)c.n;
+      Prof pm(kMomentum, st, 0.0, 4.0 * elems * (double)es);
+      cudaError_t e = launch_momentum(*tab, c.dtype, ElemMode::kMomentum, ws + off.x0, partials, momentum,
+                                      nesterov, st);
+      pm.done(st);
+      if (e != cudaSuccess) return cuda_fail(e, "momentum launch");
+      Prof pn(kNorm, st, 0.0, 4.0 * (double)b * (double)L.tiles_per_mat);
+      e = launch_norm_finalize(partials, b, (int)L.tiles_per_mat, scale, nullptr, st);
+      pn.done(st);
+      if (e != cudaSuccess) return cuda_fail(e, "norm launch");
+      void* result = nullptr;
+      rc = run_chain(L, b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &result);
+      if (rc != DMUON_OK) return rc;
+      Prof pu(kUpdate, st, 0.0, 3.0 * elems * (double)es);
+      e = launch_update(*tab, c.dtype, ElemMode::kUpdate, result, ns_steps == 0 ? scale : nullptr, lr, wd,
+                        c.n, st);
+      pu.done(st);
+      if (e != cudaSuccess) return cuda_fail(e, "update launch");
+    }
+  }
+  return DMUON_OK;
+}
+
+dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,
+                           const float* coeffs, int32_t dtype, dmuon_stream_t stream) {
+  if (!X || !out) return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  dmuon_status_t rc = check_shape(rows, cols, "dmuon_ns");
+  if (rc != DMUON_OK) return rc;
+  if (!dtype_ok(dtype)) return fail(DMUON_ERR_INVALID_ARG, "bad dtype");
+  if (steps < 0 || steps > 1000) return fail(DMUON_ERR_INVALID_ARG, "steps must be in 0..1000");
+  const uintptr_t bytes = (uintptr_t)(rows * cols) * esize(dtype);
+  const uintptr_t x = (uintptr_t)X, o = (uintptr_t)out;
+  if (x < o + bytes && o < x + bytes) return fail(DMUON_ERR_INVALID_ARG, "out may not overlap X");
+  std::vector<float> sched;
+  coeff_schedule(steps, coeffs, sched);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  const int64_t m = std::min(rows, cols), n = std::max(rows, cols);
+  const ChunkLayout L = chunk_layout(m, n, dtype);
+  const ChunkOffsets off = chunk_offsets(L, 1);
+  void* wsv = nullptr;
+  rc = get_workspace((size_t)off.total, st, &wsv);
+  if (rc != DMUON_OK) return rc;
+  char* ws = static_cast<char*>(wsv);
+  std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->m = m;
+  tab->n = n;
+  tab->ldn = L.ldn;
+  tab->count = 1;
+  tab->tiles_per_mat = (int32_t)L.tiles_per_mat;
+  MatEntry& e0 = tab->e[0];
+  e0.src = X;
+  e0.buf = nullptr;
+  e0.dst = out;
+  e0.transposed = rows > cols ? 1 : 0;
+  const bool row16 = (cols * (int64_t)esize(dtype)) % 16 == 0;
+  e0.pad = ((row16 && aligned16(X)) ? 1 : 0) | ((row16 && aligned16(out)) ? 2 : 0);
+  float* partials = reinterpret_cast<float*>(ws + off.partials);
+  float* scale = reinterpret_cast<float*>(ws + off.scale);
+  const double elems = (double)m * (double)n, es = (double)esize(dtype);
+  Prof pl(kLoad, st, 0.0, 2.0 * elems * es);
+  cudaError_t e = launch_momentum(*tab, dtype, ElemMode::kLoad, ws + off.x0, partials, 0.f, 0, st);
+  pl.done(st);
+  if (e != cudaSuccess) return cuda_fail(e, "load launch");
+  Prof pn(kNorm, st, 0.0, 4.0 * (double)L.tiles_per_mat);
+  e = launch_norm_finalize(partials, 1, (int)L.tiles_per_mat, scale, nullptr, st);
+  pn.done(st);
+  if (e != cudaSuccess) return cuda_fail(e, "norm launch");
+  void* result = nullptr;
+  rc = run_chain(L, 1, m, n, ws, off, steps, sched, ds, st, &result);
+  if (rc != DMUON_OK) return rc;
+  Prof pc(kCopyOut, st, 0.0, 2.0 * elems * es);
+  e = launch_update(*tab, dtype, ElemMode::kCopyOut, result, steps == 0 ? scale : nullptr, 0.f, 0.f, n, st);
+  pc.done(st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy-out launch");
+  return DMUON_OK;
+}
+
+dmuon_status_t dmuon_ns(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,
+                        const float* coeffs, dmuon_stream_t stream) {
+  return dmuon_ns_ex(X, out, rows, cols, steps, coeffs, DMUON_BF16, stream);
+}
+
+// ---------------------------------------------------------------- stage calls
+static dmuon_status_t check_stage(const void* const* ptrs, int np, int64_t batch, int64_t m, int64_t n,
+                                  const int64_t* lds, const int64_t* ldmin, int nl, int32_t dtype) {
+  for (int i = 0; i < np; ++i)
+    if (!ptrs[i]) return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  if (batch < 0 || batch > 65535) return fail(DMUON_ERR_INVALID_ARG, "batch must be in 0..65535");
+  dmuon_status_t rc = check_shape(m, n, "stage call");
+  if (rc != DMUON_OK) return rc;
+  if (!dtype_ok(dtype)) return fail(DMUON_ERR_INVALID_ARG, "bad dtype");
+  for (int i = 0; i < nl; ++i)
+    if (lds[i] < ldmin[i]) return fail(DMUON_ERR_INVALID_ARG, "leading dimension smaller than the row");
+  if (dtype == DMUON_BF16) {
+    for (int i = 0; i < np; ++i)
+      if (!aligned16(ptrs[i])) return fail(DMUON_ERR_INVALID_ARG, "bf16 stage calls need 16-byte aligned pointers");
+    for (int i = 0; i < nl; ++i)
+      if (lds[i] % 8 != 0) return fail(DMUON_ERR_INVALID_ARG, "bf16 stage calls need leading dimensions % 8 == 0");
+  }
+  return DMUON_OK;
+}
+
+dmuon_status_t dmuon_gram(const void* X, void* G, int64_t batch, int64_t m, int64_t n, int64_t ldx,
+                          int64_t ldg, float alpha, int32_t dtype, dmuon_stream_t stream) {
+  const void* ptrs[2] = {X, G};
+  const int64_t lds[2] = {ldx, ldg}, mins[2] = {n, m};
+  dmuon_status_t rc = check_stage(ptrs, 2, batch, m, n, lds, mins, 2, dtype);
+  if (rc != DMUON_OK) return rc;
+  if (batch == 0) return DMUON_OK;
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == DMUON_BF16
+                      ? tc_gram(X, G, (int)batch, (int)m, (int)n, ldx, ldg, alpha, nullptr, ds.status_word,
+                                ds.sm_count, st)
+                      : simt_gram(X, G, (int)batch, (int)m, (int)n, ldx, ldg, alpha, nullptr, false, st);
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_gram");
+}
+
+dmuon_status_t dmuon_gram_poly(const void* G, void* P, int64_t batch, int64_t m, int64_t ldg, int64_t ldp,
+                               float b, float c, int32_t dtype, dmuon_stream_t stream) {
+  const void* ptrs[2] = {G, P};
+  const int64_t lds[2] = {ldg, ldp}, mins[2] = {m, m};
+  dmuon_status_t rc = check_stage(ptrs, 2, batch, m, m, lds, mins, 2, dtype);
+  if (rc != DMUON_OK) return rc;
+  if (batch == 0) return DMUON_OK;
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == DMUON_BF16
+                      ? tc_poly(G, P, (int)batch, (int)m, ldg, ldp, b, c, ds.status_word, ds.sm_count, st)
+                      : simt_poly(G, P, (int)batch, (int)m, ldg, ldp, b, c, st);
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_gram_poly");
+}
+
+dmuon_status_t dmuon_poly_apply(const void* P, const void* X, void* Y, int64_t batch, int64_t m, int64_t n,
+                                int64_t ldp, int64_t ldx, int64_t ldy, float a, float alpha, int32_t dtype,
+                                dmuon_stream_t stream) {
+  const void* ptrs[3] = {P, X, Y};
+  const int64_t lds[3] = {ldp, ldx, ldy}, mins[3] = {m, n, n};
+  dmuon_status_t rc = check_stage(ptrs, 3, batch, m, n, lds, mins, 3, dtype);
+  if (rc != DMUON_OK) return rc;
+  if (batch == 0) return DMUON_OK;
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == DMUON_BF16
+                      ? tc_apply(P, X, Y, (int)batch, (int)m, (int)n, ldp, ldx, ldy, a, alpha, nullptr,
+                                 ds.status_word, ds.sm_count, st)
+                      : simt_apply(P, X, Y, (int)batch, (int)m, (int)n, ldp, ldx, ldy, a, alpha, nullptr, false,
+                                   st);
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_poly_apply");
+}
+
+dmuon_status_t dmuon_momentum(void* buf, const void* grad, void* x0, int64_t rows, int64_t cols, float momentum,
+                              int32_t nesterov, int32_t dtype, double* sumsq, dmuon_stream_t stream) {
+  if (!buf || !grad || !x0) return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  dmuon_status_t rc = check_shape(rows, cols, "dmuon_momentum");
+  if (rc != DMUON_OK) return rc;
+  if (!dtype_ok(dtype)) return fail(DMUON_ERR_INVALID_ARG, "bad dtype");
+  if (nesterov != 0 && nesterov != 1) return fail(DMUON_ERR_INVALID_ARG, "nesterov must be 0 or 1");
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->m = rows;
+  tab->n = cols;
+  tab->ldn = cols;
+  tab->count = 1;
+  tab->tiles_per_mat = (int32_t)(((rows + kElemTile - 1) / kElemTile) * ((cols + kElemTile - 1) / kElemTile));
+  const size_t es = esize(dtype);
+  const bool row16 = (cols * (int64_t)es) % 16 == 0;
+  tab->e[0] = MatEntry{grad, buf, x0, 0, (row16 && aligned16(grad) && aligned16(buf)) ? 1 : 0};
+  void* wsv = nullptr;
+  rc = get_workspace((size_t)tab->tiles_per_mat * 4 + 256, st, &wsv);
+  if (rc != DMUON_OK) return rc;
+  float* partials = static_cast<float*>(wsv);
+  cudaError_t e = launch_momentum(*tab, dtype, ElemMode::kMomentum, x0, partials, momentum, nesterov, st);
+  if (e == cudaSuccess && sumsq) e = launch_norm_finalize(partials, 1, tab->tiles_per_mat, nullptr, sumsq, st);
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_momentum");
+}
+
+dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, int64_t cols, float lr, float wd,
+                            int32_t dtype, dmuon_stream_t stream) {
+  if (!param || !O) return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  dmuon_status_t rc = check_shape(rows, cols, "dmuon_update");
+  if (rc != DMUON_OK) return rc;
+  if (!dtype_ok(dtype)) return fail(DMUON_ERR_INVALID_ARG, "bad dtype");
+  if (!std::isfinite(lr) || !std::isfinite(wd)) return fail(DMUON_ERR_INVALID_ARG, "lr and wd must be finite");
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  std::unique_ptr<ElemTable> tab(new ElemTable());
+  // not oriented: the table's (m, n) is the matrix itself
+  const int64_t n = std::max(rows, cols);
+  tab->m = rows;
+  tab->n = cols;
+  tab->ldn = cols;
+  tab->count = 1;
+  tab->tiles_per_mat = (int32_t)(((rows + kElemTile - 1) / kElemTile) * ((cols + kElemTile - 1) / kElemTile));
+  const bool row16 = (cols * (int64_t)esize(dtype)) % 16 == 0;
+  tab->e[0] = MatEntry{nullptr, nullptr, param, 0, (row16 && aligned16(param)) ? 2 : 0};
+  cudaError_t e = launch_update(*tab, dtype, ElemMode::kUpdate, O, nullptr, lr, wd, n, st);
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_update");
+}
+
+dmuon_status_t dmuon_profile_start(void) {
+  for (ProfRec& r : g_prof) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return DMUON_OK;
+}
+
+int32_t dmuon_profile_stop(dmuon_kernel_stat_t* stats, int32_t max_stats) {
+  g_prof_on = false;
+  double ms[kNumKinds] = {0}, fl[kNumKinds] = {0}, by[kNumKinds] = {0};
+  int64_t cnt[kNumKinds] = {0};
+  bool ok = true;
+  if (!g_prof.empty() && cudaEventSynchronize(g_prof.back().b) != cudaSuccess) ok = false;
+  for (ProfRec& r : g_prof) {
+    float t = 0.f;
+    if (ok && cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) {
+      ms[r.kind] += t;
+      fl[r.kind] += r.flops;
+      by[r.kind] += r.bytes;
+      cnt[r.kind] += 1;
+    } else {
+      ok = false;
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof.clear();
+  if (!ok) {
+    fail(DMUON_ERR_CUDA, "profile events failed");
+    return -1;
+  }
+  int32_t n = 0;
+  for (int k = 0; k < kNumKinds; ++k) {
+    if (cnt[k] == 0) continue;
+    if (stats && n < max_stats) {
+      dmuon_kernel_stat_t& s = stats[n];
+      std::memset(&s, 0, sizeof(s));
+      std::strncpy(s.name, kKindNames[k], sizeof(s.name) - 1);
+      s.launches = cnt[k];
+      s.total_ms = ms[k];
+      s.flops = fl[k];
+      s.bytes = by[k];
+    }
+    ++n;
+  }
+  return n;
+}
+
+dmuon_status_t dmuon_stream_status(dmuon_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream");
+  DeviceState ds;
+  dmuon_status_t rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  int word = 0;
+  e = cudaMemcpy(&word, ds.status_word, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word != 0) {
+    cudaMemset(ds.status_word, 0, sizeof(int));
+    return fail((dmuon_status_t)word, "a device-side wait ran out (kernel gave up and returned)");
+  }
+  return DMUON_OK;
+}
+
+void dmuon_release_workspace(void) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  cudaDeviceSynchronize();
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (auto it = g_workspace.begin(); it != g_workspace.end();) {
+    if (it->first.first == dev) {
+      if (it->second.first) cudaFree(it->second.first);
+      it = g_workspace.erase(it);
+    } else {
+      ++it;
+    }
+  }
+}
+
+}  // extern "C"

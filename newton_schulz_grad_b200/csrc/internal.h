@@ -1,0 +1,127 @@
+// Internal host-side interfaces between the translation units of the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "dmuon.h"
+
+namespace dmuon {
+
+// Tile edge of the elementwise kernels (source-layout tiles, 64 x 64).
+constexpr int kElemTile = 64;
+// Matrices per elementwise launch (size of the pointer table in the kernel
+// parameters: 256 entries x 32 bytes).
+constexpr int kMaxTable = 256;
+// Largest min(rows, cols) that runs the FFMA chain with fp32 Gram matrices in
+// the bf16 path (bf16 rounding of G and p(G) is too coarse for such thin
+// matrices to meet the 2e-2 budget).
+constexpr int kSmallM = 64;
+
+// One matrix of an elementwise launch.  `src` is the gradient (momentum
+// stage) or the input matrix (load stage); `buf` the momentum buffer or NULL;
+// `dst` the parameter (update stage) or the output matrix (copy-out stage).
+struct MatEntry {
+  const void* src;
+  void* buf;
+  void* dst;
+  int32_t transposed;  // 1: source is n x m and is transposed into m x n
+  int32_t pad;         // bit 0: src and buf allow 16-byte vectors; bit 1: dst does
+};
+
+// All entries of one launch share the oriented shape m x n (m <= n) and the
+// workspace row pitch ldn; source shape is (m, n) or (n, m) per entry.
+struct ElemTable {
+  int64_t m, n, ldn;
+  int32_t count;
+  int32_t tiles_per_mat;  // ceil(m/64) * ceil(n/64)
+  MatEntry e[kMaxTable];
+};
+
+enum class ElemMode : int { kMomentum = 0, kLoad = 1, kUpdate = 2, kCopyOut = 3 };
+
+// Storage type of the Newton-Schulz chain.
+enum class Path : int {
+  kTensorBf16 = 0,   // bf16 X, G, P on tcgen05 tensor cores
+  kSmallBf16 = 1,    // bf16 X, fp32 G, P on FFMA
+  kF32 = 2           // fp32 X, G, P on FFMA
+};
+
+// ---- elementwise.cu --------------------------------------------------------
+// Momentum (or load) stage: writes x0 into X (batch pitch m*ldn elements,
+// transposed where the entry says so) and one fp32 sum-of-squares partial per
+// 64x64 tile into `partials` (tiles_per_mat per matrix).
+cudaError_t launch_momentum(const ElemTable& t, int dtype, ElemMode mode, void* X,
+                            float* partials, float mu, int nesterov, cudaStream_t st);
+// Sum the partials of each matrix in a fixed order; scale[i] = 1/(sqrt(sum)+eps).
+// sumsq (optional) receives the sums in fp64.
+cudaError_t launch_norm_finalize(const float* partials, int count, int tiles_per_mat,
+                                 float* scale, double* sumsq, cudaStream_t st);
+// Update (or copy-out) stage.  O is the oriented m x n result in the
+// workspace (pitch ldn); `scale` (optional, per matrix) multiplies O first.
+// The update uses lr * 0.2 * sqrt(scale_dim) (scale_dim = max(rows, cols)).
+cudaError_t launch_update(const ElemTable& t, int dtype, ElemMode mode, const void* O,
+                          const float* scale, float lr, float wd, int64_t scale_dim,
+                          cudaStream_t st);
+
+// ---- simt_gemm.cu -----------------------------------------------------------
+// FFMA chain kernels, batched over `batch` matrices with element batch strides.
+// xbf16: X is bf16 (else fp32); G and P are bf16 only when gbf16 (stage calls
+// of the bf16 dtype never come here; gbf16 is always false in practice).
+cudaError_t simt_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,
+                      float alpha, const float* scale, bool xbf16, cudaStream_t st);
+cudaError_t simt_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp,
+                      float b, float c, cudaStream_t st);
+cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, int n,
+                       int64_t ldp, int64_t ldx, int64_t ldy, float a, float alpha,
+                       const float* scale, bool xbf16, cudaStream_t st);
+
+// ---- tc_gemm.cu -------------------------------------------------------------
+// tcgen05 chain kernels (bf16 in/out, fp32 accumulation in TMEM).
+cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,
+                    float alpha, const float* scale, int* status, int num_sms, cudaStream_t st);
+cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b,
+                    float c, int* status, int num_sms, cudaStream_t st);
+cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
+                     int64_t ldx, int64_t ldy, float a, float alpha, const float* scale,
+                     int* status, int num_sms, cudaStream_t st);
+const char* tc_config_string();
+
+// ---- plan.cpp -----------------------------------------------------------------
+struct Group {
+  int64_t rows, cols;
+  int32_t dtype;
+  std::vector<int32_t> members;  // ascending indices
+};
+// Groups by (rows, cols, dtype) in order of first appearance.
+std::vector<Group> plan_groups(const dmuon_shape_t* shapes, int32_t count);
+
+// A launch class: groups with the same oriented shape (m, n) and dtype.
+struct LaunchClass {
+  int64_t m, n;
+  int32_t dtype;
+  std::vector<int32_t> members;  // in group order, ascending within a group
+};
+std::vector<LaunchClass> plan_classes(const std::vector<Group>& groups);
+
+// Per-chunk workspace layout of a launch class.
+struct ChunkLayout {
+  Path path;
+  int64_t ldn, ldm;        // row pitches (elements) of X and of G/P
+  int64_t xbytes, gbytes;  // bytes of one X (one matrix) and of one G
+  int64_t tiles_per_mat;   // elementwise tiles
+  int64_t per_matrix;      // workspace bytes per matrix in a chunk
+};
+ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype);
+int64_t workspace_cap_bytes();
+int64_t chunk_size(const ChunkLayout& L, int64_t members);
+// Offsets of the pieces of a chunk of `b` matrices inside the workspace.
+struct ChunkOffsets {
+  int64_t x0, x1, g, p, partials, scale, total;
+};
+ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b);
+
+}  // namespace dmuon

@@ -1,0 +1,102 @@
+// Host-side planning: shape groups, launch classes and workspace layout.
+//
+// Grouping by (rows, cols, dtype), ids in order of first appearance, members
+// ascending: many same-shape matrices (every layer's q_proj, or all MoE
+// experts) then run as one batched launch.  Groups whose oriented shape
+// (min, max) and dtype agree (e.g. gate_proj R x C and down_proj C x R) share a
+// launch class, because the Newton-Schulz chain only sees the oriented m x n
+// matrix.
+#include <algorithm>
+#include <cstdlib>
+#include <map>
+#include <tuple>
+
+#include "internal.h"
+
+namespace dmuon {
+
+std::vector<Group> plan_groups(const dmuon_shape_t* shapes, int32_t count) {
+  std::vector<Group> groups;
+  std::map<std::tuple<int64_t, int64_t, int32_t>, size_t> ids;
+  for (int32_t i = 0; i < count; ++i) {
+    auto key = std::make_tuple(shapes[i].rows, shapes[i].cols, shapes[i].dtype);
+    auto it = ids.find(key);
+    if (it == ids.end()) {
+      it = ids.emplace(key, groups.size()).first;
+      groups.push_back(Group{shapes[i].rows, shapes[i].cols, shapes[i].dtype, {}});
+    }
+    groups[it->second].members.push_back(i);
+  }
+  return groups;
+}
+
+std::vector<LaunchClass> plan_classes(const std::vector<Group>& groups) {
+  std::vector<LaunchClass> classes;
+  std::map<std::tuple<int64_t, int64_t, int32_t>, size_t> ids;
+  for (const Group& g : groups) {
+    const int64_t m = std::min(g.rows, g.cols), n = std::max(g.rows, g.cols);
+    auto key = std::make_tuple(m, n, g.dtype);
+    auto it = ids.find(key);
+    if (it == ids.end()) {
+      it = ids.emplace(key, classes.size()).first;
+      classes.push_back(LaunchClass{m, n, g.dtype, {}});
+    }
+    auto& mem = classes[it->second].members;
+    mem.insert(mem.end(), g.members.begin(), g.members.end());
+  }
+  return classes;
+}
+
+static int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype) {
+  ChunkLayout L{};
+  if (dtype == DMUON_F32)
+    L.path = Path::kF32;
+  else
+    L.path = (m <= kSmallM) ? Path::kSmallBf16 : Path::kTensorBf16;
+  const int64_t xs = dtype == DMUON_BF16 ? 2 : 4;
+  const int64_t gs = L.path == Path::kTensorBf16 ? 2 : 4;
+  // 16-byte row pitch: the TMA descriptors need it, vector loads like it
+  L.ldn = round_up(n, 8);
+  L.ldm = round_up(m, 8);
+  L.xbytes = m * L.ldn * xs;
+  L.gbytes = m * L.ldm * gs;
+  L.tiles_per_mat = ((m + kElemTile - 1) / kElemTile) * ((n + kElemTile - 1) / kElemTile);
+  L.per_matrix = 2 * L.xbytes + 2 * L.gbytes + L.tiles_per_mat * 4 + 4 + 6 * 256;
+  return L;
+}
+
+int64_t workspace_cap_bytes() {
+  const char* e = std::getenv("DMUON_WS_CAP_MB");
+  if (e && *e) {
+    long long mb = std::atoll(e);
+    if (mb > 0) return (int64_t)mb << 20;
+  }
+  return (int64_t)8 << 30;
+}
+
+// Largest chunk that fits the cap, then evened out over the chunks needed so
+// that no chunk is left with a small remainder.
+int64_t chunk_size(const ChunkLayout& L, int64_t members) {
+  int64_t c = workspace_cap_bytes() / std::max<int64_t>(1, L.per_matrix);
+  c = std::min<int64_t>(c, kMaxTable);
+  c = std::max<int64_t>(1, std::min<int64_t>(c, members));
+  const int64_t chunks = (members + c - 1) / c;
+  return std::max<int64_t>(1, (members + chunks - 1) / chunks);
+}
+
+ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b) {
+  ChunkOffsets o{};
+  int64_t at = 0;
+  o.x0 = at; at += round_up(b * L.xbytes, 256);
+  o.x1 = at; at += round_up(b * L.xbytes, 256);
+  o.g = at; at += round_up(b * L.gbytes, 256);
+  o.p = at; at += round_up(b * L.gbytes, 256);
+  o.partials = at; at += round_up(b * L.tiles_per_mat * 4, 256);
+  o.scale = at; at += round_up(b * 4, 256);
+  o.total = at;
+  return o;
+}
+
+}  // namespace dmuon

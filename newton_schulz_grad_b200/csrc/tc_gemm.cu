@@ -1,0 +1,593 @@
+// tcgen05 tensor-core kernels of the Gram Newton-Schulz chain (sm_100a).
+//
+// One iteration of Gram Newton-Schulz (the DMuon FAQ's related-work entry
+// for the default "gram" backend; Training Guide, ns_steps / ns_backend
+// rows) is three products over an m x n matrix X (m <= n):
+//   gram:  G = alpha X X^T        m x m, K = n   (symmetric: one triangle)
+//   poly:  P = b G + c G G        m x m, K = m   (G symmetric => G G = G G^T,
+//                                                  one triangle again)
+//   apply: Y = alpha (a X + P X)  m x n, K = m   (X is the MN-major operand)
+//
+// Kernel structure (one persistent CTA per SM, 192 threads):
+//   warp 0     TMA producer: 128B-swizzled K-slices of A (128 x 64) and B
+//              (256 x 64) into a 4-stage shared-memory ring, mbarrier
+//              transaction counts;
+//   warp 1     allocates 512 TMEM columns; one elected thread issues
+//              tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32) and commits
+//              stage releases / accumulator-ready to mbarriers;
+//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator (row = TMEM
+//              lane), the fused polynomial terms (alpha, b G, a X), bf16
+//              rounding and stores.  For gram/poly only tiles touching the
+//              lower triangle are computed; every element r >= c is stored,
+//              and r > c also at its mirror (c, r), so each element is
+//              written exactly once and G, P are exactly symmetric.
+// Two accumulators (2 x 256 columns) let the epilogue of tile t overlap the
+// MMAs of tile t+1.  Every mbarrier wait is bounded (%globaltimer); a wait
+// that runs out records DMUON_ERR_TIMEOUT in the status word, the CTA waits
+// (bounded) for its own copies and MMAs in flight, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace dmuon {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int UK = 16;  // K of one tcgen05.mma kind::f16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int kThreads = 192;
+constexpr int kBarriers = 2 * STAGES + 2 + 2 + 1;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s per wait
+
+enum { kGram = 0, kPoly = 1, kApply = 2 };
+
+struct TcArgs {
+  __nv_bfloat16* C;
+  const __nv_bfloat16* E;
+  int64_t sC, sE, ldc, lde;
+  int m, n, k;
+  int tiles_m, tiles_n, tiles_per_mat, total_tiles;
+  float p0, p1;
+  const float* scale;
+  int* status;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false when the limit ran out or another thread already failed.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 128; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(status) != 0) return false;
+    if (global_timer() - t0 > kTimeoutNs) {
+      atomicCAS(status, 0, (int)DMUON_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols));
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
+}
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
+// address, leading and stride byte offsets in 16-byte units, version 1 at
+// bit 46, swizzle mode 2 at bits 61-63).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: fp32 D, bf16 A and B, A K-major,
+// B K-major or MN-major, N = 256, M = 128.
+__host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+template <int MODE>
+__device__ __forceinline__ void decode_tile(const TcArgs& a, int t, int& b, int& I, int& J) {
+  b = t / a.tiles_per_mat;
+  int l = t - b * a.tiles_per_mat;
+  if (MODE == kApply) {
+    // column panels of X outermost, so concurrently running CTAs share them
+    I = l % a.tiles_m;
+    J = l / a.tiles_m;
+  } else {
+    int i = 0;
+    while (true) {
+      const int c = min(a.tiles_n, i / 2 + 1);
+      if (l < c) break;
+      l -= c;
+      ++i;
+    }
+    I = i;
+    J = l;
+  }
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& raw, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+__device__ __forceinline__ uint4 pack_bf16x8(const float* f) {
+  uint4 raw;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return raw;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+         const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarriers);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(tfull0 + 8 * s, 1);
+      mbar_init(tempty0 + 8 * s, 128);
+    }
+    mbar_init(done_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = (a.k + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
+        int b, I, J;
+        decode_tile<MODE>(a, t, b, I, J);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bar(empty0 + 8 * stage, phase ^ 1u, a.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          tma_load_3d(sa, &tmA, fb, kb * BK, I * BM, b);
+          if (MODE == kApply) {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmB, fb, J * BN + q * 64, kb * BK, b);
+          } else {
+            tma_load_3d(sb, &tmB, fb, kb * BK, J * BN, b);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // wait for the copies still in flight (all have landed on the normal path)
+      const int64_t first = issued > STAGES ? issued - STAGES : 0;
+      for (int64_t i = first; i < issued; ++i) {
+        const int s = (int)(i % STAGES);
+        const uint32_t par = (uint32_t)((i / STAGES) & 1);
+        if (!wait_bar(full0 + 8 * s, par, a.status)) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------------- MMA
+      constexpr uint32_t idesc = make_idesc(MODE == kApply);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
+        if (!wait_bar(tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bar(full0 + 8 * stage, phase, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k) {
+            const uint64_t ad = sdesc_sw128(sa + k * (UK * 2), 16, 1024);
+            const uint64_t bd = (MODE == kApply) ? sdesc_sw128(sb + k * (UK * 128), 8192, 1024)
+                                                 : sdesc_sw128(sb + k * (UK * 2), 16, 1024);
+            tc_mma(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // all MMAs issued by this thread complete before the CTA frees TMEM
+      tc_commit(done_bar);
+      wait_bar(done_bar, 0, a.status);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int wq = warp & 3;  // TMEM lanes 32*wq .. 32*wq+31
+    const int row_in_tile = wq * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
+      int b, I, J;
+      decode_tile<MODE>(a, t, b, I, J);
+      if (!wait_bar(tfull0 + 8 * acc, acc_phase, a.status)) break;
+      tc_fence_after();
+      const int r = I * BM + row_in_tile;
+      const bool row_ok = r < a.m;
+      float alpha = 1.f;
+      if (MODE == kGram) {
+        const float s = a.scale ? a.scale[b] : 1.f;
+        alpha = a.p0 * (s * s);
+      } else if (MODE == kApply) {
+        alpha = a.p1 * (a.scale ? a.scale[b] : 1.f);
+      }
+      __nv_bfloat16* Cm = a.C + (int64_t)b * a.sC;
+      const __nv_bfloat16* Em = a.E ? a.E + (int64_t)b * a.sE : nullptr;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int c0 = J * BN + ch * 32;
+        if (c0 >= a.n) break;  // warp-uniform
+        uint32_t raw[32];
+        tmem_ld32(tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN + ch * 32), raw);
+        tmem_ld_wait();
+        if (!row_ok) continue;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]);
+        const bool full_chunk = c0 + 32 <= a.n;
+        if (MODE == kApply) {
+          float e[32];
+          const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
+          if (full_chunk) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ep[j]) : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = alpha * fmaf(a.p0, e[j], v[j]);
+          __nv_bfloat16* cp = Cm + (int64_t)r * a.ldc + c0;
+          if (full_chunk) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(cp)[q] = pack_bf16x8(v + 8 * q);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < a.n) cp[j] = __float2bfloat16_rn(v[j]);
+          }
+        } else {
+          if (MODE == kPoly) {
+            float e[32];
+            const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
+            if (full_chunk) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ep[j]) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = fmaf(a.p1, v[j], a.p0 * e[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = alpha * v[j];
+          }
+          // lower triangle incl. diagonal at (r, c); strictly lower also at (c, r)
+          __nv_bfloat16 h[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) h[j] = __float2bfloat16_rn(v[j]);
+          __nv_bfloat16* rowp = Cm + (int64_t)r * a.ldc + c0;
+          if (full_chunk && r > c0 + 31) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(rowp)[q] = pack_bf16x8(v + 8 * q);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) Cm[(int64_t)(c0 + j) * a.ldc + r] = h[j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int c = c0 + j;
+              if (c < a.n && r >= c) {
+                rowp[j] = h[j];
+                if (r > c) Cm[(int64_t)c * a.ldc + r] = h[j];
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3D bf16 map: (inner, rows, batch), row pitch ld, batch pitch rows*ld.
+cudaError_t make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t batch,
+                     int64_t ld, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(rows * ld * 2)};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int tri_tiles_tc(int tiles_m, int tiles_n) {
+  int t = 0;
+  for (int i = 0; i < tiles_m; ++i) t += (tiles_n < i / 2 + 1) ? tiles_n : i / 2 + 1;
+  return t;
+}
+
+template <int MODE>
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms,
+                   cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int64_t total = (int64_t)a.tiles_per_mat * batch;
+  if (total <= 0) return cudaSuccess;
+  if (total > 0x7fffffff) return cudaErrorInvalidValue;
+  a.total_tiles = (int)total;
+  const int grid = (int)(total < num_sms ? total : num_sms);
+  k_tc<MODE><<<grid, kThreads, SMEM_BYTES, st>>>(ma, mb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg, float alpha,
+                    const float* scale, int* status, int num_sms, cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  CUtensorMap ma, mb;
+  cudaError_t e = make_map(&ma, X, n, m, batch, ldx, BK, BM);
+  if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, BK, BN);
+  if (e != cudaSuccess) return e;
+  TcArgs a{};
+  a.C = static_cast<__nv_bfloat16*>(G);
+  a.E = nullptr;
+  a.sC = (int64_t)m * ldg;
+  a.ldc = ldg;
+  a.m = m; a.n = m; a.k = n;
+  a.tiles_m = (m + BM - 1) / BM;
+  a.tiles_n = (m + BN - 1) / BN;
+  a.tiles_per_mat = tri_tiles_tc(a.tiles_m, a.tiles_n);
+  a.p0 = alpha;
+  a.scale = scale;
+  a.status = status;
+  return launch<kGram>(ma, mb, a, batch, num_sms, st);
+}
+
+cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b, float c,
+                    int* status, int num_sms, cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  CUtensorMap ma, mb;
+  cudaError_t e = make_map(&ma, G, m, m, batch, ldg, BK, BM);
+  if (e == cudaSuccess) e = make_map(&mb, G, m, m, batch, ldg, BK, BN);
+  if (e != cudaSuccess) return e;
+  TcArgs a{};
+  a.C = static_cast<__nv_bfloat16*>(P);
+  a.E = static_cast<const __nv_bfloat16*>(G);
+  a.sC = (int64_t)m * ldp;
+  a.sE = (int64_t)m * ldg;
+  a.ldc = ldp;
+  a.lde = ldg;
+  a.m = m; a.n = m; a.k = m;
+  a.tiles_m = (m + BM - 1) / BM;
+  a.tiles_n = (m + BN - 1) / BN;
+  a.tiles_per_mat = tri_tiles_tc(a.tiles_m, a.tiles_n);
+  a.p0 = b;
+  a.p1 = c;
+  a.status = status;
+  return launch<kPoly>(ma, mb, a, batch, num_sms, st);
+}
+
+cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
+                     int64_t ldx, int64_t ldy, float a_coef, float alpha, const float* scale, int* status,
+                     int num_sms, cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  CUtensorMap ma, mb;
+  cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, BM);
+  if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
+  if (e != cudaSuccess) return e;
+  TcArgs a{};
+  a.C = static_cast<__nv_bfloat16*>(Y);
+  a.E = static_cast<const __nv_bfloat16*>(X);
+  a.sC = (int64_t)m * ldy;
+  a.sE = (int64_t)m * ldx;
+  a.ldc = ldy;
+  a.lde = ldx;
+  a.m = m; a.n = n; a.k = m;
+  a.tiles_m = (m + BM - 1) / BM;
+  a.tiles_n = (n + BN - 1) / BN;
+  a.tiles_per_mat = a.tiles_m * a.tiles_n;
+  a.p0 = a_coef;
+  a.p1 = alpha;
+  a.scale = scale;
+  a.status = status;
+  return launch<kApply>(ma, mb, a, batch, num_sms, st);
+}
+
+const char* tc_config_string() {
+  return "tcgen05 cta_group::1 M128xN256xK16 bf16->fp32, BK=64 SW128, 4 stages, 2 TMEM accumulators, "
+         "persistent 192-thread CTAs (TMA warp, MMA warp, 4 epilogue warps)";
+}
+
+}  // namespace dmuon

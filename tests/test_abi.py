@@ -1,0 +1,120 @@
+"""Host-side tests of the C ABI: symbols, planning, validation (no GPU work)."""
+import ctypes
+import os
+import random
+import re
+
+import pytest
+import torch
+
+import newton_schulz_grad_b200 as nsg
+import workloads
+from oracle import muon as om
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dmuon.h")
+NO_GPU = not torch.cuda.is_available()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DMUON_API\s+[\w\s\*]+?\b(dmuon_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert len(syms) >= 15
+    lib = nsg.library()
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) == set(nsg.EXPORTED)
+
+
+def test_build_info_names_target():
+    info = nsg.dmuon_build_info()
+    assert "sm_100a" in info and "tcgen05" in info
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_plan_groups_matches_oracle(seed):
+    rng = random.Random(seed)
+    n = rng.randint(0, 60)
+    shapes = [(rng.choice([1, 32, 1024, 2816]), rng.choice([1, 32, 1024]), rng.randint(0, 1))
+              for _ in range(n)]
+    assert nsg.dmuon_plan_groups(shapes) == om.shape_groups(shapes)
+
+
+@pytest.mark.parametrize("w", workloads.WORKLOADS, ids=lambda w: w.name)
+def test_plan_groups_on_workloads(w):
+    code = 0 if w.dtype == "f32" else 1
+    shapes = [(r, c, code) for r, c in w.shapes]
+    g, order, k = nsg.dmuon_plan_groups(shapes)
+    assert (g, order, k) == om.shape_groups(shapes)
+    expect = {"single_256x512_f32": 1, "small_layer_bf16": 4, "llama3_2_3b_bf16": 4,
+              "llama_7b_bf16": 3, "moe_skewed_bf16": 4}[w.name]
+    assert k == expect
+
+
+def test_launch_count_and_workspace_llama7b():
+    w = workloads.get("llama_7b_bf16")
+    shapes = [(r, c, 1) for r, c in w.shapes]
+    # classes: 4096x4096 (128 matrices, 128 MiB of workspace each: 3 chunks of
+    # <= 43 under the 8 GiB cap) and 4096x11008 oriented (gate/up transposed +
+    # down: 96 matrices, 244 MiB each: 3 chunks of 32); per chunk momentum +
+    # norm + 3 per iteration + update
+    assert nsg.dmuon_step_launches(shapes, 5) == 6 * (3 + 15)
+    ws = nsg.dmuon_workspace_bytes(shapes, 5)
+    assert 5 << 30 < ws <= 8 << 30
+
+
+def _raw_step(count, params, grads, bufs, shapes, ns_steps=5, nesterov=1, lr=0.02):
+    lib = nsg.library()
+    vp = ctypes.c_void_p
+    pa = (vp * max(1, len(params)))(*params)
+    ga = (vp * max(1, len(grads)))(*grads)
+    ba = (vp * max(1, len(bufs)))(*bufs)
+    return lib.dmuon_step(pa, ga, ba, nsg._shape_array(shapes), count, lr, 0.95, nesterov,
+                          ns_steps, None, 0.0, None)
+
+
+def test_step_validation_errors():
+    A = 1 << 40
+    ok_shape = [(4, 8, 1)]
+    assert _raw_step(-1, [A], [A + 4096], [A + 8192], ok_shape) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(0, [], [], [], []) == nsg.DMUON_OK
+    assert _raw_step(1, [0], [A + 4096], [A + 8192], ok_shape) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(1, [A], [A + 4096], [A + 8192], [(0, 8, 1)]) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(1, [A], [A + 4096], [A + 8192], [(4, 8, 7)]) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(1, [A], [A + 4096], [A + 8192], [(1 << 21, 8, 1)]) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(1, [A], [A + 4096], [A + 8192], ok_shape, ns_steps=-1) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(1, [A], [A + 4096], [A + 8192], ok_shape, nesterov=2) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_step(1, [A], [A + 4096], [A + 8192], ok_shape, lr=float("nan")) == nsg.DMUON_ERR_INVALID_ARG
+    # overlap: the grad starts inside the param (4*8*2 = 64 bytes)
+    assert _raw_step(1, [A], [A + 32], [A + 8192], ok_shape) == nsg.DMUON_ERR_INVALID_ARG
+    assert "overlap" in nsg.dmuon_get_last_error()
+    # two matrices sharing a buffer
+    assert _raw_step(2, [A, A + 100000], [A + 4096, A + 200000], [A + 8192, A + 8192],
+                     ok_shape * 2) == nsg.DMUON_ERR_INVALID_ARG
+
+
+def test_stage_validation_errors():
+    lib = nsg.library()
+    A = 1 << 40
+    # bf16 stage calls need ld % 8 == 0 and 16-byte aligned pointers
+    assert lib.dmuon_gram(A, A + (1 << 20), 1, 100, 100, 100, 100, 1.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_gram(A + 2, A + (1 << 20), 1, 96, 96, 96, 96, 1.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_gram(A, A + (1 << 20), 1, 96, 96, 64, 96, 1.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_gram_poly(A, 0, 1, 96, 96, 96, 1.0, 1.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_poly_apply(A, A, A, -1, 8, 8, 8, 8, 8, 1.0, 1.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_ns_ex(A, A + 16, 4, 4, 5, None, 1, None) == nsg.DMUON_ERR_INVALID_ARG  # overlap
+    assert lib.dmuon_ns_ex(A, A + 4096, 4, 4, -2, None, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_momentum(A, A + 4096, A + 8192, 4, 4, 0.9, 3, 1, None, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_update(A, 0, 4, 4, 0.1, 0.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(not NO_GPU, reason="checks the no-device path")
+def test_valid_call_without_device_reports_cuda_error():
+    A = 1 << 40
+    rc = _raw_step(1, [A], [A + 4096], [A + 8192], [(4, 8, 1)])
+    assert rc in (nsg.DMUON_ERR_CUDA, nsg.DMUON_ERR_UNSUPPORTED)
+    assert nsg.dmuon_get_last_error()

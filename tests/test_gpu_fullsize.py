@@ -1,0 +1,42 @@
+"""Parity at the full benchmark size: the 224-matrix Llama-7B projection set.
+
+The whole set runs through one dmuon_step call, exactly as the benchmark
+launches it; the oracle then recomputes one sampled matrix per launch class
+(4096x4096, 11008x4096 transposed, 4096x11008) in fp64 on the host.
+"""
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_grad_b200 as nsg
+import workloads
+from oracle import emulate as em
+from oracle import muon as om
+from tests.gpu_util import to64
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def test_llama7b_full_step_sampled_parity():
+    w = workloads.get("llama_7b_bf16")
+    ps, gs, bs = workloads.make_all(w, "cuda")
+    sample = [1, 4, 6]  # k_proj (4096x4096), gate_proj (11008x4096), down_proj (4096x11008)
+    sample += [w.count - 3]  # a last-layer gate_proj (last chunk of its class)
+    saved = {i: (to64(ps[i]), gs[i].float().cpu().numpy(), bs[i].float().cpu().numpy())
+             for i in sample}
+    nsg.dmuon_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
+                   ns_steps=w.ns_steps, wd=w.wd)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    for i in sample:
+        p0, g, b = saved[i]
+        want_b, _ = em.momentum_fp32(b, g, w.momentum, w.nesterov, "bf16")
+        assert np.array_equal(bs[i].float().cpu().numpy().view(np.uint32), want_b.view(np.uint32))
+        p_new, _, _ = om.muon_step([p0], [g.astype(np.float64)], [b.astype(np.float64)], w.lr,
+                                   w.momentum, w.nesterov, w.ns_steps, None, w.wd)
+        got = to64(ps[i])
+        step = np.linalg.norm(p_new[0] - p0)
+        err = np.linalg.norm(got - p_new[0])
+        assert err <= 2e-2 * step + 2 ** -8 * np.linalg.norm(p_new[0]), (i, err / step)
+    # every parameter moved and stayed finite
+    for p in ps:
+        assert torch.isfinite(p).all()

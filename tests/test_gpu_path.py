@@ -1,0 +1,194 @@
+"""Whole-path GPU parity against the fp64 oracle, through the C ABI.
+
+Tolerances (per matrix, relative Frobenius):
+* Newton-Schulz output O: 2e-2 for bf16 storage, 1e-4 for fp32;
+* parameters: ||p_gpu - p_orc|| <= 2e-2 ||p_orc - p_old|| + 2^-8 ||p_orc||
+  (the update is small next to p, and bf16 storage of p rounds at 2^-9);
+* momentum buffers: bit for bit against the fp32 rounding-contract emulation.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_grad_b200 as nsg
+import workloads
+from oracle import emulate as em
+from oracle import muon as om
+from tests.gpu_util import bits, dtype_name, rel_fro, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NS_TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
+
+
+def lowrank_plus_noise(r, c, seed, dtype, rank=16, noise=1e-3):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    u, _ = torch.linalg.qr(torch.randn(r, min(rank, r, c), generator=g))
+    v, _ = torch.linalg.qr(torch.randn(c, min(rank, r, c), generator=g))
+    s = 1.0 / torch.arange(1, u.shape[1] + 1, dtype=torch.float32)
+    m = (u * s) @ v.T + noise * torch.randn(r, c, generator=g)
+    return m.to(dtype).to(DEV)
+
+
+NS_CASES = [
+    ((256, 512), torch.float32), ((40, 70), torch.float32), ((300, 129), torch.float32),
+    ((256, 512), torch.bfloat16), ((1024, 1024), torch.bfloat16), ((2816, 1024), torch.bfloat16),
+    ((1408, 2048), torch.bfloat16), ((2048, 1408), torch.bfloat16), ((32, 4096), torch.bfloat16),
+    ((4096, 32), torch.bfloat16), ((96, 200), torch.bfloat16), ((200, 97), torch.bfloat16),
+    ((65, 1000), torch.bfloat16), ((1, 300), torch.bfloat16), ((3, 5), torch.float32),
+]
+
+
+@pytest.mark.parametrize("shape,dtype", NS_CASES, ids=lambda v: str(v))
+def test_ns_matches_oracle(shape, dtype):
+    X = lowrank_plus_noise(*shape, seed=shape[0] * 7 + shape[1], dtype=dtype)
+    out = torch.empty_like(X)
+    nsg.dmuon_ns(X, out, steps=5)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    want = om.newton_schulz(to64(X), 5)
+    assert rel_fro(to64(out), want) < NS_TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_ns_custom_coefficients_and_zero_steps(dtype):
+    X = lowrank_plus_noise(192, 320, 5, dtype)
+    out = torch.empty_like(X)
+    coeffs = [(3.0, -3.2, 1.2), (2.0, -1.5, 0.5), (1.5, -0.5, 0.0)]
+    nsg.dmuon_ns(X, out, steps=3, coeffs=coeffs)
+    c32 = [tuple(float(np.float32(v)) for v in t) for t in coeffs]
+    assert rel_fro(to64(out), om.newton_schulz(to64(X), 3, c32)) < NS_TOL[dtype]
+    nsg.dmuon_ns(X, out, steps=0)
+    assert rel_fro(to64(out), om.newton_schulz(to64(X), 0)) < (4e-3 if dtype == torch.bfloat16 else 1e-6)
+
+
+def test_ns_convergent_polynomial_reaches_polar_factor():
+    X = lowrank_plus_noise(128, 256, 9, torch.float32, rank=128, noise=1e-2)
+    out = torch.empty_like(X)
+    nsg.dmuon_ns(X, out, steps=25, coeffs=(1.5, -0.5, 0.0))
+    u, _, vt = np.linalg.svd(to64(X), full_matrices=False)
+    assert rel_fro(to64(out), u @ vt) < 1e-4
+
+
+def test_ns_transpose_equivariance_bf16():
+    X = lowrank_plus_noise(384, 640, 3, torch.bfloat16)
+    a, b = torch.empty_like(X), torch.empty_like(X.T.contiguous())
+    nsg.dmuon_ns(X, a)
+    nsg.dmuon_ns(X.T.contiguous(), b)
+    torch.cuda.synchronize()
+    # the tall input is transposed into the same oriented matrix: identical bits
+    assert np.array_equal(bits(a), bits(b.T.contiguous()))
+
+
+def test_ns_zero_matrix():
+    X = torch.zeros(128, 256, dtype=torch.bfloat16, device=DEV)
+    out = torch.full_like(X, 7.0)
+    nsg.dmuon_ns(X, out)
+    assert torch.count_nonzero(out).item() == 0
+
+
+def run_step_check(w, idx=None, check_all=True):
+    """dmuon_step over workload w (or the matrices idx of it) against the oracle."""
+    sk = workloads.skewed_indices(w)
+    idx = list(range(w.count)) if idx is None else idx
+    mats = [workloads.make_matrix(w, i, DEV, sk) for i in idx]
+    ps = [m[0] for m in mats]
+    gs = [m[1] for m in mats]
+    bs = [m[2] for m in mats]
+    p_old = [to64(p) for p in ps]
+    g_h = [g.float().cpu().numpy() for g in gs]
+    b_h = [b.float().cpu().numpy() for b in bs]
+    nsg.dmuon_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
+                   ns_steps=w.ns_steps, wd=w.wd)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    worst = 0.0
+    for k in range(len(idx)):
+        dn = dtype_name(ps[k])
+        want_b, want_x = em.momentum_fp32(b_h[k], g_h[k], w.momentum, w.nesterov, dn)
+        assert np.array_equal(bs[k].float().cpu().numpy().view(np.uint32), want_b.view(np.uint32))
+        if not check_all and k % 1:
+            continue
+        p_new, _, _ = om.muon_step([p_old[k]], [g_h[k].astype(np.float64)],
+                                   [b_h[k].astype(np.float64)], w.lr, w.momentum, w.nesterov,
+                                   w.ns_steps, None, w.wd)
+        got = to64(ps[k])
+        step = np.linalg.norm(p_new[0] - p_old[k])
+        err = np.linalg.norm(got - p_new[0])
+        tol_rel = 2e-2 if dn == "bf16" else 1e-4
+        store = 2.0 ** -8 if dn == "bf16" else 1e-6
+        assert err <= tol_rel * step + store * np.linalg.norm(p_new[0]), (idx[k], err, step)
+        worst = max(worst, err / step)
+    return worst
+
+
+def test_step_single_matrix_f32():
+    run_step_check(workloads.get("single_256x512_f32"))
+
+
+def test_step_small_layer_bf16():
+    run_step_check(workloads.get("small_layer_bf16"))
+
+
+def test_step_moe_sampled():
+    w = workloads.get("moe_skewed_bf16")
+    sk = workloads.skewed_indices(w)
+    # two experts' matrices (one gate-shaped, one down-shaped), two skewed ones,
+    # three GateDelta 32x4096 and one tall 16384x2048
+    pick = sorted(set([0, 2, sk[0], sk[-1], 192, 200, 239, 240]))
+    run_step_check(w, pick)
+
+
+def test_step_batched_equals_solo_and_permuted():
+    w = workloads.get("small_layer_bf16")
+    mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
+
+    def run(order):
+        ps = [mats[i][0].clone() for i in order]
+        gs = [mats[i][1].clone() for i in order]
+        bs = [mats[i][2].clone() for i in order]
+        nsg.dmuon_step(ps, gs, bs)
+        torch.cuda.synchronize()
+        return {i: (bits(p), bits(b)) for i, p, b in zip(order, ps, bs)}
+
+    together = run(list(range(w.count)))
+    perm = run([6, 2, 0, 5, 3, 1, 4])
+    for i in range(w.count):
+        solo = run([i])
+        for res in (perm, solo):
+            assert np.array_equal(res[i][0], together[i][0])
+            assert np.array_equal(res[i][1], together[i][1])
+
+
+def test_step_zero_steps_and_no_nesterov():
+    w = workloads.get("small_layer_bf16")
+    ps, gs, bs = workloads.make_all(w, DEV)
+    p_old = [to64(p) for p in ps]
+    g_h = [g.float().cpu().numpy() for g in gs]
+    b_h = [b.float().cpu().numpy() for b in bs]
+    nsg.dmuon_step(ps, gs, bs, nesterov=False, ns_steps=0, wd=0.5, lr=0.01)
+    torch.cuda.synchronize()
+    for k in range(w.count):
+        p_new, _, _ = om.muon_step([p_old[k]], [g_h[k]], [b_h[k]], 0.01, 0.95, False, 0, None, 0.5)
+        err = np.linalg.norm(to64(ps[k]) - p_new[0])
+        assert err <= 2e-2 * np.linalg.norm(p_new[0] - p_old[k]) + 2 ** -8 * np.linalg.norm(p_new[0])
+
+
+def test_step_injected_allocation_failure_leaves_inputs(monkeypatch):
+    w = workloads.get("small_layer_bf16")
+    ps, gs, bs = workloads.make_all(w, DEV)
+    before = [bits(t) for t in ps + bs]
+    nsg.dmuon_release_workspace()
+    monkeypatch.setenv("DMUON_FAULT_INJECT", "alloc")
+    with pytest.raises(nsg.DmuonError) as ei:
+        nsg.dmuon_step(ps, gs, bs)
+    assert ei.value.status == nsg.DMUON_ERR_OOM
+    monkeypatch.delenv("DMUON_FAULT_INJECT")
+    torch.cuda.synchronize()
+    after = [bits(t) for t in ps + bs]
+    assert all(np.array_equal(a, b) for a, b in zip(before, after))
+
+
+def test_step_empty_list():
+    nsg.dmuon_step([], [], [])
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK

@@ -55,6 +55,11 @@ def parse_args(argv=None):
                     help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update"],
+                    help="time one kernel through its stage call instead of the whole step")
+    ap.add_argument("--batch", type=int, default=8)
+    ap.add_argument("--m", type=int, default=4096)
+    ap.add_argument("--n", type=int, default=4096)
     return ap.parse_args(argv)
 
 
@@ -447,9 +452,65 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_stage(args):
+    """One kernel through its stage call (bf16), e.g. for an ncu capture of a small case."""
+    import newton_schulz_grad_b200 as nsg
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    b, m, n = args.batch, args.m, args.n
+    gen = torch.Generator(device=dev).manual_seed(7)
+    bf = torch.bfloat16
+    if args.stage == "gram":
+        X = torch.randn(b, m, n, generator=gen, device=dev).to(bf)
+        out = torch.empty(b, m, m, dtype=bf, device=dev)
+        run = lambda: nsg.dmuon_gram(X, out)  # noqa: E731
+        flops, nbytes = b * m * m * n, 2 * b * (m * n + m * m)
+    elif args.stage == "poly":
+        G = torch.randn(b, m, m, generator=gen, device=dev)
+        G = ((G + G.transpose(1, 2)) / (2 * math.sqrt(m))).to(bf).contiguous()
+        out = torch.empty_like(G)
+        run = lambda: nsg.dmuon_gram_poly(G, out, -4.775, 2.0315)  # noqa: E731
+        flops, nbytes = b * m ** 3, 2 * b * 2 * m * m
+    elif args.stage == "apply":
+        P = (torch.randn(b, m, m, generator=gen, device=dev) / math.sqrt(m)).to(bf)
+        X = torch.randn(b, m, n, generator=gen, device=dev).to(bf)
+        out = torch.empty_like(X)
+        run = lambda: nsg.dmuon_poly_apply(P, X, out, 3.4445)  # noqa: E731
+        flops, nbytes = 2 * b * m * m * n, 2 * b * (m * m + 2 * m * n)
+    elif args.stage == "momentum":
+        g = torch.randn(m, n, generator=gen, device=dev).to(bf)
+        buf = torch.randn(m, n, generator=gen, device=dev).to(bf)
+        x0 = torch.empty_like(g)
+        run = lambda: nsg.dmuon_momentum(buf, g, x0, 0.95, True)  # noqa: E731
+        flops, nbytes = 0, 8 * m * n
+    else:
+        p = torch.randn(m, n, generator=gen, device=dev).to(bf)
+        o = torch.randn(m, n, generator=gen, device=dev).to(bf)
+        run = lambda: nsg.dmuon_update(p, o, 0.02, 0.0)  # noqa: E731
+        flops, nbytes = 0, 6 * m * n
+    for _ in range(max(args.warmup, 0)):
+        run()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        run()
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if nsg.dmuon_stream_status() != nsg.DMUON_OK:
+        raise RuntimeError("stage call failed")
+    print(json.dumps({"stage": args.stage, "batch": b, "m": m, "n": n, "ms": round(ms, 4),
+                      "tflops": round(flops / (ms / 1e3) / 1e12, 1) if flops else None,
+                      "GB/s": round(nbytes / (ms / 1e3) / 1e9, 1)}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.stage:
+        run_stage(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

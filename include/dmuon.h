@@ -197,6 +197,45 @@ DMUON_API dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, 
                             float wd, int32_t dtype, dmuon_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Allocation-free variant                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Size of the fixed scratch array behind dmuon_ns_noalloc (16 MiB).  Every
+ * GPU on which the library is loaded holds this array until the process
+ * exits. */
+#define DMUON_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * dmuon_ns_noalloc - dmuon_ns_ex for callers that must not allocate device
+ * memory.  The DMuon documentation has no counterpart: this entry point
+ * exists for callers such as a framework that has handed the whole device to
+ * its own caching allocator, or a loop that may not allocate after start-up
+ * (cudaMalloc can synchronise the device and its cost is unpredictable).
+ * Instead of the cached workspace of dmuon_ns_ex it uses one fixed
+ * DMUON_NOALLOC_SCRATCH_BYTES array in device memory that the library
+ * reserves when it is loaded; it never calls cudaMalloc or cudaFree.
+ *   X, out, rows, cols, steps, coeffs, dtype  as for dmuon_ns_ex
+ *   status  device, 1 int32, or NULL: cleared at the start of the call, then
+ *           set to DMUON_ERR_TIMEOUT if a bounded device wait ran out (with
+ *           NULL the word lives in the scratch array and is not reported)
+ * Limit: the problem must fit the array; a matrix whose workspace (two m x n
+ * copies of X, two m x m Gram-sized matrices and the norm partials, m =
+ * min(rows, cols)) exceeds it is rejected with DMUON_ERR_INVALID_ARG and a
+ * message naming both sizes.  Examples that fit: bf16 2048 x 1024, fp32
+ * 1024 x 512.
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's device address; make that first call before any stream
+ * capture.
+ * Sharing: every call on a device uses the same array and leaves its
+ * contents behind; calls that can overlap on the GPU (different streams
+ * without ordering between them, or several host threads) race on it and
+ * must be serialised by the caller.
+ */
+DMUON_API dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t rows, int64_t cols,
+                                          int32_t steps, const float* coeffs, int32_t dtype,
+                                          int32_t* status, dmuon_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Status, workspace, build information                                      */
 /* ------------------------------------------------------------------------ */
 

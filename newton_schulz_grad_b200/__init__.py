@@ -34,7 +34,7 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_gram_poly", "dmuon_poly_apply", "dmuon_momentum", "dmuon_update",
             "dmuon_get_last_error", "dmuon_stream_status", "dmuon_release_workspace",
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
-            "dmuon_profile_start", "dmuon_profile_stop")
+            "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc")
 
 
 class DmuonError(RuntimeError):
@@ -81,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_build_info": ([], ctypes.c_char_p),
         "dmuon_profile_start": ([], i32),
         "dmuon_profile_stop": ([ctypes.POINTER(KernelStat), i32], i32),
+        "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -177,6 +178,29 @@ def dmuon_ns(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=None, st
     c = _coeffs(steps, coeffs)
     _check(_lib.dmuon_ns_ex(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps, c,
                             _dtype_code(X), _stream(stream)))
+
+
+def dmuon_ns_noalloc(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=None,
+                     status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """dmuon_ns for callers that cannot allocate device memory.
+
+    The library keeps a fixed scratch array (``DMUON_NOALLOC_SCRATCH_BYTES``)
+    on each device and runs the same kernels as ``dmuon_ns`` in it, so this
+    call never allocates.  Matrices too large for the array are rejected.
+    ``status`` (a CUDA int32 tensor of one element, optional) receives
+    DMUON_ERR_TIMEOUT if a bounded device wait ran out.  Calls share the
+    array: calls that could overlap on the GPU must be serialised.
+    """
+    _need_cuda(X, out)
+    if X.shape != out.shape or X.dim() != 2 or X.dtype != out.dtype:
+        raise ValueError("X and out must be 2D tensors of equal shape and dtype")
+    if not (X.is_contiguous() and out.is_contiguous()):
+        raise ValueError("X and out must be contiguous")
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise ValueError("status must be a CUDA int32 tensor")
+    _check(_lib.dmuon_ns_noalloc(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps,
+                                 _coeffs(steps, coeffs), _dtype_code(X), _ptr(status),
+                                 _stream(stream)))
 
 
 def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],

@@ -230,6 +230,9 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
 int64_t chunk_launches(int32_t steps) { return 3 + 3 * (int64_t)steps; }
 
 }  // namespace
+
+dmuon_status_t record_error(dmuon_status_t s, const std::string& msg) { return fail(s, msg); }
+
 }  // namespace dmuon
 
 using namespace dmuon;

@@ -90,6 +90,10 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
                      int* status, int num_sms, cudaStream_t st);
 const char* tc_config_string();
 
+// ---- api.cu -------------------------------------------------------------------
+// Sets the message returned by dmuon_get_last_error on this thread; returns s.
+dmuon_status_t record_error(dmuon_status_t s, const std::string& msg);
+
 // ---- plan.cpp -----------------------------------------------------------------
 struct Group {
   int64_t rows, cols;

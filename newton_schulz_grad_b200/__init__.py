@@ -16,7 +16,8 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdmuon_b200.so")
+# DMUON_LIBRARY may name another build of the same library (e.g. a debug build)
+LIB_PATH = os.environ.get("DMUON_LIBRARY") or os.path.join(_HERE, "libdmuon_b200.so")
 
 DMUON_OK = 0
 DMUON_ERR_INVALID_ARG = 1

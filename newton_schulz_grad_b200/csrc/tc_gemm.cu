@@ -8,28 +8,40 @@
 //                                                  one triangle again)
 //   apply: Y = alpha (a X + P X)  m x n, K = m   (X is the MN-major operand)
 //
-// Kernel structure (one persistent CTA per SM, 192 threads):
-//   warp 0     TMA producer: 128B-swizzled K-slices of A (128 x 64) and B
-//              (256 x 64) into a 4-stage shared-memory ring, mbarrier
-//              transaction counts;
-//   warp 1     allocates 512 TMEM columns; one elected thread issues
-//              tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32) and commits
-//              stage releases / accumulator-ready to mbarriers;
-//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator (row = TMEM
-//              lane), the fused polynomial terms (alpha, b G, a X), bf16
-//              rounding and stores.  For gram/poly only tiles touching the
-//              lower triangle are computed; every element r >= c is stored,
-//              and r > c also at its mirror (c, r), so each element is
-//              written exactly once and G, P are exactly symmetric.
-// Two accumulators (2 x 256 columns) let the epilogue of tile t overlap the
-// MMAs of tile t+1.  Every mbarrier wait is bounded (%globaltimer); a wait
-// that runs out records DMUON_ERR_TIMEOUT in the status word, the CTA waits
-// (bounded) for its own copies and MMAs in flight, frees its TMEM and exits.
+// Two kernels share the tile decode and the epilogue:
+//
+// k_tc2 (m >= 256): a CTA pair (cluster of 2) computes 256 x 256 tiles with
+//   tcgen05.mma.cta_group::2 (M=256, N=256, K=16).  Each CTA stages its own
+//   128 rows of A and its own 128 columns of B (6 stages of 32 KB), so every
+//   byte brought into shared memory feeds twice the MMA work of a one-CTA
+//   128 x 256 tile.  Both CTAs' TMA copies complete on the leader CTA's
+//   full barrier (mapa address, .cta_group::2 copies); the leader's single
+//   MMA thread issues the pair's MMAs and its commits multicast to both CTAs'
+//   stage-release and accumulator-ready barriers; each CTA's epilogue reads
+//   its own 128 TMEM lanes and reports back to the leader.
+// k_tc (m < 256): one CTA per SM, 128 x 256 tiles, tcgen05.mma.cta_group::1
+//   (M=128), 4 stages of 48 KB.
+//
+// Both are persistent (one CTA, or CTA pair, per SM / SM pair), warp
+// specialised (warp 0 TMA producer, warp 1 TMEM allocator + single MMA
+// thread, warps 2-5 epilogue), with two TMEM accumulators (2 x 256 fp32
+// columns) so the epilogue of one tile overlaps the MMAs of the next.  The
+// polynomial terms (alpha, b G, a X) are fused into the epilogue.  For gram
+// and poly only tiles that touch the lower triangle are computed; every
+// element r >= c is stored, and r > c also at its mirror (c, r), so each
+// element is written exactly once and G, P are exactly symmetric.
+//
+// Every mbarrier wait is bounded (%globaltimer); a wait that runs out records
+// DMUON_ERR_TIMEOUT in the status word, the CTA waits (bounded) for its own
+// copies and MMAs in flight, frees its TMEM and exits.  No TMA load uses
+// cluster multicast.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "internal.h"
@@ -37,19 +49,30 @@
 namespace dmuon {
 namespace {
 
-constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int UK = 16;  // K of one tcgen05.mma kind::f16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int kThreads = 192;
-constexpr int kBarriers = 2 * STAGES + 2 + 2 + 1;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s per wait
+
+// one-CTA kernel
+constexpr int BM1 = 128;
+constexpr int STAGES1 = 4;
+constexpr int A1_BYTES = BM1 * BK * 2;   // 16 KB
+constexpr int B1_BYTES = BN * BK * 2;    // 32 KB
+constexpr int STAGE1_BYTES = A1_BYTES + B1_BYTES;
+// CTA-pair kernel (per CTA: 128 rows of A, 128 columns of B)
+constexpr int BM2 = 256;
+constexpr int STAGES2 = 6;
+constexpr int A2_BYTES = 128 * BK * 2;   // 16 KB
+constexpr int B2_BYTES = 128 * BK * 2;   // 16 KB
+constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
+
+constexpr int kMaxStages = STAGES2 > STAGES1 ? STAGES2 : STAGES1;
+constexpr int kBarriers = 2 * kMaxStages + 2 + 2 + 1;
+constexpr int SMEM1_BYTES = STAGES1 * STAGE1_BYTES + 1024 + 256;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 256;
 
 enum { kGram = 0, kPoly = 1, kApply = 2 };
 
@@ -58,6 +81,7 @@ struct TcArgs {
   const __nv_bfloat16* E;
   int64_t sC, sE, ldc, lde;
   int m, n, k;
+  int tm;  // tile rows: 128 (one CTA) or 256 (CTA pair)
   int tiles_m, tiles_n, tiles_per_mat, total_tiles;
   float p0, p1;
   const float* scale;
@@ -73,6 +97,20 @@ __device__ __forceinline__ uint64_t global_timer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
@@ -82,6 +120,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// arrive on a barrier given by its shared::cluster address (own or peer CTA)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -117,32 +159,76 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// CTA-pair copy into this CTA's shared memory, completing on the barrier at
+// `bar_cluster` (the leader CTA's full barrier).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+template <int G>
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols));
+  if (G == 1)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols));
+  else
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols));
 }
+template <int G>
 __device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  if (G == 1)
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
 }
+template <int G>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
+  if (G == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
+  else
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
 }
+template <int G>
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  if (G == 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// Completion of this thread's prior MMAs arrives on `bar` (own CTA) ...
+template <int G>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+  if (G == 1)
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+// ... or on the barrier at the same offset in every CTA of `mask`.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(mask)
+      : "memory");
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -171,12 +257,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 // Instruction descriptor, kind::f16: fp32 D, bf16 A and B, A K-major,
-// B K-major or MN-major, N = 256, M = 128.
-__host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major) {
+// B K-major or MN-major, N = 256, M = 128 (one CTA) or 256 (CTA pair).
+__host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int M) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Tile t -> (matrix b, row block I, column block J).
 template <int MODE>
 __device__ __forceinline__ void decode_tile(const TcArgs& a, int t, int& b, int& I, int& J) {
   b = t / a.tiles_per_mat;
@@ -186,9 +273,10 @@ __device__ __forceinline__ void decode_tile(const TcArgs& a, int t, int& b, int&
     I = l % a.tiles_m;
     J = l / a.tiles_m;
   } else {
+    // row block i holds the column blocks that reach the diagonal
     int i = 0;
     while (true) {
-      const int c = min(a.tiles_n, i / 2 + 1);
+      const int c = min(a.tiles_n, (i * a.tm + a.tm - 1) / BN + 1);
       if (l < c) break;
       l -= c;
       ++i;
@@ -215,6 +303,102 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* f) {
   return raw;
 }
 
+// Epilogue of one tile for one accumulator row: TMEM lane quarter `wq` of
+// accumulator columns [col0, col0 + 256), output row r, output columns from
+// J * 256.  Warp-collective (tcgen05.ld).
+template <int MODE>
+__device__ __forceinline__ void epilogue_row(const TcArgs& a, uint32_t taddr, int b, int r, int J) {
+  const bool row_ok = r < a.m;
+  float alpha = 1.f;
+  if (MODE == kGram) {
+    const float s = a.scale ? a.scale[b] : 1.f;
+    alpha = a.p0 * (s * s);
+  } else if (MODE == kApply) {
+    alpha = a.p1 * (a.scale ? a.scale[b] : 1.f);
+  }
+  __nv_bfloat16* Cm = a.C + (int64_t)b * a.sC;
+  const __nv_bfloat16* Em = a.E ? a.E + (int64_t)b * a.sE : nullptr;
+#pragma unroll 1
+  for (int ch = 0; ch < BN / 32; ++ch) {
+    const int c0 = J * BN + ch * 32;
+    if (c0 >= a.n) break;  // warp-uniform
+    uint32_t raw[32];
+    tmem_ld32(taddr + (uint32_t)(ch * 32), raw);
+    tmem_ld_wait();
+    if (!row_ok) continue;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]);
+    const bool full_chunk = c0 + 32 <= a.n;
+    if (MODE == kApply || MODE == kPoly) {
+      float e[32];
+      const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
+      if (full_chunk) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ep[j]) : 0.f;
+      }
+      if (MODE == kApply) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = alpha * fmaf(a.p0, e[j], v[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = fmaf(a.p1, v[j], a.p0 * e[j]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = alpha * v[j];
+    }
+    __nv_bfloat16* rowp = Cm + (int64_t)r * a.ldc + c0;
+    if (MODE == kApply) {
+      if (full_chunk) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(rowp)[q] = pack_bf16x8(v + 8 * q);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < a.n) rowp[j] = __float2bfloat16_rn(v[j]);
+      }
+    } else {
+      // lower triangle incl. diagonal at (r, c); strictly lower also at (c, r)
+      __nv_bfloat16 h[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) h[j] = __float2bfloat16_rn(v[j]);
+      if (full_chunk && r > c0 + 31) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(rowp)[q] = pack_bf16x8(v + 8 * q);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) Cm[(int64_t)(c0 + j) * a.ldc + r] = h[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int c = c0 + j;
+          if (c < a.n && r >= c) {
+            rowp[j] = h[j];
+            if (r > c) Cm[(int64_t)c * a.ldc + r] = h[j];
+          }
+        }
+      }
+    }
+  }
+}
+
+struct Bars {
+  uint32_t full0, empty0, tfull0, tempty0, done;
+};
+__device__ __forceinline__ Bars bar_layout(uint64_t* bars) {
+  Bars b;
+  b.full0 = smem_u32(bars);
+  b.empty0 = smem_u32(bars + kMaxStages);
+  b.tfull0 = smem_u32(bars + 2 * kMaxStages);
+  b.tempty0 = smem_u32(bars + 2 * kMaxStages + 2);
+  b.done = smem_u32(bars + 2 * kMaxStages + 4);
+  return b;
+}
+
+// ================================================================ one CTA
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -222,33 +406,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES1 * STAGE1_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarriers);
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + STAGES);
-  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
-  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+  const Bars B = bar_layout(bars);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
+    for (int s = 0; s < STAGES1; ++s) {
+      mbar_init(B.full0 + 8 * s, 1);
+      mbar_init(B.empty0 + 8 * s, 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(tfull0 + 8 * s, 1);
-      mbar_init(tempty0 + 8 * s, 128);
+      mbar_init(B.tfull0 + 8 * s, 1);
+      mbar_init(B.tempty0 + 8 * s, 4);  // one arrival per epilogue warp
     }
-    mbar_init(done_bar, 1);
+    mbar_init(B.done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<1>(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish<1>();
   }
   tc_fence_before();
   __syncthreads();
@@ -267,15 +447,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int b, I, J;
         decode_tile<MODE>(a, t, b, I, J);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(empty0 + 8 * stage, phase ^ 1u, a.status)) {
+          if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, a.status)) {
             ok = false;
             break;
           }
-          const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
-          tma_load_3d(sa, &tmA, fb, kb * BK, I * BM, b);
+          const uint32_t fb = B.full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, STAGE1_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * STAGE1_BYTES);
+          const uint32_t sb = sa + A1_BYTES;
+          tma_load_3d(sa, &tmA, fb, kb * BK, I * BM1, b);
           if (MODE == kApply) {
 #pragma unroll
             for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmB, fb, J * BN + q * 64, kb * BK, b);
@@ -283,163 +463,80 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sb, &tmB, fb, kb * BK, J * BN, b);
           }
           ++issued;
-          if (++stage == STAGES) {
+          if (++stage == STAGES1) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       // wait for the copies still in flight (all have landed on the normal path)
-      const int64_t first = issued > STAGES ? issued - STAGES : 0;
+      const int64_t first = issued > STAGES1 ? issued - STAGES1 : 0;
       for (int64_t i = first; i < issued; ++i) {
-        const int s = (int)(i % STAGES);
-        const uint32_t par = (uint32_t)((i / STAGES) & 1);
-        if (!wait_bar(full0 + 8 * s, par, a.status)) break;
+        if (!wait_bar(B.full0 + 8 * (int)(i % STAGES1), (uint32_t)((i / STAGES1) & 1), a.status)) break;
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       // ----------------------------------------------------------------- MMA
-      constexpr uint32_t idesc = make_idesc(MODE == kApply);
+      constexpr uint32_t idesc = make_idesc(MODE == kApply, BM1);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
-        if (!wait_bar(tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
+        if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(full0 + 8 * stage, phase, a.status)) {
+          if (!wait_bar(B.full0 + 8 * stage, phase, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sa = smem_u32(smem + stage * STAGE1_BYTES);
+          const uint32_t sb = sa + A1_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k) {
             const uint64_t ad = sdesc_sw128(sa + k * (UK * 2), 16, 1024);
             const uint64_t bd = (MODE == kApply) ? sdesc_sw128(sb + k * (UK * 128), 8192, 1024)
                                                  : sdesc_sw128(sb + k * (UK * 2), 16, 1024);
-            tc_mma(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            tc_mma<1>(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          tc_commit(empty0 + 8 * stage);
-          if (++stage == STAGES) {
+          tc_commit<1>(B.empty0 + 8 * stage);
+          if (++stage == STAGES1) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(tfull0 + 8 * acc);
+        tc_commit<1>(B.tfull0 + 8 * acc);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // all MMAs issued by this thread complete before the CTA frees TMEM
-      tc_commit(done_bar);
-      wait_bar(done_bar, 0, a.status);
+      tc_commit<1>(B.done);
+      wait_bar(B.done, 0, a.status);
     }
     __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue
     const int wq = warp & 3;  // TMEM lanes 32*wq .. 32*wq+31
-    const int row_in_tile = wq * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
       int b, I, J;
       decode_tile<MODE>(a, t, b, I, J);
-      if (!wait_bar(tfull0 + 8 * acc, acc_phase, a.status)) break;
+      if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
-      const int r = I * BM + row_in_tile;
-      const bool row_ok = r < a.m;
-      float alpha = 1.f;
-      if (MODE == kGram) {
-        const float s = a.scale ? a.scale[b] : 1.f;
-        alpha = a.p0 * (s * s);
-      } else if (MODE == kApply) {
-        alpha = a.p1 * (a.scale ? a.scale[b] : 1.f);
-      }
-      __nv_bfloat16* Cm = a.C + (int64_t)b * a.sC;
-      const __nv_bfloat16* Em = a.E ? a.E + (int64_t)b * a.sE : nullptr;
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int c0 = J * BN + ch * 32;
-        if (c0 >= a.n) break;  // warp-uniform
-        uint32_t raw[32];
-        tmem_ld32(tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN + ch * 32), raw);
-        tmem_ld_wait();
-        if (!row_ok) continue;
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]);
-        const bool full_chunk = c0 + 32 <= a.n;
-        if (MODE == kApply) {
-          float e[32];
-          const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
-          if (full_chunk) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ep[j]) : 0.f;
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = alpha * fmaf(a.p0, e[j], v[j]);
-          __nv_bfloat16* cp = Cm + (int64_t)r * a.ldc + c0;
-          if (full_chunk) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(cp)[q] = pack_bf16x8(v + 8 * q);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < a.n) cp[j] = __float2bfloat16_rn(v[j]);
-          }
-        } else {
-          if (MODE == kPoly) {
-            float e[32];
-            const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
-            if (full_chunk) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ep[j]) : 0.f;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = fmaf(a.p1, v[j], a.p0 * e[j]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = alpha * v[j];
-          }
-          // lower triangle incl. diagonal at (r, c); strictly lower also at (c, r)
-          __nv_bfloat16 h[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) h[j] = __float2bfloat16_rn(v[j]);
-          __nv_bfloat16* rowp = Cm + (int64_t)r * a.ldc + c0;
-          if (full_chunk && r > c0 + 31) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(rowp)[q] = pack_bf16x8(v + 8 * q);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) Cm[(int64_t)(c0 + j) * a.ldc + r] = h[j];
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = c0 + j;
-              if (c < a.n && r >= c) {
-                rowp[j] = h[j];
-                if (r > c) Cm[(int64_t)c * a.ldc + r] = h[j];
-              }
-            }
-          }
-        }
-      }
+      epilogue_row<MODE>(a, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
+                         I * BM1 + wq * 32 + lane, J);
       tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B.tempty0 + 8 * acc);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -449,7 +546,169 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc<1>(tmem_base, TMEM_COLS);
+  }
+}
+
+// =============================================================== CTA pair
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    k_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES2 * STAGE2_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarriers);
+  const Bars B = bar_layout(bars);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(B.full0 + 8 * s, 1);   // used in the leader: its arrive.expect_tx
+      mbar_init(B.empty0 + 8 * s, 1);  // the leader's MMA commit, multicast to both
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(B.tfull0 + 8 * s, 1);   // the leader's commit, multicast to both
+      mbar_init(B.tempty0 + 8 * s, 8);  // in the leader: one per epilogue warp of both CTAs
+    }
+    mbar_init(B.done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc<2>(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish<2>();
+  }
+  tc_fence_before();
+  cluster_sync();  // barrier initialisation and TMEM address visible in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = (a.k + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------- producer (both CTAs)
+      const uint32_t full_leader0 = mapa_shared(B.full0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < a.total_tiles; t += npairs) {
+        int b, I, J;
+        decode_tile<MODE>(a, t, b, I, J);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, a.status)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(B.full0 + 8 * stage, 2 * STAGE2_BYTES);
+          const uint32_t fb = full_leader0 + 8 * stage;
+          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
+          const uint32_t sb = sa + A2_BYTES;
+          tma_load_3d_pair(sa, &tmA, fb, kb * BK, I * BM2 + (int)rank * 128, b);
+          if (MODE == kApply) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+              tma_load_3d_pair(sb + q * 8192, &tmB, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
+          } else {
+            tma_load_3d_pair(sb, &tmB, fb, kb * BK, J * BN + (int)rank * 128, b);
+          }
+          ++issued;
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // the leader sees both CTAs' copies land on its full barriers
+      if (leader) {
+        const int64_t first = issued > STAGES2 ? issued - STAGES2 : 0;
+        for (int64_t i = first; i < issued; ++i) {
+          if (!wait_bar(B.full0 + 8 * (int)(i % STAGES2), (uint32_t)((i / STAGES2) & 1), a.status)) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------ MMA (leader)
+      constexpr uint32_t idesc = make_idesc(MODE == kApply, BM2);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < a.total_tiles; t += npairs) {
+        if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bar(B.full0 + 8 * stage, phase, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
+          const uint32_t sb = sa + A2_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k) {
+            const uint64_t ad = sdesc_sw128(sa + k * (UK * 2), 16, 1024);
+            const uint64_t bd = (MODE == kApply) ? sdesc_sw128(sb + k * (UK * 128), 8192, 1024)
+                                                 : sdesc_sw128(sb + k * (UK * 2), 16, 1024);
+            tc_mma<2>(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(B.empty0 + 8 * stage, 0x3);
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(B.tfull0 + 8 * acc, 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // all MMAs of the pair complete before either CTA frees TMEM
+      tc_commit<2>(B.done);
+      wait_bar(B.done, 0, a.status);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------- epilogue (both CTAs)
+    const int wq = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(B.tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < a.total_tiles; t += npairs) {
+      int b, I, J;
+      decode_tile<MODE>(a, t, b, I, J);
+      if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
+      tc_fence_after();
+      epilogue_row<MODE>(a, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
+                         I * BM2 + (int)rank * 128 + wq * 32 + lane, J);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while the pair may still signal its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<2>(tmem_base, TMEM_COLS);
   }
 }
 
@@ -487,27 +746,49 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int tri_tiles_tc(int tiles_m, int tiles_n) {
+int tri_tiles(int tiles_m, int tiles_n, int tm) {
   int t = 0;
-  for (int i = 0; i < tiles_m; ++i) t += (tiles_n < i / 2 + 1) ? tiles_n : i / 2 + 1;
+  for (int i = 0; i < tiles_m; ++i) {
+    const int c = (i * tm + tm - 1) / BN + 1;
+    t += tiles_n < c ? tiles_n : c;
+  }
   return t;
 }
 
+// The CTA-pair kernel runs when the matrix fills 256-row tiles; setting
+// DMUON_TC_CTA_PAIR=0 forces the one-CTA kernel (for comparisons).
+bool use_pair(int m) {
+  static int mode = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const char* e = std::getenv("DMUON_TC_CTA_PAIR");
+    mode = (e && std::strcmp(e, "0") == 0) ? 0 : 1;
+  });
+  return mode == 1 && m >= 256;
+}
+
 template <int MODE>
-cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms,
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms, bool pair,
                    cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(k_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(k_tc2<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int64_t total = (int64_t)a.tiles_per_mat * batch;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffff) return cudaErrorInvalidValue;
   a.total_tiles = (int)total;
-  const int grid = (int)(total < num_sms ? total : num_sms);
-  k_tc<MODE><<<grid, kThreads, SMEM_BYTES, st>>>(ma, mb, a);
+  if (pair) {
+    const int64_t pairs = total < num_sms / 2 ? total : num_sms / 2;
+    k_tc2<MODE><<<(int)(2 * pairs), kThreads, SMEM2_BYTES, st>>>(ma, mb, a);
+  } else {
+    const int grid = (int)(total < num_sms ? total : num_sms);
+    k_tc<MODE><<<grid, kThreads, SMEM1_BYTES, st>>>(ma, mb, a);
+  }
   return cudaGetLastError();
 }
 
@@ -516,9 +797,11 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int 
 cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg, float alpha,
                     const float* scale, int* status, int num_sms, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
+  const bool pair = use_pair(m);
   CUtensorMap ma, mb;
-  cudaError_t e = make_map(&ma, X, n, m, batch, ldx, BK, BM);
-  if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, BK, BN);
+  // A: 128 rows per CTA; B: 256 rows (one CTA) or 128 rows per CTA (pair)
+  cudaError_t e = make_map(&ma, X, n, m, batch, ldx, BK, 128);
+  if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, BK, pair ? 128 : BN);
   if (e != cudaSuccess) return e;
   TcArgs a{};
   a.C = static_cast<__nv_bfloat16*>(G);
@@ -526,21 +809,23 @@ cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx
   a.sC = (int64_t)m * ldg;
   a.ldc = ldg;
   a.m = m; a.n = m; a.k = n;
-  a.tiles_m = (m + BM - 1) / BM;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
   a.tiles_n = (m + BN - 1) / BN;
-  a.tiles_per_mat = tri_tiles_tc(a.tiles_m, a.tiles_n);
+  a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
   a.p0 = alpha;
   a.scale = scale;
   a.status = status;
-  return launch<kGram>(ma, mb, a, batch, num_sms, st);
+  return launch<kGram>(ma, mb, a, batch, num_sms, pair, st);
 }
 
 cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b, float c,
                     int* status, int num_sms, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
+  const bool pair = use_pair(m);
   CUtensorMap ma, mb;
-  cudaError_t e = make_map(&ma, G, m, m, batch, ldg, BK, BM);
-  if (e == cudaSuccess) e = make_map(&mb, G, m, m, batch, ldg, BK, BN);
+  cudaError_t e = make_map(&ma, G, m, m, batch, ldg, BK, 128);
+  if (e == cudaSuccess) e = make_map(&mb, G, m, m, batch, ldg, BK, pair ? 128 : BN);
   if (e != cudaSuccess) return e;
   TcArgs a{};
   a.C = static_cast<__nv_bfloat16*>(P);
@@ -550,21 +835,23 @@ cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64
   a.ldc = ldp;
   a.lde = ldg;
   a.m = m; a.n = m; a.k = m;
-  a.tiles_m = (m + BM - 1) / BM;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
   a.tiles_n = (m + BN - 1) / BN;
-  a.tiles_per_mat = tri_tiles_tc(a.tiles_m, a.tiles_n);
+  a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
   a.p0 = b;
   a.p1 = c;
   a.status = status;
-  return launch<kPoly>(ma, mb, a, batch, num_sms, st);
+  return launch<kPoly>(ma, mb, a, batch, num_sms, pair, st);
 }
 
 cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
                      int64_t ldx, int64_t ldy, float a_coef, float alpha, const float* scale, int* status,
                      int num_sms, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
+  const bool pair = use_pair(m);
   CUtensorMap ma, mb;
-  cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, BM);
+  cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
   if (e != cudaSuccess) return e;
   TcArgs a{};
@@ -575,19 +862,21 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
   a.ldc = ldy;
   a.lde = ldx;
   a.m = m; a.n = n; a.k = m;
-  a.tiles_m = (m + BM - 1) / BM;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
   a.tiles_n = (n + BN - 1) / BN;
   a.tiles_per_mat = a.tiles_m * a.tiles_n;
   a.p0 = a_coef;
   a.p1 = alpha;
   a.scale = scale;
   a.status = status;
-  return launch<kApply>(ma, mb, a, batch, num_sms, st);
+  return launch<kApply>(ma, mb, a, batch, num_sms, pair, st);
 }
 
 const char* tc_config_string() {
-  return "tcgen05 cta_group::1 M128xN256xK16 bf16->fp32, BK=64 SW128, 4 stages, 2 TMEM accumulators, "
-         "persistent 192-thread CTAs (TMA warp, MMA warp, 4 epilogue warps)";
+  return "tcgen05 bf16->fp32: CTA-pair kernel (cta_group::2, M256xN256xK16, 6 x 32 KB stages per CTA) for "
+         "m >= 256, one-CTA kernel (cta_group::1, M128xN256xK16, 4 x 48 KB stages) otherwise; BK=64 SW128, 2 TMEM "
+         "accumulators, persistent 192-thread CTAs (TMA warp, MMA warp, 4 epilogue warps)";
 }
 
 }  // namespace dmuon

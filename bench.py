@@ -55,6 +55,8 @@ def parse_args(argv=None):
                     help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ns-steps", type=int, default=None,
+                    help="override the workload's Newton-Schulz iteration count")
     ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update"],
                     help="time one kernel through its stage call instead of the whole step")
     ap.add_argument("--batch", type=int, default=8)
@@ -257,6 +259,9 @@ def run_ours(args):
                                 device_id=dev)
         pg = dist
     w = workloads.get(args.workload)
+    if args.ns_steps is not None:
+        import dataclasses
+        w = dataclasses.replace(w, ns_steps=args.ns_steps)
     ps, gs, bs = workloads.make_all(w, dev)
     code = 1 if w.dtype == "bf16" else 0
     shapes = [(r, c, code) for r, c in w.shapes]

@@ -38,6 +38,7 @@ NS_CASES = [
     ((1408, 2048), torch.bfloat16), ((2048, 1408), torch.bfloat16), ((32, 4096), torch.bfloat16),
     ((4096, 32), torch.bfloat16), ((96, 200), torch.bfloat16), ((200, 97), torch.bfloat16),
     ((65, 1000), torch.bfloat16), ((1, 300), torch.bfloat16), ((3, 5), torch.float32),
+    ((130, 1001), torch.bfloat16), ((1001, 130), torch.bfloat16), ((77, 333), torch.float32),
 ]
 
 

@@ -106,6 +106,38 @@ dmuon_status_t get_workspace(size_t bytes, cudaStream_t st, void** out) {
   return DMUON_OK;
 }
 
+// Auxiliary stream per (device, caller stream) for the elementwise stages of
+// an overlapped step.
+std::map<std::pair<int, uintptr_t>, cudaStream_t> g_aux;
+
+dmuon_status_t get_aux_stream(cudaStream_t st, cudaStream_t* out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto key = std::make_pair(dev, reinterpret_cast<uintptr_t>(st));
+  auto it = g_aux.find(key);
+  if (it == g_aux.end()) {
+    cudaStream_t aux = nullptr;
+    e = cudaStreamCreateWithFlags(&aux, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
+    it = g_aux.emplace(key, aux).first;
+  }
+  *out = it->second;
+  return DMUON_OK;
+}
+
+// `waiter` waits for everything enqueued so far on `signaller`.
+cudaError_t stream_after(cudaStream_t waiter, cudaStream_t signaller) {
+  cudaEvent_t ev;
+  cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+  if (e != cudaSuccess) return e;
+  e = cudaEventRecord(ev, signaller);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(waiter, ev, 0);
+  cudaEventDestroy(ev);  // released once the recorded work completes
+  return e;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t esize(int32_t dtype) { return dtype == DMUON_BF16 ? 2 : 4; }
 bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
@@ -266,24 +298,13 @@ dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int
 int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
   (void)ns_steps;
   if (count <= 0 || !shapes) return 0;
-  int64_t best = 0;
-  for (const LaunchClass& c : plan_classes(plan_groups(shapes, count))) {
-    ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
-    best = std::max(best, chunk_offsets(L, chunk_size(L, (int64_t)c.members.size())).total);
-  }
-  return best;
+  const StepPlan P = make_step_plan(shapes, count);
+  return P.buffer_bytes * (P.overlap ? 2 : 1);
 }
 
 int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
   if (count <= 0 || !shapes) return 0;
-  int64_t n = 0;
-  for (const LaunchClass& c : plan_classes(plan_groups(shapes, count))) {
-    ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
-    const int64_t cs = chunk_size(L, (int64_t)c.members.size());
-    const int64_t chunks = ((int64_t)c.members.size() + cs - 1) / cs;
-    n += chunks * chunk_launches(ns_steps);
-  }
-  return n;
+  return (int64_t)make_step_plan(shapes, count).chunks.size() * chunk_launches(ns_steps);
 }
 
 dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
@@ -322,63 +343,128 @@ dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* c
   DeviceState ds;
   dmuon_status_t rc = device_state(&ds);
   if (rc != DMUON_OK) return rc;
-  std::vector<LaunchClass> classes = plan_classes(plan_groups(shapes, count));
-  int64_t ws_bytes = 0;
-  for (const LaunchClass& c : classes) {
-    ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
-    ws_bytes = std::max(ws_bytes, chunk_offsets(L, chunk_size(L, (int64_t)c.members.size())).total);
-  }
+  const StepPlan P = make_step_plan(shapes, count);
+  const int nbuf = P.overlap ? 2 : 1;
   void* wsv = nullptr;
-  rc = get_workspace((size_t)ws_bytes, st, &wsv);
+  rc = get_workspace((size_t)(P.buffer_bytes * nbuf), st, &wsv);
   if (rc != DMUON_OK) return rc;
-  char* ws = static_cast<char*>(wsv);
-  std::unique_ptr<ElemTable> tab(new ElemTable());
+  // elementwise stages run on `aux` when overlapping, else on the caller's stream
+  cudaStream_t aux = st;
+  if (P.overlap) {
+    rc = get_aux_stream(st, &aux);
+    if (rc != DMUON_OK) return rc;
+    cudaError_t e = stream_after(aux, st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream fork");
+  }
+  std::unique_ptr<ElemTable[]> tabs(new ElemTable[2]);
+  std::vector<void*> results(P.chunks.size(), nullptr);
+
+  auto fill_table = [&](const ChunkRef& ck, ElemTable& tab) {
+    const LaunchClass& c = P.classes[ck.cls];
+    const size_t es = esize(c.dtype);
+    tab.m = c.m;
+    tab.n = c.n;
+    tab.ldn = P.layouts[ck.cls].ldn;
+    tab.count = ck.b;
+    tab.tiles_per_mat = (int32_t)P.layouts[ck.cls].tiles_per_mat;
+    for (int j = 0; j < ck.b; ++j) {
+      const int32_t i = c.members[ck.start + j];
+      MatEntry& e = tab.e[j];
+      e.src = grads[i];
+      e.buf = mom_bufs[i];
+      e.dst = params[i];
+      e.transposed = shapes[i].rows > shapes[i].cols ? 1 : 0;
+      const bool row16 = ((int64_t)shapes[i].cols * (int64_t)es) % 16 == 0;
+      e.pad = ((row16 && aligned16(grads[i]) && aligned16(mom_bufs[i])) ? 1 : 0) |
+              ((row16 && aligned16(params[i])) ? 2 : 0);
+    }
+  };
+  auto buffer = [&](size_t i) { return static_cast<char*>(wsv) + (int64_t)(i % nbuf) * P.buffer_bytes; };
+  auto update = [&](size_t i) -> dmuon_status_t {
+    const ChunkRef& ck = P.chunks[i];
+    const LaunchClass& c = P.classes[ck.cls];
+    const ChunkOffsets off = chunk_offsets(P.layouts[ck.cls], ck.b);
+    const float* scale = reinterpret_cast<const float*>(buffer(i) + off.scale);
+    const double elems = (double)ck.b * (double)c.m * (double)c.n;
+    Prof pu(kUpdate, aux, 0.0, 3.0 * elems * (double)esize(c.dtype));
+    cudaError_t e = launch_update(tabs[i % 2], c.dtype, ElemMode::kUpdate, results[i], ns_steps == 0 ? scale : nullptr,
+                                  lr, wd, c.n, aux);
+    pu.done(aux);
+    return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "update launch");
+  };
 
   // ------------------------------------------------------------ execution
-  for (const LaunchClass& c : classes) {
-    const ChunkLayout L = chunk_layout(c.m, c.n, c.dtype);
-    const int64_t cs = chunk_size(L, (int64_t)c.members.size());
-    const size_t es = esize(c.dtype);
-    for (size_t start = 0; start < c.members.size(); start += (size_t)cs) {
-      const int b = (int)std::min<int64_t>(cs, (int64_t)(c.members.size() - start));
-      const ChunkOffsets off = chunk_offsets(L, b);
-      tab->m = c.m;
-      tab->n = c.n;
-      tab->ldn = L.ldn;
-      tab->count = b;
-      tab->tiles_per_mat = (int32_t)L.tiles_per_mat;
-      for (int j = 0; j < b; ++j) {
-        const int32_t i = c.members[start + j];
-        MatEntry& e = tab->e[j];
-        e.src = grads[i];
-        e.buf = mom_bufs[i];
-        e.dst = params[i];
-        e.transposed = shapes[i].rows > shapes[i].cols ? 1 : 0;
-        const bool row16 = ((int64_t)shapes[i].cols * (int64_t)es) % 16 == 0;
-        e.pad = ((row16 && aligned16(grads[i]) && aligned16(mom_bufs[i])) ? 1 : 0) |
-                ((row16 && aligned16(params[i])) ? 2 : 0);
-      }
-      float* partials = reinterpret_cast<float*>(ws + off.partials);
-      float* scale = reinterpret_cast<float*>(ws + off.scale);
-      const double elems = (double)b * (double)c.m * (double)c.n;
-      Prof pm(kMomentum, st, 0.0, 4.0 * elems * (double)es);
-      cudaError_t e = launch_momentum(*tab, c.dtype, ElemMode::kMomentum, ws + off.x0, partials, momentum,
-                                      nesterov, st);
-      pm.done(st);
-      if (e != cudaSuccess) return cuda_fail(e, "momentum launch");
-      Prof pn(kNorm, st, 0.0, 4.0 * (double)b * (double)L.tiles_per_mat);
-      e = launch_norm_finalize(partials, b, (int)L.tiles_per_mat, scale, nullptr, st);
-      pn.done(st);
-      if (e != cudaSuccess) return cuda_fail(e, "norm launch");
-      void* result = nullptr;
-      rc = run_chain(L, b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &result);
-      if (rc != DMUON_OK) return rc;
-      Prof pu(kUpdate, st, 0.0, 3.0 * elems * (double)es);
-      e = launch_update(*tab, c.dtype, ElemMode::kUpdate, result, ns_steps == 0 ? scale : nullptr, lr, wd,
-                        c.n, st);
-      pu.done(st);
-      if (e != cudaSuccess) return cuda_fail(e, "update launch");
+  // aux: M0 N0 | M1 N1 U0 | M2 N2 U1 | ...   caller: chain0 | chain1 | ...
+  // U(i-1) waits only for chain(i-1) (event recorded when it was enqueued).
+  cudaEvent_t chain_done = nullptr;
+  auto drop = [&]() {
+    if (chain_done) cudaEventDestroy(chain_done);  // released once complete
+    chain_done = nullptr;
+  };
+  for (size_t i = 0; i < P.chunks.size(); ++i) {
+    const ChunkRef& ck = P.chunks[i];
+    const LaunchClass& c = P.classes[ck.cls];
+    const ChunkLayout& L = P.layouts[ck.cls];
+    const ChunkOffsets off = chunk_offsets(L, ck.b);
+    char* ws = buffer(i);
+    fill_table(ck, tabs[i % 2]);
+    float* partials = reinterpret_cast<float*>(ws + off.partials);
+    float* scale = reinterpret_cast<float*>(ws + off.scale);
+    const double elems = (double)ck.b * (double)c.m * (double)c.n;
+    Prof pm(kMomentum, aux, 0.0, 4.0 * elems * (double)esize(c.dtype));
+    cudaError_t e = launch_momentum(tabs[i % 2], c.dtype, ElemMode::kMomentum, ws + off.x0, partials, momentum,
+                                    nesterov, aux);
+    pm.done(aux);
+    if (e != cudaSuccess) {
+      drop();
+      return cuda_fail(e, "momentum launch");
     }
+    Prof pn(kNorm, aux, 0.0, 4.0 * (double)ck.b * (double)L.tiles_per_mat);
+    e = launch_norm_finalize(partials, ck.b, (int)L.tiles_per_mat, scale, nullptr, aux);
+    pn.done(aux);
+    if (e == cudaSuccess && P.overlap) e = stream_after(st, aux);
+    if (e != cudaSuccess) {
+      drop();
+      return cuda_fail(e, "norm launch / stream join");
+    }
+    rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &results[i]);
+    if (rc != DMUON_OK) {
+      drop();
+      return rc;
+    }
+    if (!P.overlap) {
+      rc = update(i);
+      if (rc != DMUON_OK) return rc;
+      continue;
+    }
+    if (i >= 1) {
+      e = cudaStreamWaitEvent(aux, chain_done, 0);
+      if (e != cudaSuccess) {
+        drop();
+        return cuda_fail(e, "stream fork");
+      }
+      rc = update(i - 1);
+      if (rc != DMUON_OK) {
+        drop();
+        return rc;
+      }
+    }
+    drop();
+    e = cudaEventCreateWithFlags(&chain_done, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(chain_done, st);
+    if (e != cudaSuccess) {
+      drop();
+      return cuda_fail(e, "chain event");
+    }
+  }
+  if (P.overlap) {
+    cudaError_t e = cudaStreamWaitEvent(aux, chain_done, 0);
+    drop();
+    if (e != cudaSuccess) return cuda_fail(e, "stream fork");
+    rc = update(P.chunks.size() - 1);
+    if (rc != DMUON_OK) return rc;
+    e = stream_after(st, aux);
+    if (e != cudaSuccess) return cuda_fail(e, "stream join");
   }
   return DMUON_OK;
 }
@@ -652,6 +738,14 @@ void dmuon_release_workspace(void) {
     if (it->first.first == dev) {
       if (it->second.first) cudaFree(it->second.first);
       it = g_workspace.erase(it);
+    } else {
+      ++it;
+    }
+  }
+  for (auto it = g_aux.begin(); it != g_aux.end();) {
+    if (it->first.first == dev) {
+      cudaStreamDestroy(it->second);
+      it = g_aux.erase(it);
     } else {
       ++it;
     }

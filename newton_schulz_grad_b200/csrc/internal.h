@@ -121,11 +121,29 @@ struct ChunkLayout {
 };
 ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype);
 int64_t workspace_cap_bytes();
-int64_t chunk_size(const ChunkLayout& L, int64_t members);
+int64_t chunk_size(const ChunkLayout& L, int64_t members, int64_t cap);
 // Offsets of the pieces of a chunk of `b` matrices inside the workspace.
 struct ChunkOffsets {
   int64_t x0, x1, g, p, partials, scale, total;
 };
 ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b);
+
+// The chunks of one dmuon_step in execution order.  With two or more chunks
+// (and DMUON_OVERLAP not "0") the step runs overlapped: two workspace buffers
+// of half the cap each, chunk i in buffer i % 2, the elementwise stages of
+// neighbouring chunks on an auxiliary stream under the Newton-Schulz chain.
+struct ChunkRef {
+  size_t cls;    // launch class
+  size_t start;  // first member of the class in this chunk
+  int b;         // matrices in the chunk
+};
+struct StepPlan {
+  std::vector<LaunchClass> classes;
+  std::vector<ChunkLayout> layouts;
+  std::vector<ChunkRef> chunks;
+  bool overlap = false;
+  int64_t buffer_bytes = 0;  // one buffer (two are used when overlapping)
+};
+StepPlan make_step_plan(const dmuon_shape_t* shapes, int32_t count);
 
 }  // namespace dmuon

@@ -78,12 +78,39 @@ int64_t workspace_cap_bytes() {
 
 // Largest chunk that fits the cap, then evened out over the chunks needed so
 // that no chunk is left with a small remainder.
-int64_t chunk_size(const ChunkLayout& L, int64_t members) {
-  int64_t c = workspace_cap_bytes() / std::max<int64_t>(1, L.per_matrix);
+int64_t chunk_size(const ChunkLayout& L, int64_t members, int64_t cap) {
+  int64_t c = cap / std::max<int64_t>(1, L.per_matrix);
   c = std::min<int64_t>(c, kMaxTable);
   c = std::max<int64_t>(1, std::min<int64_t>(c, members));
   const int64_t chunks = (members + c - 1) / c;
   return std::max<int64_t>(1, (members + chunks - 1) / chunks);
+}
+
+StepPlan make_step_plan(const dmuon_shape_t* shapes, int32_t count) {
+  StepPlan P;
+  P.classes = plan_classes(plan_groups(shapes, count));
+  for (const LaunchClass& c : P.classes) P.layouts.push_back(chunk_layout(c.m, c.n, c.dtype));
+  const char* ov = std::getenv("DMUON_OVERLAP");
+  const bool allow = !(ov && ov[0] == '0');
+  const int64_t cap = workspace_cap_bytes();
+  for (int pass = 0; pass < 2; ++pass) {
+    // pass 0: one buffer with the whole cap; pass 1: two buffers of half the cap
+    const int64_t cap_b = pass == 0 ? cap : cap / 2;
+    P.chunks.clear();
+    P.buffer_bytes = 0;
+    for (size_t k = 0; k < P.classes.size(); ++k) {
+      const int64_t mem = (int64_t)P.classes[k].members.size();
+      const int64_t cs = chunk_size(P.layouts[k], mem, cap_b);
+      for (int64_t start = 0; start < mem; start += cs) {
+        const int b = (int)std::min<int64_t>(cs, mem - start);
+        P.chunks.push_back(ChunkRef{k, (size_t)start, b});
+        P.buffer_bytes = std::max(P.buffer_bytes, chunk_offsets(P.layouts[k], b).total);
+      }
+    }
+    P.overlap = pass == 1;
+    if (pass == 0 && (!allow || P.chunks.size() < 2)) break;
+  }
+  return P;
 }
 
 ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b) {

@@ -58,13 +58,22 @@ def test_plan_groups_on_workloads(w):
 def test_launch_count_and_workspace_llama7b():
     w = workloads.get("llama_7b_bf16")
     shapes = [(r, c, 1) for r, c in w.shapes]
-    # classes: 4096x4096 (128 matrices, 128 MiB of workspace each: 3 chunks of
-    # <= 43 under the 8 GiB cap) and 4096x11008 oriented (gate/up transposed +
-    # down: 96 matrices, 244 MiB each: 3 chunks of 32); per chunk momentum +
-    # norm + 3 per iteration + update
-    assert nsg.dmuon_step_launches(shapes, 5) == 6 * (3 + 15)
+    # classes: 4096x4096 (128 matrices, 128 MiB of workspace each) and
+    # 4096x11008 oriented (gate/up transposed + down: 96 matrices, 244 MiB
+    # each).  Several chunks -> overlapped execution with two buffers of half
+    # the 8 GiB cap: 5 chunks of <= 26 and 6 chunks of 16; per chunk momentum
+    # + norm + 3 per iteration + update
+    assert nsg.dmuon_step_launches(shapes, 5) == 11 * (3 + 15)
     ws = nsg.dmuon_workspace_bytes(shapes, 5)
     assert 5 << 30 < ws <= 8 << 30
+
+
+def test_overlap_can_be_disabled(monkeypatch):
+    w = workloads.get("llama_7b_bf16")
+    shapes = [(r, c, 1) for r, c in w.shapes]
+    monkeypatch.setenv("DMUON_OVERLAP", "0")
+    assert nsg.dmuon_step_launches(shapes, 5) == 6 * (3 + 15)
+    assert nsg.dmuon_workspace_bytes(shapes, 5) <= 8 << 30
 
 
 def _raw_step(count, params, grads, bufs, shapes, ns_steps=5, nesterov=1, lr=0.02):

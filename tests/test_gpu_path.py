@@ -161,6 +161,32 @@ def test_step_batched_equals_solo_and_permuted():
             assert np.array_equal(res[i][1], together[i][1])
 
 
+def test_step_overlapped_equals_serial(monkeypatch):
+    # several chunks (tiny workspace cap) run overlapped on two streams; the
+    # result must be bitwise the one of the serial schedule
+    w = workloads.get("small_layer_bf16")
+    mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
+
+    def run(env):
+        for k, v in env.items():
+            monkeypatch.setenv(k, v)
+        ps = [m[0].clone() for m in mats]
+        gs = [m[1].clone() for m in mats]
+        bs = [m[2].clone() for m in mats]
+        nsg.dmuon_step(ps, gs, bs, wd=0.1)
+        torch.cuda.synchronize()
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        return [bits(t) for t in ps + bs]
+
+    serial = run({"DMUON_OVERLAP": "0", "DMUON_WS_CAP_MB": "20"})
+    nsg.dmuon_release_workspace()
+    over = run({"DMUON_OVERLAP": "1", "DMUON_WS_CAP_MB": "20"})
+    nsg.dmuon_release_workspace()
+    monkeypatch.delenv("DMUON_WS_CAP_MB")
+    monkeypatch.delenv("DMUON_OVERLAP")
+    assert all(np.array_equal(a, b) for a, b in zip(serial, over))
+
+
 def test_step_zero_steps_and_no_nesterov():
     w = workloads.get("small_layer_bf16")
     ps, gs, bs = workloads.make_all(w, DEV)

@@ -144,10 +144,10 @@ bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
 
 // ------------------------------------------------------------ kernel timing
 enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
-            kLoad, kCopyOut, kNumKinds };
+            kLoad, kCopyOut, kSymmTc, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
                                            "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
-                                           "copy_out"};
+                                           "copy_out", "symm_tc"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -229,37 +229,90 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   const bool tc = L.path == Path::kTensorBf16;
   const bool xbf16 = L.path == Path::kSmallBf16;
   const double fm = (double)m, fn = (double)n, fb = (double)b;
-  for (int32_t k = 0; k < steps; ++k) {
-    const float a = sched[3 * k], bb = sched[3 * k + 1], c = sched[3 * k + 2];
+  const int mi = (int)m, ni = (int)n;
+  int* sw = ds.status_word;
+  const int sms = ds.sm_count;
+  cudaError_t e = cudaSuccess;
+  // m x m slot s of the chunk (slot 0 is G, the rest follow P)
+  auto slot = [&](int s) -> char* { return s == 0 ? (char*)G : (char*)P + (int64_t)(s - 1) * ((off.p - off.g)); };
+  auto gram = [&](const void* X, void* out, const float* sc) {
+    Prof p(tc ? kGramTc : kGramFfma, st, fb * fm * fm * fn, 0.0);
+    e = tc ? tc_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, sw, sms, st)
+           : simt_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, xbf16, st);
+    p.done(st);
+  };
+  auto apply = [&](const void* Pm, const void* X, void* Y, float a, const float* sc) {
+    Prof p(tc ? kApplyTc : kApplyFfma, st, 2.0 * fb * fm * fm * fn, 0.0);
+    e = tc ? tc_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, sw, sms, st)
+           : simt_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st);
+    p.done(st);
+  };
+  // C = p1 (A B) + p0 E + p2 I on the tensor path (A, B symmetric and commuting)
+  auto symm = [&](const void* A, const void* B, const void* E, void* C, float p0, float p1, float p2, int kind) {
+    Prof p(kind, st, fb * fm * fm * fm, 0.0);
+    e = tc_symm(A, B, E, C, b, mi, L.ldm, L.ldm, L.ldm, L.ldm, p0, p1, p2, sw, sms, st);
+    p.done(st);
+  };
+  const auto coef = [&](int k, int i) { return sched[3 * k + i]; };
+
+  // Blocks of iterations (chain_blocks).  A block of one is the iteration as
+  // written: G = X X^T, P = b G + c G G, X <- a X + P X.  In a longer block
+  // every matrix is a polynomial of the block's Gram matrix G:
+  //   P_j = p_j(G_j) (with a I),  G_{j+1} = P_j G_j P_j,  Q = P_j ... P_0,
+  // and the block ends with X <- Q X (a fresh G starts the next block).
+  int k = 0;
+  for (int len : chain_blocks(L, steps)) {
+    if (e != cudaSuccess) break;
     const float* sc = k == 0 ? scale : nullptr;
-    cudaError_t e;
-    {
-      Prof p(tc ? kGramTc : kGramFfma, st, fb * fm * fm * fn, 0.0);
-      e = tc ? tc_gram(cur, G, b, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, ds.status_word, ds.sm_count, st)
-             : simt_gram(cur, G, b, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, xbf16, st);
-      p.done(st);
+    if (len == 1) {
+      gram(cur, G, sc);
+      if (e != cudaSuccess) break;
+      {
+        Prof p(tc ? kPolyTc : kPolyFfma, st, fb * fm * fm * fm, 0.0);
+        e = tc ? tc_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), sw, sms, st)
+               : simt_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), st);
+        p.done(st);
+      }
+      if (e != cudaSuccess) break;
+      apply(P, cur, nxt, coef(k, 0), sc);
+      std::swap(cur, nxt);
+      k += 1;
+      continue;
     }
-    if (e == cudaSuccess) {
-      Prof p(tc ? kPolyTc : kPolyFfma, st, fb * fm * fm * fm, 0.0);
-      e = tc ? tc_poly(G, P, b, (int)m, L.ldm, L.ldm, bb, c, ds.status_word, ds.sm_count, st)
-             : simt_poly(G, P, b, (int)m, L.ldm, L.ldm, bb, c, st);
-      p.done(st);
+    char* S0 = slot(0);  // G, G1, G2
+    char* S1 = slot(1);  // P0, P2
+    char* S2 = slot(2);  // T, Q2
+    char* S3 = slot(3);  // P1
+    char* S4 = slot(4);  // Q
+    gram(cur, S0, sc);
+    void* Q = S4;
+    if (e == cudaSuccess) symm(S0, S0, S0, S1, coef(k, 1), coef(k, 2), coef(k, 0), kPolyTc);  // P0
+    if (e == cudaSuccess) symm(S1, S0, nullptr, S2, 0.f, 1.f, 0.f, kSymmTc);                 // T = P0 G
+    if (e == cudaSuccess) symm(S2, S1, nullptr, S0, 0.f, 1.f, 0.f, kSymmTc);                 // G1 = T P0
+    if (e == cudaSuccess) symm(S0, S0, S0, S3, coef(k + 1, 1), coef(k + 1, 2), coef(k + 1, 0), kPolyTc);  // P1
+    if (e == cudaSuccess) symm(S3, S1, nullptr, S4, 0.f, 1.f, 0.f, kSymmTc);                 // Q = P1 P0
+    if (len == 3) {
+      if (e == cudaSuccess) symm(S3, S0, nullptr, S2, 0.f, 1.f, 0.f, kSymmTc);  // T = P1 G1
+      if (e == cudaSuccess) symm(S2, S3, nullptr, S0, 0.f, 1.f, 0.f, kSymmTc);  // G2 = T P1
+      if (e == cudaSuccess) symm(S0, S0, S0, S1, coef(k + 2, 1), coef(k + 2, 2), coef(k + 2, 0), kPolyTc);  // P2
+      if (e == cudaSuccess) symm(S1, S4, nullptr, S2, 0.f, 1.f, 0.f, kSymmTc);  // Q2 = P2 Q
+      Q = S2;
     }
-    if (e == cudaSuccess) {
-      Prof p(tc ? kApplyTc : kApplyFfma, st, 2.0 * fb * fm * fm * fn, 0.0);
-      e = tc ? tc_apply(P, cur, nxt, b, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, ds.status_word,
-                        ds.sm_count, st)
-             : simt_apply(P, cur, nxt, b, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st);
-      p.done(st);
-    }
-    if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
+    if (e == cudaSuccess) apply(Q, cur, nxt, 0.f, sc);  // X <- Q X (scaled by s when k == 0)
     std::swap(cur, nxt);
+    k += len;
   }
+  if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
   *result = cur;
   return DMUON_OK;
 }
 
-int64_t chunk_launches(int32_t steps) { return 3 + 3 * (int64_t)steps; }
+// Kernels one chunk launches: momentum, norm, the chain, update.
+int64_t chunk_launches_for(const ChunkLayout& L, int32_t steps) {
+  int64_t n = 3;
+  for (int len : chain_blocks(L, steps)) n += len == 1 ? 3 : (len == 2 ? 7 : 11);  // gram + products + apply
+  return n;
+}
 
 }  // namespace
 
@@ -304,7 +357,10 @@ int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_
 
 int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
   if (count <= 0 || !shapes) return 0;
-  return (int64_t)make_step_plan(shapes, count).chunks.size() * chunk_launches(ns_steps);
+  const StepPlan P = make_step_plan(shapes, count);
+  int64_t n = 0;
+  for (const ChunkRef& ck : P.chunks) n += chunk_launches_for(P.layouts[ck.cls], ns_steps);
+  return n;
 }
 
 dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,

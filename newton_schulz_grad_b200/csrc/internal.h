@@ -85,6 +85,11 @@ cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx
                     float alpha, const float* scale, int* status, int num_sms, cudaStream_t st);
 cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b,
                     float c, int* status, int num_sms, cudaStream_t st);
+// C = p1 (A B) + p0 E + p2 I for symmetric, commuting A, B (E may be NULL);
+// one triangle computed, mirrored.
+cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int batch, int m, int64_t lda,
+                    int64_t ldb, int64_t lde, int64_t ldc, float p0, float p1, float p2, int* status,
+                    int num_sms, cudaStream_t st);
 cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
                      int64_t ldx, int64_t ldy, float a, float alpha, const float* scale,
                      int* status, int num_sms, cudaStream_t st);
@@ -114,12 +119,20 @@ std::vector<LaunchClass> plan_classes(const std::vector<Group>& groups);
 // Per-chunk workspace layout of a launch class.
 struct ChunkLayout {
   Path path;
+  bool blocked;            // Gram-space blocks of iterations (tensor path, n >= 1.25 m)
+  int gslots;              // m x m buffers: 2 (G, P) or 5 (blocked)
   int64_t ldn, ldm;        // row pitches (elements) of X and of G/P
   int64_t xbytes, gbytes;  // bytes of one X (one matrix) and of one G
   int64_t tiles_per_mat;   // elementwise tiles
   int64_t per_matrix;      // workspace bytes per matrix in a chunk
 };
-ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype);
+// allow_blocked = false keeps the per-iteration form (two m x m buffers).
+ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype, bool allow_blocked = true);
+// Iteration blocks of the chain for `steps` iterations: all 1 in the
+// per-iteration form; otherwise the Gram-space schedule of DMUON_GRAM_BLOCKS
+// (default: per-iteration steps, then the last two iterations as one block;
+// "2": blocks of 2, 3, 3, ...).
+std::vector<int> chain_blocks(const ChunkLayout& L, int32_t steps);
 int64_t workspace_cap_bytes();
 int64_t chunk_size(const ChunkLayout& L, int64_t members, int64_t cap);
 // Offsets of the pieces of a chunk of `b` matrices inside the workspace.

@@ -81,7 +81,7 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
   const uintptr_t bytes = (uintptr_t)(rows * cols * es), x = (uintptr_t)X, o = (uintptr_t)out;
   if (x < o + bytes && o < x + bytes) return record_error(DMUON_ERR_INVALID_ARG, "out may not overlap X");
   const int64_t m = std::min(rows, cols), n = std::max(rows, cols);
-  const ChunkLayout L = chunk_layout(m, n, dtype);
+  const ChunkLayout L = chunk_layout(m, n, dtype, /*allow_blocked=*/false);
   const ChunkOffsets off = chunk_offsets(L, 1);
   const size_t need = kHeader + (size_t)off.total;
   if (need > (size_t)DMUON_NOALLOC_SCRATCH_BYTES)

@@ -49,12 +49,26 @@ std::vector<LaunchClass> plan_classes(const std::vector<Group>& groups) {
 
 static int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
-ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype) {
+// DMUON_GRAM_BLOCKS: "0" per-iteration form only; unset/"1" the last two
+// iterations in Gram space; "2" blocks of 2, 3, 3, ... (fewest flops, least
+// accurate on ill-conditioned matrices).
+static int gram_block_mode() {
+  const char* e = std::getenv("DMUON_GRAM_BLOCKS");
+  if (e && e[0] == '0') return 0;
+  if (e && e[0] == '2') return 2;
+  return 1;
+}
+
+ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype, bool allow_blocked) {
   ChunkLayout L{};
   if (dtype == DMUON_F32)
     L.path = Path::kF32;
   else
     L.path = (m <= kSmallM) ? Path::kSmallBf16 : Path::kTensorBf16;
+  // Gram-space blocks cost 3 m^2 n + (4L - 3) m^3 per block of L iterations
+  // against L (3 m^2 n + m^3) iteration by iteration: fewer flops once n > m.
+  L.blocked = allow_blocked && gram_block_mode() != 0 && L.path == Path::kTensorBf16 && 4 * n >= 5 * m;
+  L.gslots = L.blocked ? 5 : 2;
   const int64_t xs = dtype == DMUON_BF16 ? 2 : 4;
   const int64_t gs = L.path == Path::kTensorBf16 ? 2 : 4;
   // 16-byte row pitch: the TMA descriptors need it, vector loads like it
@@ -63,7 +77,7 @@ ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype) {
   L.xbytes = m * L.ldn * xs;
   L.gbytes = m * L.ldm * gs;
   L.tiles_per_mat = ((m + kElemTile - 1) / kElemTile) * ((n + kElemTile - 1) / kElemTile);
-  L.per_matrix = 2 * L.xbytes + 2 * L.gbytes + L.tiles_per_mat * 4 + 4 + 6 * 256;
+  L.per_matrix = 2 * L.xbytes + L.gslots * L.gbytes + L.tiles_per_mat * 4 + 4 + 6 * 256;
   return L;
 }
 
@@ -113,13 +127,33 @@ StepPlan make_step_plan(const dmuon_shape_t* shapes, int32_t count) {
   return P;
 }
 
+std::vector<int> chain_blocks(const ChunkLayout& L, int32_t steps) {
+  std::vector<int> b;
+  const int mode = L.blocked ? gram_block_mode() : 0;
+  if (mode == 0 || steps < 2) {
+    b.assign(steps, 1);
+  } else if (mode == 1) {
+    // Gram space squares the singular values, so bf16 rounding there hurts
+    // small ones; by the last two iterations they have grown by a^(steps-2).
+    b.assign(steps - 2, 1);
+    b.push_back(2);
+  } else {
+    for (int k = 0, first = 1; k < steps; first = 0) {
+      const int len = std::min(first ? 2 : 3, steps - k);
+      b.push_back(len);
+      k += len;
+    }
+  }
+  return b;
+}
+
 ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b) {
   ChunkOffsets o{};
   int64_t at = 0;
   o.x0 = at; at += round_up(b * L.xbytes, 256);
   o.x1 = at; at += round_up(b * L.xbytes, 256);
   o.g = at; at += round_up(b * L.gbytes, 256);
-  o.p = at; at += round_up(b * L.gbytes, 256);
+  o.p = at; at += round_up(b * L.gbytes, 256) * (L.gslots - 1);
   o.partials = at; at += round_up(b * L.tiles_per_mat * 4, 256);
   o.scale = at; at += round_up(b * 4, 256);
   o.total = at;

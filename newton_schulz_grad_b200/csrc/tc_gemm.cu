@@ -6,6 +6,10 @@
 //   gram:  G = alpha X X^T        m x m, K = n   (symmetric: one triangle)
 //   poly:  P = b G + c G G        m x m, K = m   (G symmetric => G G = G G^T,
 //                                                  one triangle again)
+// The poly kernel is the general symmetric product C = p1 (A B) + p0 E + p2 I
+// for symmetric, commuting A and B (so A B is symmetric and B's rows are its
+// columns): the Gram-space form of the chain multiplies polynomials of one
+// Gram matrix this way.
 //   apply: Y = alpha (a X + P X)  m x n, K = m   (X is the MN-major operand)
 //
 // Two kernels share the tile decode and the epilogue:
@@ -83,7 +87,7 @@ struct TcArgs {
   int m, n, k;
   int tm;  // tile rows: 128 (one CTA) or 256 (CTA pair)
   int tiles_m, tiles_n, tiles_per_mat, total_tiles;
-  float p0, p1;
+  float p0, p1, p2;  // gram: alpha; poly: p1 (A B) + p0 E + p2 I; apply: alpha (p0 X + P X)
   const float* scale;
   int* status;
 };
@@ -330,7 +334,7 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, uint32_t taddr, in
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]);
     const bool full_chunk = c0 + 32 <= a.n;
-    if (MODE == kApply || MODE == kPoly) {
+    if ((MODE == kApply && a.p0 != 0.f) || (MODE == kPoly && Em != nullptr)) {
       float e[32];
       const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
       if (full_chunk) {
@@ -347,9 +351,17 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, uint32_t taddr, in
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = fmaf(a.p1, v[j], a.p0 * e[j]);
       }
+    } else if (MODE == kPoly) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = a.p1 * v[j];
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = alpha * v[j];
+    }
+    if (MODE == kPoly && a.p2 != 0.f && r >= c0 && r < c0 + 32) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j == r) v[j] += a.p2;
     }
     __nv_bfloat16* rowp = Cm + (int64_t)r * a.ldc + c0;
     if (MODE == kApply) {
@@ -819,30 +831,37 @@ cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx
   return launch<kGram>(ma, mb, a, batch, num_sms, pair, st);
 }
 
-cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b, float c,
-                    int* status, int num_sms, cudaStream_t st) {
+cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int batch, int m, int64_t lda,
+                    int64_t ldb, int64_t lde, int64_t ldc, float p0, float p1, float p2, int* status, int num_sms,
+                    cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
   const bool pair = use_pair(m);
   CUtensorMap ma, mb;
-  cudaError_t e = make_map(&ma, G, m, m, batch, ldg, BK, 128);
-  if (e == cudaSuccess) e = make_map(&mb, G, m, m, batch, ldg, BK, pair ? 128 : BN);
+  cudaError_t e = make_map(&ma, A, m, m, batch, lda, BK, 128);
+  if (e == cudaSuccess) e = make_map(&mb, B, m, m, batch, ldb, BK, pair ? 128 : BN);
   if (e != cudaSuccess) return e;
   TcArgs a{};
-  a.C = static_cast<__nv_bfloat16*>(P);
-  a.E = static_cast<const __nv_bfloat16*>(G);
-  a.sC = (int64_t)m * ldp;
-  a.sE = (int64_t)m * ldg;
-  a.ldc = ldp;
-  a.lde = ldg;
+  a.C = static_cast<__nv_bfloat16*>(C);
+  a.E = static_cast<const __nv_bfloat16*>(E);
+  a.sC = (int64_t)m * ldc;
+  a.sE = (int64_t)m * lde;
+  a.ldc = ldc;
+  a.lde = lde;
   a.m = m; a.n = m; a.k = m;
   a.tm = pair ? BM2 : BM1;
   a.tiles_m = (m + a.tm - 1) / a.tm;
   a.tiles_n = (m + BN - 1) / BN;
   a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
-  a.p0 = b;
-  a.p1 = c;
+  a.p0 = p0;
+  a.p1 = p1;
+  a.p2 = p2;
   a.status = status;
   return launch<kPoly>(ma, mb, a, batch, num_sms, pair, st);
+}
+
+cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b, float c,
+                    int* status, int num_sms, cudaStream_t st) {
+  return tc_symm(G, G, G, P, batch, m, ldg, ldg, ldg, ldp, b, c, 0.f, status, num_sms, st);
 }
 
 cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,

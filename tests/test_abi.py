@@ -58,12 +58,19 @@ def test_plan_groups_on_workloads(w):
 def test_launch_count_and_workspace_llama7b():
     w = workloads.get("llama_7b_bf16")
     shapes = [(r, c, 1) for r, c in w.shapes]
-    # classes: 4096x4096 (128 matrices, 128 MiB of workspace each) and
-    # 4096x11008 oriented (gate/up transposed + down: 96 matrices, 244 MiB
-    # each).  Several chunks -> overlapped execution with two buffers of half
-    # the 8 GiB cap: 5 chunks of <= 26 and 6 chunks of 16; per chunk momentum
-    # + norm + 3 per iteration + update
-    assert nsg.dmuon_step_launches(shapes, 5) == 11 * (3 + 15)
+    # classes: 4096x4096 (128 matrices, 128 MiB of workspace each, one
+    # iteration at a time) and 4096x11008 oriented (gate/up transposed + down:
+    # 96 matrices; three iterations one at a time, then the last two as one
+    # Gram-space block; five m x m slots: 340 MiB each).  Several chunks ->
+    # overlapped execution with two buffers of half the 8 GiB cap: 5 chunks of
+    # <= 26 and 8 chunks of 12.  Per chunk: momentum + norm + update, plus 3 per
+    # single iteration and gram + 5 products + apply for the block of two.
+    assert nsg.dmuon_step_launches(shapes, 5) == 5 * (3 + 15) + 8 * (3 + 9 + 7)
+    os.environ["DMUON_GRAM_BLOCKS"] = "2"
+    try:  # blocks of 2 and 3: gram + 5 products + apply, gram + 9 products + apply
+        assert nsg.dmuon_step_launches(shapes, 5) == 5 * (3 + 15) + 8 * (3 + 7 + 11)
+    finally:
+        del os.environ["DMUON_GRAM_BLOCKS"]
     ws = nsg.dmuon_workspace_bytes(shapes, 5)
     assert 5 << 30 < ws <= 8 << 30
 
@@ -72,6 +79,7 @@ def test_overlap_can_be_disabled(monkeypatch):
     w = workloads.get("llama_7b_bf16")
     shapes = [(r, c, 1) for r, c in w.shapes]
     monkeypatch.setenv("DMUON_OVERLAP", "0")
+    monkeypatch.setenv("DMUON_GRAM_BLOCKS", "0")
     assert nsg.dmuon_step_launches(shapes, 5) == 6 * (3 + 15)
     assert nsg.dmuon_workspace_bytes(shapes, 5) <= 8 << 30
 

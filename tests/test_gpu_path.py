@@ -64,6 +64,33 @@ def test_ns_custom_coefficients_and_zero_steps(dtype):
     assert rel_fro(to64(out), om.newton_schulz(to64(X), 0)) < (4e-3 if dtype == torch.bfloat16 else 1e-6)
 
 
+@pytest.mark.parametrize("mode", ["1", "2"])
+@pytest.mark.parametrize("steps", [1, 2, 3, 4, 6, 12])
+def test_ns_gram_space_blocks_match_oracle(steps, mode, monkeypatch):
+    # wide bf16 matrices run their last two iterations as one Gram-space block
+    # (mode 1, the default) or all of them in blocks of 2, 3, 3, ... (mode 2):
+    # every block length and remainder appears across these steps
+    monkeypatch.setenv("DMUON_GRAM_BLOCKS", mode)
+    X = lowrank_plus_noise(300, 700, 21 + steps, torch.bfloat16, rank=32, noise=1e-2)
+    out = torch.empty_like(X)
+    coeffs = [(3.4445, -4.7750, 2.0315), (2.5, -2.0, 0.6), (1.5, -0.5, 0.0)] * 4
+    nsg.dmuon_ns(X, out, steps=steps, coeffs=coeffs[:steps])
+    c32 = [tuple(float(np.float32(v)) for v in t) for t in coeffs[:steps]]
+    assert rel_fro(to64(out), om.newton_schulz(to64(X), steps, c32)) < 2e-2
+
+
+def test_ns_gram_space_and_per_iteration_forms_agree(monkeypatch):
+    X = lowrank_plus_noise(1024, 2816, 3, torch.bfloat16, rank=64, noise=1e-3)
+    a, b = torch.empty_like(X), torch.empty_like(X)
+    nsg.dmuon_ns(X, a)
+    monkeypatch.setenv("DMUON_GRAM_BLOCKS", "0")
+    nsg.dmuon_ns(X, b)
+    torch.cuda.synchronize()
+    want = om.newton_schulz(to64(X), 5)
+    assert rel_fro(to64(a), want) < 2e-2 and rel_fro(to64(b), want) < 2e-2
+    assert rel_fro(to64(a), to64(b)) < 3e-2
+
+
 def test_ns_convergent_polynomial_reaches_polar_factor():
     X = lowrank_plus_noise(128, 256, 9, torch.float32, rank=128, noise=1e-2)
     out = torch.empty_like(X)

@@ -158,6 +158,13 @@ def test_step_small_layer_bf16():
     run_step_check(workloads.get("small_layer_bf16"))
 
 
+def test_step_llama3_2_3b_sampled():
+    # one matrix of each shape class (q 3072^2, k 1024x3072, gate 8192x3072
+    # transposed, down 3072x8192) plus a last-layer up_proj; wd = 0.1
+    w = workloads.get("llama3_2_3b_bf16")
+    run_step_check(w, [0, 1, 4, 6, w.count - 2])
+
+
 def test_step_moe_sampled():
     w = workloads.get("moe_skewed_bf16")
     sk = workloads.skewed_indices(w)

@@ -76,26 +76,47 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def traffic_record(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it still matches the source."""
+def launches_per_matrix(kernel: str, m: int, n: int, dtype: str, steps: int):
+    """How many launches of `kernel` one matrix of oriented shape m x n sees in
+    a step (the library's default schedule: wide bf16 matrices on the tensor
+    path run their last two iterations as one Gram-space block)."""
+    if kernel != "apply_tc" or dtype != "bf16" or m <= 64:
+        return None
+    mode = os.environ.get("DMUON_GRAM_BLOCKS", "1")[:1]
+    blocked = mode != "0" and 4 * n >= 5 * m and steps >= 2
+    if blocked and mode == "2":
+        return None
+    return steps - 1 if blocked else steps
+
+
+def traffic_record(kernel: str, w, launches: int):
+    """Average DRAM bytes per launch of `kernel` in one step of workload w, from
+    the committed per-matrix ncu figures, or None if they do not cover it or
+    the kernel source changed since they were taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f)
+            ent = json.load(f).get(kernel)
     except (OSError, ValueError):
         return None
-    ent = rec.get(f"{kernel}@{workload}")
-    if not ent:
+    if not ent or launches <= 0:
         return None
     src = os.path.join(ROOT, "newton_schulz_grad_b200", "csrc", ent.get("source", ""))
     try:
         with open(src, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
+            if hashlib.sha256(f.read()).hexdigest() != ent.get("sha256"):
+                return None
     except OSError:
         return None
-    if digest != ent.get("sha256"):
-        return None  # the kernel changed since the counters were taken
-    return ent.get("bytes_per_launch")
+    per = ent.get("bytes_per_matrix", {})
+    total = 0.0
+    for r, c in w.shapes:
+        m, n = min(r, c), max(r, c)
+        k = launches_per_matrix(kernel, m, n, w.dtype, w.ns_steps)
+        if k is None or f"{m}x{n}" not in per:
+            return None
+        total += k * per[f"{m}x{n}"]
+    return total / launches
 
 
 # ------------------------------------------------------------------ clocks
@@ -381,7 +402,7 @@ def run_ours(args):
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
         "roofline": {"kernel": dname, "bound": bound, "achieved": round(achieved, 1), "peak": peak,
                      "unit": unit, "frac": round(achieved / peak, 4),
-                     "traffic": traffic_record(dname, w.name),
+                     "traffic": traffic_record(dname, w, d["launches"] // max(1, args.steps)),
                      "per_launch": {"flops": d["flops"] / d["launches"],
                                     "bytes": d["bytes"] / d["launches"], "avg_ms": avg_ms}},
         "elementwise": elem,

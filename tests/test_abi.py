@@ -17,7 +17,8 @@ NO_GPU = not torch.cuda.is_available()
 
 
 def declared_symbols():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     return sorted(set(re.findall(r"DMUON_API\s+[\w\s\*]+?\b(dmuon_\w+)\s*\(", text)))
 
 

@@ -55,6 +55,8 @@ def parse_args(argv=None):
                     help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--ns-steps", type=int, default=None,
                     help="override the workload's Newton-Schulz iteration count")
     ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update"],
@@ -290,17 +292,33 @@ def run_ours(args):
     gp = [t.data_ptr() for t in gs]
     bp = [t.data_ptr() for t in bs]
     stream = torch.cuda.current_stream(dev)
+    # graph capture needs a non-default stream; the library keeps one
+    # workspace per stream, so warm-up and capture use the same one
+    run_stream = torch.cuda.Stream(dev) if args.graph else stream
     launches_per_step = nsg.dmuon_step_launches(shapes, w.ns_steps)
 
     def step():
         nsg.dmuon_step_ptrs(pp, gp, bp, shapes, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
-                            ns_steps=w.ns_steps, wd=w.wd, stream=stream)
+                            ns_steps=w.ns_steps, wd=w.wd, stream=run_stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
-    st = nsg.dmuon_stream_status(stream)
+    st = nsg.dmuon_stream_status(run_stream)
     if st != nsg.DMUON_OK:
         raise RuntimeError(f"warm-up failed: {nsg.STATUS_NAMES[st]} {nsg.dmuon_get_last_error()}")
+    eager_step = step
+    if args.graph:
+        # one step captured once (after the warm-up allocated the workspace);
+        # the timed loop replays it on the timing stream
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=run_stream):
+            eager_step()
+
+        def step():  # noqa: F811
+            graph.replay()
+        step()
+        torch.cuda.synchronize(dev)
 
     if pg:
         pg.barrier()
@@ -316,6 +334,14 @@ def run_ours(args):
     e1.record(stream)
     e1.synchronize()
     kstats = nsg.dmuon_profile_stop()
+    if args.graph:
+        # replays bypass the library's event timing: break the kernels down on
+        # eager steps right after the timed region
+        torch.cuda.synchronize(dev)
+        nsg.dmuon_profile_start()
+        for _ in range(args.steps):
+            eager_step()
+        kstats = nsg.dmuon_profile_stop()
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
@@ -412,6 +438,7 @@ def run_ours(args):
         "elementwise_isolated": elem_iso,
         "kernels": kernels,
         "gpu_launches": launches_per_step * args.steps,
+        "cuda_graph": bool(args.graph),
         "clocks": clk,
     }
     if e2e is not None:

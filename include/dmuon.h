@@ -247,6 +247,14 @@ DMUON_API const char* dmuon_get_last_error(void);
  * last call, DMUON_ERR_CUDA if the stream reports an error, else DMUON_OK. */
 DMUON_API dmuon_status_t dmuon_stream_status(dmuon_stream_t stream);
 
+/* Self-test of failure detection: launches one thread that waits on a device
+ * barrier nothing will arrive on, with the same bounded wait the tensor-core
+ * kernels use, limited to limit_us (1..2000000) microseconds.  The wait gives
+ * up, records DMUON_ERR_TIMEOUT in the device status word and the kernel
+ * returns; the next dmuon_stream_status() reports DMUON_ERR_TIMEOUT and clears
+ * the word, and the context stays usable. */
+DMUON_API dmuon_status_t dmuon_selftest_timeout(int32_t limit_us, dmuon_stream_t stream);
+
 /* Frees every cached workspace of the calling thread's current device after
  * synchronising the device.  Safe to call at any time between calls. */
 DMUON_API void dmuon_release_workspace(void);

@@ -35,7 +35,7 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_gram_poly", "dmuon_poly_apply", "dmuon_momentum", "dmuon_update",
             "dmuon_get_last_error", "dmuon_stream_status", "dmuon_release_workspace",
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
-            "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc")
+            "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout")
 
 
 class DmuonError(RuntimeError):
@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_profile_start": ([], i32),
         "dmuon_profile_stop": ([ctypes.POINTER(KernelStat), i32], i32),
         "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
+        "dmuon_selftest_timeout": ([i32, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -326,6 +327,11 @@ def dmuon_update(param: torch.Tensor, O: torch.Tensor, lr: float, wd: float = 0.
 def dmuon_stream_status(stream=None) -> int:
     """Synchronise the stream and return (without raising) the library status."""
     return int(_lib.dmuon_stream_status(_stream(stream)))
+
+
+def dmuon_selftest_timeout(limit_us: int = 50000, stream=None) -> None:
+    """Launch a kernel whose bounded device wait is made to run out (see dmuon.h)."""
+    _check(_lib.dmuon_selftest_timeout(int(limit_us), _stream(stream)))
 
 
 def dmuon_get_last_error() -> str:

@@ -768,6 +768,15 @@ int32_t dmuon_profile_stop(dmuon_kernel_stat_t* stats, int32_t max_stats) {
   return n;
 }
 
+dmuon_status_t dmuon_selftest_timeout(int32_t limit_us, dmuon_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000) return fail(DMUON_ERR_INVALID_ARG, "limit_us must be in 1..2000000");
+  DeviceState ds;
+  dmuon_status_t rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  cudaError_t e = wait_selftest(ds.status_word, limit_us, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "self-test launch");
+}
+
 dmuon_status_t dmuon_stream_status(dmuon_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);

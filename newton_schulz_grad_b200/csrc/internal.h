@@ -94,6 +94,8 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
                      int64_t ldx, int64_t ldy, float a, float alpha, const float* scale,
                      int* status, int num_sms, cudaStream_t st);
 const char* tc_config_string();
+// One-thread kernel whose bounded wait runs out after limit_us (status word).
+cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st);
 
 // ---- api.cu -------------------------------------------------------------------
 // Sets the message returned by dmuon_get_last_error on this thread; returns s.

@@ -141,7 +141,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait; false when the limit ran out or another thread already failed.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status) {
+__device__ __noinline__ bool wait_bar_limit(uint32_t bar, uint32_t parity, int* status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
   while (true) {
@@ -149,11 +149,24 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status
     for (int i = 0; i < 128; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*reinterpret_cast<volatile int*>(status) != 0) return false;
-    if (global_timer() - t0 > kTimeoutNs) {
+    if (global_timer() - t0 > limit_ns) {
       atomicCAS(status, 0, (int)DMUON_ERR_TIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status) {
+  return wait_bar_limit(bar, parity, status, kTimeoutNs);
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// arrives on; the wait gives up after limit_ns and records the timeout.
+__global__ void k_wait_selftest(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  wait_bar_limit(b, 0, status, limit_ns);
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
                                             int c1, int c2) {
@@ -890,6 +903,11 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
   a.scale = scale;
   a.status = status;
   return launch<kApply>(ma, mb, a, batch, num_sms, pair, st);
+}
+
+cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st) {
+  k_wait_selftest<<<1, 1, 0, st>>>(status, (uint64_t)limit_us * 1000ull);
+  return cudaGetLastError();
 }
 
 const char* tc_config_string() {

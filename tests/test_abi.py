@@ -128,6 +128,7 @@ def test_stage_validation_errors():
     assert lib.dmuon_ns_ex(A, A + 4096, 4, 4, -2, None, 1, None) == nsg.DMUON_ERR_INVALID_ARG
     assert lib.dmuon_momentum(A, A + 4096, A + 8192, 4, 4, 0.9, 3, 1, None, None) == nsg.DMUON_ERR_INVALID_ARG
     assert lib.dmuon_update(A, 0, 4, 4, 0.1, 0.0, 1, None) == nsg.DMUON_ERR_INVALID_ARG
+    assert lib.dmuon_selftest_timeout(0, None) == nsg.DMUON_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(not NO_GPU, reason="checks the no-device path")

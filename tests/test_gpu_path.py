@@ -253,3 +253,47 @@ def test_step_injected_allocation_failure_leaves_inputs(monkeypatch):
 def test_step_empty_list():
     nsg.dmuon_step([], [], [])
     assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+
+
+def test_bounded_device_wait_reports_timeout_and_context_survives():
+    # a wait on a barrier that nothing arrives on gives up after 50 ms
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    nsg.dmuon_selftest_timeout(50000)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_ERR_TIMEOUT
+    assert "ran out" in nsg.dmuon_get_last_error()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK       # the word was cleared
+    X = lowrank_plus_noise(256, 512, 3, torch.bfloat16)     # the context still works
+    out = torch.empty_like(X)
+    nsg.dmuon_ns(X, out)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    assert rel_fro(to64(out), om.newton_schulz(to64(X), 5)) < 2e-2
+
+
+@pytest.mark.parametrize("name", ["small_layer_bf16", "single_256x512_f32"])
+def test_step_replays_from_a_cuda_graph(name):
+    # after one eager call (workspace and internal stream exist) a step can be
+    # captured into a CUDA graph; replays give the eager step's bits
+    w = workloads.get(name)
+    mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
+    eager = [[t.clone() for t in m] for m in mats]
+    graphed = [[t.clone() for t in m] for m in mats]
+
+    def step(sets, stream=None):
+        nsg.dmuon_step([m[0] for m in sets], [m[1] for m in sets], [m[2] for m in sets],
+                       lr=w.lr, wd=0.05, stream=stream)
+
+    step(eager)                    # warm-up: allocations happen here
+    step(eager)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        step(graphed, stream=side)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    for a, b in zip(eager, graphed):
+        for x, y in zip(a, b):
+            assert np.array_equal(bits(x), bits(y))

@@ -95,7 +95,10 @@ typedef struct {
  *   coeffs HOST array of 3*steps floats (a_k, b_k, c_k for iteration k), or
  *          NULL for the default triple at every iteration
  * Works over the smaller side (transposes internally when rows > cols).
- * Uses the library's cached workspace for this (device, stream).
+ * Uses the library's cached workspace for this (device, stream).  When
+ * max(rows, cols) >= 1.25 min(rows, cols) and the tensor path runs, the last
+ * two iterations are carried out as one block in Gram space (the same result
+ * in exact arithmetic, fewer flops); see dmuon_gram_poly.
  */
 DMUON_API dmuon_status_t dmuon_ns(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,
                         const float* coeffs, dmuon_stream_t stream);
@@ -119,7 +122,13 @@ DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int
  *   ns_steps  >= 0 (default 5); coeffs as for dmuon_ns
  *   wd     decoupled weight decay: p <- p (1 - lr wd) - ...
  * Matrices are grouped by shape (dmuon_plan_groups) and each group runs as
- * batched launches.
+ * batched launches.  The library's workspace (cached per device and stream,
+ * at most DMUON_WS_CAP_MB, default 8 GiB) is allocated stream-ordered on
+ * first use or growth; after one call with the same shapes, a call allocates
+ * nothing and can be captured in a CUDA graph.  With several chunks the
+ * momentum and update stages run on an internal stream underneath the
+ * Newton-Schulz chain and are joined back into `stream` before the call's
+ * work ends; the results do not depend on that schedule.
  */
 DMUON_API dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
                           const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
@@ -160,7 +169,9 @@ DMUON_API dmuon_status_t dmuon_gram(const void* X, void* G, int64_t batch, int64
 
 /*
  * dmuon_gram_poly - P = b G + c G G for a symmetric G (so that
- * p(G) = a I + P).  One triangle computed, the other mirrored.
+ * p(G) = a I + P).  One triangle computed, the other mirrored.  The kernel
+ * behind it computes the general symmetric product p1 (A B) + p0 E + p2 I of
+ * commuting symmetric A, B, which the Gram-space block uses internally.
  *   G  device, batch x m x m (ldg); P device, batch x m x m (ldp), no overlap
  */
 DMUON_API dmuon_status_t dmuon_gram_poly(const void* G, void* P, int64_t batch, int64_t m, int64_t ldg,

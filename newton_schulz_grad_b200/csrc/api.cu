@@ -4,9 +4,19 @@
 // dmuon_step (DMuon Training Guide, "Step 4": momentum + NS + update for the
 // dedicated parameters) runs, per launch class (same oriented shape and
 // dtype) and per chunk of at most 256 matrices that fits the workspace cap:
-//   momentum+norm partials -> norm finalise -> ns_steps x (gram, poly, apply)
-//   -> update
-// all enqueued on the caller's stream with no host synchronisation.
+//   momentum+norm partials -> norm finalise -> the Newton-Schulz chain
+//   (ns_steps x (gram, poly, apply); wide matrices on the tensor path run
+//   their last two iterations as one Gram-space block) -> update
+// With several chunks the elementwise stages run on an internal stream
+// underneath the chains of neighbouring chunks (two workspace buffers),
+// ordered by events and joined back into the caller's stream; there is no
+// host synchronisation.
+//
+// Environment switches (read per call): DMUON_WS_CAP_MB (workspace cap,
+// default 8 GiB), DMUON_OVERLAP=0 (serial schedule), DMUON_GRAM_BLOCKS=0|2
+// (per-iteration form | Gram-space blocks of 2, 3, 3, ...),
+// DMUON_TC_CTA_PAIR=0 (one-CTA tensor-core kernel only, read once),
+// DMUON_FAULT_INJECT=alloc (workspace allocation fails, for tests).
 #include <cuda_runtime.h>
 
 #include <algorithm>

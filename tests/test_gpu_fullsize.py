@@ -40,3 +40,30 @@ def test_llama7b_full_step_sampled_parity():
     # every parameter moved and stayed finite
     for p in ps:
         assert torch.isfinite(p).all()
+
+
+@pytest.mark.parametrize("shape", [(16384, 24576), (24576, 16384)])
+def test_large_diagonal_closed_form(shape):
+    # X = [D | 0] (or its transpose) with D diagonal: every product stays
+    # diagonal, so at any size NS(X) = diag(f^5(d_i / ||d||)) exactly in real
+    # arithmetic, with f(s) = a s + b s^3 + c s^5, and exact zeros elsewhere.
+    # 16384 x 24576 runs every tile of the CTA-pair kernels and the Gram-space
+    # block (n >= 1.25 m).
+    R, C = shape
+    m = min(R, C)
+    d = (1.0 + torch.arange(m, dtype=torch.float32) / m).to(torch.bfloat16)
+    X = torch.zeros(R, C, dtype=torch.bfloat16, device="cuda")
+    X.diagonal().copy_(d.cuda())
+    out = torch.full_like(X, float("nan"))
+    nsg.dmuon_ns(X, out, steps=5)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    dd = d.double().numpy()
+    s = dd / (np.linalg.norm(dd) + om.NORM_EPS)
+    a, b, c = (float(np.float32(v)) for v in om.DEFAULT_COEFFS)
+    for _ in range(5):
+        s = a * s + b * s ** 3 + c * s ** 5
+    got = out.diagonal().double().cpu().numpy()
+    assert np.linalg.norm(got - s) / np.linalg.norm(s) < 2e-2
+    total = float(out.double().pow(2).sum().item())
+    assert abs(total - float(np.sum(got ** 2))) <= 1e-12 * total   # nothing off the diagonal
+    assert torch.isfinite(out).all()

@@ -16,6 +16,7 @@
 // default 8 GiB), DMUON_OVERLAP=0 (serial schedule), DMUON_GRAM_BLOCKS=0|2
 // (per-iteration form | Gram-space blocks of 2, 3, 3, ...),
 // DMUON_TC_CTA_PAIR=0 (one-CTA tensor-core kernel only, read once),
+// DMUON_SMALL_CHAIN=0 (thin matrices on the per-product FFMA kernels),
 // DMUON_FAULT_INJECT=alloc (workspace allocation fails, for tests).
 #include <cuda_runtime.h>
 
@@ -80,6 +81,11 @@ dmuon_status_t device_state(DeviceState* out) {
   }
   *out = it->second;
   return DMUON_OK;
+}
+
+bool env_is(const char* name, char first) {
+  const char* e = std::getenv(name);
+  return e && e[0] == first;
 }
 
 bool fault_injected(const char* what) {
@@ -154,10 +160,10 @@ bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
 
 // ------------------------------------------------------------ kernel timing
 enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
-            kLoad, kCopyOut, kSymmTc, kNumKinds };
+            kLoad, kCopyOut, kSymmTc, kChainSmall, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
                                            "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
-                                           "copy_out", "symm_tc"};
+                                           "copy_out", "symm_tc", "chain_small"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -264,6 +270,17 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
     p.done(st);
   };
   const auto coef = [&](int k, int i) { return sched[3 * k + i]; };
+
+  // thin matrices: the whole chain in one clustered launch, in place on X0
+  if (!tc && m <= kSmallM && steps >= 1 && steps <= 16 &&
+      n <= small_ns_max_n((int)m, xbf16 ? 2 : 4) && !env_is("DMUON_SMALL_CHAIN", '0')) {
+    Prof p(kChainSmall, st, fb * (3.0 * fm * fm * fn + fm * fm * fm) * steps, 0.0);
+    e = small_ns(cur, b, mi, ni, L.ldn, steps, sched.data(), scale, xbf16, st);
+    p.done(st);
+    if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
+    *result = cur;
+    return DMUON_OK;
+  }
 
   // Blocks of iterations (chain_blocks).  A block of one is the iteration as
   // written: G = X X^T, P = b G + c G G, X <- a X + P X.  In a longer block

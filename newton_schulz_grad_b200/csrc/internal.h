@@ -79,6 +79,16 @@ cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, 
                        int64_t ldp, int64_t ldx, int64_t ldy, float a, float alpha,
                        const float* scale, bool xbf16, cudaStream_t st);
 
+// ---- small_ns.cu -------------------------------------------------------------
+// The whole chain for min side m <= 64 in one launch: one cluster of 8 CTAs per
+// matrix, X's columns split over the CTAs and kept in shared memory, the fp32
+// Gram matrix all-reduced over distributed shared memory each iteration.  X (in
+// place, batch pitch m*ld) holds x0 on entry and the result on exit.
+// Valid for steps <= 16 and n <= small_ns_max_n(m, element size).
+int small_ns_max_n(int m, size_t es);
+cudaError_t small_ns(void* X, int batch, int m, int n, int64_t ld, int steps, const float* coeffs,
+                     const float* scale, bool xbf16, cudaStream_t st);
+
 // ---- tc_gemm.cu -------------------------------------------------------------
 // tcgen05 chain kernels (bf16 in/out, fp32 accumulation in TMEM).
 cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,

@@ -297,3 +297,24 @@ def test_step_replays_from_a_cuda_graph(name):
     for a, b in zip(eager, graphed):
         for x, y in zip(a, b):
             assert np.array_equal(bits(x), bits(y))
+
+
+@pytest.mark.parametrize("shape,dtype", [((32, 4096), torch.bfloat16), ((4096, 32), torch.bfloat16),
+                                         ((64, 1000), torch.bfloat16), ((16, 20000), torch.bfloat16),
+                                         ((64, 9000), torch.bfloat16), ((64, 12000), torch.bfloat16),
+                                         ((48, 4801), torch.float32), ((7, 300), torch.float32),
+                                         ((1, 300), torch.bfloat16)], ids=str)
+def test_thin_matrix_chain_matches_oracle_fused_and_unfused(shape, dtype, monkeypatch):
+    # m <= 64 runs the whole chain in one clustered launch when the columns fit
+    # the cluster's shared memory (64 x 12000 does not and falls back)
+    X = lowrank_plus_noise(*shape, seed=sum(shape), dtype=dtype, rank=8, noise=1e-2)
+    want = om.newton_schulz(to64(X), 5)
+    fused = torch.empty_like(X)
+    nsg.dmuon_ns(X, fused)
+    monkeypatch.setenv("DMUON_SMALL_CHAIN", "0")
+    plain = torch.empty_like(X)
+    nsg.dmuon_ns(X, plain)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    tol = NS_TOL[dtype]
+    assert rel_fro(to64(fused), want) < tol
+    assert rel_fro(to64(plain), want) < tol

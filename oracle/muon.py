@@ -155,6 +155,29 @@ def muon_step(params: Sequence[np.ndarray], grads: Sequence[np.ndarray],
     return out_p, out_b, out_o
 
 
+# Reading (the Training Guide's "Gradient Clipping" section names global p-norm
+# clipping of the Muon gradients and pairs it with PyTorch's clip_grad_norm_):
+# the same formula, 1e-6 added to the norm, coefficient clamped to 1.
+CLIP_EPS: float = 1e-6
+
+
+def clip_grad_norm(grads: Sequence[np.ndarray], max_norm: float, norm_type: float = 2.0):
+    """Global p-norm clipping of a list of gradients.
+
+    total = (sum_i sum |g|^p)^(1/p) (p = inf: max |g|); coef = min(1, max_norm /
+    (total + 1e-6)); returns (clipped gradients, total, coef).  Training Guide,
+    "Gradient Clipping": after the reduce, before momentum + Newton-Schulz.
+    """
+    gs = [np.asarray(g, dtype=np.float64) for g in grads]
+    if norm_type == float("inf"):
+        total = max((float(np.max(np.abs(g))) if g.size else 0.0) for g in gs) if gs else 0.0
+    else:
+        p = float(norm_type)
+        total = sum(float(np.sum(np.abs(g) ** p)) for g in gs) ** (1.0 / p)
+    coef = min(1.0, max_norm / (total + CLIP_EPS))
+    return [g * coef for g in gs], total, coef
+
+
 def shape_groups(shapes: Sequence[Tuple[int, int, int]]):
     """Partition matrices by (rows, cols, dtype).
 

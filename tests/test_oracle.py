@@ -320,3 +320,38 @@ def test_pins_catch_planted_update_mistakes():
              p - 0.1 * s * o]                                                 # no decay
     for w in wrong:
         assert not np.allclose(w, want, atol=1e-12)
+
+
+
+# ---------------------------------------------------------------- clipping
+def test_clip_hand_computed_l2():
+    g1 = np.array([[3.0, 4.0]])
+    g2 = np.array([[0.0, 12.0]])
+    out, total, coef = om.clip_grad_norm([g1, g2], 6.5)
+    assert total == 13.0
+    assert abs(coef - 6.5 / (13.0 + 1e-6)) < 1e-15
+    assert np.allclose(out[0], g1 * 6.5 / (13.0 + 1e-6)) and np.allclose(out[1], g2 * coef)
+
+
+def test_clip_below_threshold_is_identity():
+    g = gauss((3, 5), 1)
+    out, total, coef = om.clip_grad_norm([g], 1e6)
+    assert coef == 1.0 and np.array_equal(out[0], g)
+    assert abs(total - np.linalg.norm(g)) < 1e-12
+
+
+def test_clip_inf_and_l1_norms():
+    g1 = np.array([[1.0, -7.0]])
+    g2 = np.array([[2.0, 0.5], [-3.0, 0.0]])
+    _, t_inf, c_inf = om.clip_grad_norm([g1, g2], 3.5, float("inf"))
+    assert t_inf == 7.0 and abs(c_inf - 3.5 / (7.0 + 1e-6)) < 1e-15
+    _, t_1, _ = om.clip_grad_norm([g1, g2], 1.0, 1.0)
+    assert t_1 == 1.0 + 7.0 + 2.0 + 0.5 + 3.0
+
+
+def test_clip_global_norm_couples_matrices():
+    # the clip is global: a large gradient also shrinks a small one
+    small, big = np.full((2, 2), 1e-3), np.full((2, 2), 100.0)
+    out, total, coef = om.clip_grad_norm([small, big], 1.0)
+    assert abs(total - np.sqrt(4 * 1e-6 + 4 * 1e4)) < 1e-9
+    assert np.allclose(out[0], small * coef) and coef < 0.01

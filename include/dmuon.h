@@ -136,6 +136,44 @@ DMUON_API dmuon_status_t dmuon_step(void* const* params, const void* const* grad
                           dmuon_stream_t stream);
 
 /*
+ * dmuon_step_clipped - dmuon_step on globally clipped gradients (DMuon
+ * Training Guide, "Gradient Clipping": clip after the reduce, before
+ * momentum + Newton-Schulz).  One norm pass reads every gradient, one block
+ * forms coef = min(1, max_norm / (total + 1e-6)); the momentum kernel then
+ * uses fl_T(g * fl32(coef)) (fl_T: rounding to the gradient's own dtype) in
+ * place of g.  The result equals dmuon_clip_grad_norm followed by dmuon_step,
+ * bit for bit, but the gradients are NOT modified (read-only, as in
+ * dmuon_step) and no scaled copy is written.  Arguments as dmuon_step, plus
+ * max_norm / norm_type / total_norm as dmuon_clip_grad_norm.
+ */
+DMUON_API dmuon_status_t dmuon_step_clipped(void* const* params, const void* const* grads, void* const* mom_bufs,
+                                            const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
+                                            int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
+                                            float max_norm, float norm_type, double* total_norm,
+                                            dmuon_stream_t stream);
+
+/*
+ * dmuon_clip_grad_norm - global p-norm clipping of the Muon gradients, in
+ * place (DMuon Training Guide, "Gradient Clipping": the Muon-only clip runs
+ * after the gradient reduce and before momentum + Newton-Schulz; the default
+ * strategy is global p-norm clipping).  Read with PyTorch's clip_grad_norm_
+ * formula, which the same section pairs it with:
+ *   total = (sum over every element of every matrix of |g|^p)^(1/p)
+ *           (p = inf: max |g|)
+ *   coef  = min(1, max_norm / (total + 1e-6)),  g <- fl(g * fl32(coef))
+ * Every gradient is rewritten; with coef = 1 the values are unchanged.
+ *   grads      HOST array of `count` DEVICE pointers (shapes[i], row-major)
+ *   shapes     HOST array of `count` shapes; gradients must not overlap
+ *   max_norm   finite, >= 0
+ *   norm_type  1, 2 or INFINITY (others: DMUON_ERR_UNSUPPORTED)
+ *   total_norm DEVICE double or NULL: receives `total`
+ * Deterministic (fixed-order fp64 reduction of per-tile fp32 partials).
+ */
+DMUON_API dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* shapes, int32_t count,
+                                              float max_norm, float norm_type, double* total_norm,
+                                              dmuon_stream_t stream);
+
+/*
  * dmuon_plan_groups - the shape grouping dmuon_step uses (host only, no GPU).
  * Matrices with equal (rows, cols, dtype) form a group; group ids follow
  * first appearance; `order` lists the groups one after another, members in

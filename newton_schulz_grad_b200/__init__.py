@@ -35,7 +35,8 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_gram_poly", "dmuon_poly_apply", "dmuon_momentum", "dmuon_update",
             "dmuon_get_last_error", "dmuon_stream_status", "dmuon_release_workspace",
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
-            "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout")
+            "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout",
+            "dmuon_clip_grad_norm", "dmuon_step_clipped")
 
 
 class DmuonError(RuntimeError):
@@ -67,6 +68,8 @@ def _load() -> ctypes.CDLL:
         "dmuon_ns_ex": ([vp, vp, i64, i64, i32, fp, i32, vp], i32),
         "dmuon_step": ([ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                         ctypes.POINTER(Shape), i32, f32, f32, i32, i32, fp, f32, vp], i32),
+        "dmuon_step_clipped": ([ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                ctypes.POINTER(Shape), i32, f32, f32, i32, i32, fp, f32, f32, f32, vp, vp], i32),
         "dmuon_plan_groups": ([ctypes.POINTER(Shape), i32, ctypes.POINTER(i32),
                                ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
         "dmuon_gram": ([vp, vp, i64, i64, i64, i64, i64, f32, i32, vp], i32),
@@ -84,6 +87,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_profile_stop": ([ctypes.POINTER(KernelStat), i32], i32),
         "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
         "dmuon_selftest_timeout": ([i32, vp], i32),
+        "dmuon_clip_grad_norm": ([ctypes.POINTER(vp), ctypes.POINTER(Shape), i32, f32, f32, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -208,8 +212,13 @@ def dmuon_ns_noalloc(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=
 def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
                mom_bufs: Sequence[torch.Tensor], lr: float = 0.02, momentum: float = 0.95,
                nesterov: bool = True, ns_steps: int = 5, coeffs=None, wd: float = 0.0,
-               stream=None) -> None:
-    """One Muon step over lists of 2D tensors; params and mom_bufs updated in place."""
+               stream=None, max_norm: Optional[float] = None, norm_type: float = 2.0,
+               total_norm: Optional[torch.Tensor] = None) -> None:
+    """One Muon step over lists of 2D tensors; params and mom_bufs updated in place.
+
+    With ``max_norm`` set, the call is dmuon_step_clipped: the gradients are
+    clipped by their global ``norm_type`` norm inside the step (not in memory).
+    """
     n = len(params)
     if len(grads) != n or len(mom_bufs) != n:
         raise ValueError("params, grads and mom_bufs must have the same length")
@@ -228,8 +237,15 @@ def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
     ga = (vp * max(1, n))(*[t.data_ptr() for t in grads])
     ba = (vp * max(1, n))(*[t.data_ptr() for t in mom_bufs])
     c = _coeffs(ns_steps, coeffs)
-    _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
-                           ns_steps, c, wd, _stream(stream)))
+    if max_norm is None:
+        _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
+                               ns_steps, c, wd, _stream(stream)))
+        return
+    if total_norm is not None and (total_norm.dtype != torch.float64 or not total_norm.is_cuda):
+        raise ValueError("total_norm must be a CUDA float64 tensor")
+    _check(_lib.dmuon_step_clipped(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
+                                   ns_steps, c, wd, float(max_norm), float(norm_type), _ptr(total_norm),
+                                   _stream(stream)))
 
 
 def dmuon_step_ptrs(params: Sequence[int], grads: Sequence[int], mom_bufs: Sequence[int],
@@ -244,6 +260,23 @@ def dmuon_step_ptrs(params: Sequence[int], grads: Sequence[int], mom_bufs: Seque
     ba = (vp * max(1, n))(*mom_bufs)
     _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
                            ns_steps, _coeffs(ns_steps, coeffs), wd, _stream(stream)))
+
+
+def dmuon_clip_grad_norm(grads: Sequence[torch.Tensor], max_norm: float, norm_type: float = 2.0,
+                         total_norm: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Global p-norm clipping of the gradients, in place (see dmuon.h)."""
+    shapes = []
+    for g in grads:
+        _need_cuda(g)
+        if g.dim() != 2 or not g.is_contiguous():
+            raise ValueError("gradients must be contiguous 2D tensors")
+        shapes.append((g.shape[0], g.shape[1], _dtype_code(g)))
+    if total_norm is not None and (total_norm.dtype != torch.float64 or not total_norm.is_cuda):
+        raise ValueError("total_norm must be a CUDA float64 tensor")
+    n = len(grads)
+    ga = (ctypes.c_void_p * max(1, n))(*[g.data_ptr() for g in grads])
+    _check(_lib.dmuon_clip_grad_norm(ga, _shape_array(shapes), n, float(max_norm), float(norm_type),
+                                     _ptr(total_norm), _stream(stream)))
 
 
 def dmuon_plan_groups(shapes: Sequence[Tuple[int, int, int]]):

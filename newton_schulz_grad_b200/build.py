@@ -25,7 +25,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libdmuon_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 
-SOURCES = ["api.cu", "plan.cpp", "elementwise.cu", "simt_gemm.cu", "tc_gemm.cu", "noalloc.cu", "small_ns.cu"]
+SOURCES = ["api.cu", "plan.cpp", "elementwise.cu", "simt_gemm.cu", "tc_gemm.cu", "noalloc.cu", "small_ns.cu", "clip.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",
           "-I", INCLUDE, "-I", CSRC]

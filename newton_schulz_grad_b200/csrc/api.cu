@@ -160,10 +160,10 @@ bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
 
 // ------------------------------------------------------------ kernel timing
 enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
-            kLoad, kCopyOut, kSymmTc, kChainSmall, kNumKinds };
+            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
                                            "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
-                                           "copy_out", "symm_tc", "chain_small"};
+                                           "copy_out", "symm_tc", "chain_small", "clip_norm", "clip_scale"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -341,59 +341,86 @@ int64_t chunk_launches_for(const ChunkLayout& L, int32_t steps) {
   return n;
 }
 
-}  // namespace
+// ----------------------------------------------------------- gradient clipping
 
-dmuon_status_t record_error(dmuon_status_t s, const std::string& msg) { return fail(s, msg); }
+struct ClipReq {
+  int p;            // 2, 1, or 0 for the infinity norm
+  float max_norm;
+  double* total;    // device, optional
+};
 
-}  // namespace dmuon
-
-using namespace dmuon;
-
-extern "C" {
-
-const char* dmuon_get_last_error(void) { return g_last_error.c_str(); }
-
-const char* dmuon_build_info(void) {
-  static std::string s = std::string("dmuon-b200 0.1.0; sm_100a; ") + tc_config_string() +
-                         "; FFMA chain for fp32 and min side <= 64; elementwise 64x64 tiles";
-  return s.c_str();
-}
-
-dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int32_t* group_of,
-                                 int32_t* order, int32_t* num_groups) {
-  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
-  if (!num_groups || (count > 0 && (!shapes || !group_of || !order)))
-    return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
-  std::vector<Group> groups = plan_groups(shapes, count);
-  int32_t pos = 0;
-  for (size_t g = 0; g < groups.size(); ++g)
-    for (int32_t i : groups[g].members) {
-      group_of[i] = (int32_t)g;
-      order[pos++] = i;
-    }
-  *num_groups = (int32_t)groups.size();
+dmuon_status_t parse_clip(float max_norm, float norm_type, int* p) {
+  if (!std::isfinite(max_norm) || max_norm < 0.f) return fail(DMUON_ERR_INVALID_ARG, "max_norm must be finite and >= 0");
+  if (norm_type == 2.f) *p = 2;
+  else if (norm_type == 1.f) *p = 1;
+  else if (std::isinf(norm_type) && norm_type > 0.f) *p = 0;
+  else return fail(DMUON_ERR_UNSUPPORTED, "norm_type must be 1, 2 or inf");
   return DMUON_OK;
 }
 
-int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
-  (void)ns_steps;
-  if (count <= 0 || !shapes) return 0;
-  const StepPlan P = make_step_plan(shapes, count);
-  return P.buffer_bytes * (P.overlap ? 2 : 1);
+int64_t tiles_of(int64_t rows, int64_t cols) {
+  return ((rows + kElemTile - 1) / kElemTile) * ((cols + kElemTile - 1) / kElemTile);
 }
 
-int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
-  if (count <= 0 || !shapes) return 0;
-  const StepPlan P = make_step_plan(shapes, count);
-  int64_t n = 0;
-  for (const ChunkRef& ck : P.chunks) n += chunk_launches_for(P.layouts[ck.cls], ns_steps);
-  return n;
+int64_t clip_tiles(const std::vector<Group>& groups) {
+  int64_t t = 0;
+  for (const Group& g : groups) t += (int64_t)g.members.size() * tiles_of(g.rows, g.cols);
+  return t;
 }
 
-dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
-                          const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
-                          int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
-                          dmuon_stream_t stream) {
+// Bytes of clip workspace: one fp32 partial per 64x64 tile, then the coefficient.
+size_t clip_ws_bytes(int64_t tiles) { return (size_t)(((tiles * 4 + 15) / 16) * 16 + 16); }
+float* clip_coef_ptr(void* ws, int64_t tiles) {
+  return reinterpret_cast<float*>(static_cast<char*>(ws) + ((tiles * 4 + 15) / 16) * 16);
+}
+
+// Calls fn(table, dtype, partials offset, bytes) for every table of at most
+// kMaxTable matrices of one source shape (src = buf = the gradient).
+template <typename Fn>
+cudaError_t for_each_clip_table(const std::vector<Group>& groups, const void* const* grads, ElemTable* tab, Fn&& fn) {
+  int64_t offset = 0;
+  for (const Group& g : groups) {
+    const size_t es = esize(g.dtype);
+    const int32_t tpm = (int32_t)tiles_of(g.rows, g.cols);
+    for (size_t start = 0; start < g.members.size(); start += kMaxTable) {
+      const int b = (int)std::min<size_t>(kMaxTable, g.members.size() - start);
+      tab->m = g.rows;
+      tab->n = g.cols;
+      tab->ldn = g.cols;
+      tab->count = b;
+      tab->tiles_per_mat = tpm;
+      for (int j = 0; j < b; ++j) {
+        const int32_t i = g.members[start + j];
+        const bool row16 = (g.cols * (int64_t)es) % 16 == 0 && aligned16(grads[i]);
+        tab->e[j] = MatEntry{grads[i], const_cast<void*>(grads[i]), nullptr, 0, row16 ? 1 : 0};
+      }
+      cudaError_t e = fn(*tab, g.dtype, offset, (double)b * (double)g.rows * (double)g.cols * (double)es);
+      if (e != cudaSuccess) return e;
+      offset += (int64_t)b * tpm;
+    }
+  }
+  return cudaSuccess;
+}
+
+// The norm pass and the coefficient: coef = min(1, max_norm / (total + 1e-6)).
+cudaError_t clip_norm_stage(const std::vector<Group>& groups, const void* const* grads, const ClipReq& req,
+                            void* ws, int64_t tiles, ElemTable* tab, cudaStream_t st) {
+  float* partials = static_cast<float*>(ws);
+  cudaError_t e = for_each_clip_table(groups, grads, tab, [&](const ElemTable& t, int32_t dtype, int64_t off, double bytes) {
+    Prof pr(kClipNorm, st, 0.0, bytes);
+    cudaError_t r = launch_clip_partials(t, dtype, req.p, partials + off, st);
+    pr.done(st);
+    return r;
+  });
+  if (e == cudaSuccess) e = launch_clip_coef(partials, tiles, req.p, req.max_norm, clip_coef_ptr(ws, tiles), req.total, st);
+  return e;
+}
+
+
+dmuon_status_t step_impl(void* const* params, const void* const* grads, void* const* mom_bufs,
+                         const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
+                         int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
+                         const ClipReq* clip, dmuon_stream_t stream) {
   // ---------------------------------------------------------- validation
   if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
   if (ns_steps < 0 || ns_steps > 1000) return fail(DMUON_ERR_INVALID_ARG, "ns_steps must be in 0..1000");
@@ -428,9 +455,25 @@ dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* c
   if (rc != DMUON_OK) return rc;
   const StepPlan P = make_step_plan(shapes, count);
   const int nbuf = P.overlap ? 2 : 1;
+  // clipping: one fp32 partial per gradient tile and the coefficient, after the chunk buffers
+  std::vector<Group> clip_groups;
+  int64_t clip_tile_count = 0;
+  const size_t clip_off = (((size_t)P.buffer_bytes * nbuf + 255) / 256) * 256;
+  if (clip) {
+    clip_groups = plan_groups(shapes, count);
+    clip_tile_count = clip_tiles(clip_groups);
+  }
   void* wsv = nullptr;
-  rc = get_workspace((size_t)(P.buffer_bytes * nbuf), st, &wsv);
+  rc = get_workspace(clip ? clip_off + clip_ws_bytes(clip_tile_count) : (size_t)(P.buffer_bytes * nbuf), st, &wsv);
   if (rc != DMUON_OK) return rc;
+  std::unique_ptr<ElemTable[]> tabs(new ElemTable[2]);
+  const float* clip_coef = nullptr;
+  if (clip) {
+    void* cws = static_cast<char*>(wsv) + clip_off;
+    cudaError_t e = clip_norm_stage(clip_groups, grads, *clip, cws, clip_tile_count, &tabs[0], st);
+    if (e != cudaSuccess) return cuda_fail(e, "clip norm launch");
+    clip_coef = clip_coef_ptr(cws, clip_tile_count);
+  }
   // elementwise stages run on `aux` when overlapping, else on the caller's stream
   cudaStream_t aux = st;
   if (P.overlap) {
@@ -439,7 +482,6 @@ dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* c
     cudaError_t e = stream_after(aux, st);
     if (e != cudaSuccess) return cuda_fail(e, "stream fork");
   }
-  std::unique_ptr<ElemTable[]> tabs(new ElemTable[2]);
   std::vector<void*> results(P.chunks.size(), nullptr);
 
   auto fill_table = [&](const ChunkRef& ck, ElemTable& tab) {
@@ -496,7 +538,7 @@ dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* c
     const double elems = (double)ck.b * (double)c.m * (double)c.n;
     Prof pm(kMomentum, aux, 0.0, 4.0 * elems * (double)esize(c.dtype));
     cudaError_t e = launch_momentum(tabs[i % 2], c.dtype, ElemMode::kMomentum, ws + off.x0, partials, momentum,
-                                    nesterov, aux);
+                                    nesterov, aux, clip_coef);
     pm.done(aux);
     if (e != cudaSuccess) {
       drop();
@@ -550,6 +592,120 @@ dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* c
     if (e != cudaSuccess) return cuda_fail(e, "stream join");
   }
   return DMUON_OK;
+}
+
+}  // namespace
+
+dmuon_status_t record_error(dmuon_status_t s, const std::string& msg) { return fail(s, msg); }
+
+}  // namespace dmuon
+
+using namespace dmuon;
+
+extern "C" {
+
+const char* dmuon_get_last_error(void) { return g_last_error.c_str(); }
+
+const char* dmuon_build_info(void) {
+  static std::string s = std::string("dmuon-b200 0.1.0; sm_100a; ") + tc_config_string() +
+                         "; FFMA chain for fp32 and min side <= 64; elementwise 64x64 tiles";
+  return s.c_str();
+}
+
+dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int32_t* group_of,
+                                 int32_t* order, int32_t* num_groups) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
+  if (!num_groups || (count > 0 && (!shapes || !group_of || !order)))
+    return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  std::vector<Group> groups = plan_groups(shapes, count);
+  int32_t pos = 0;
+  for (size_t g = 0; g < groups.size(); ++g)
+    for (int32_t i : groups[g].members) {
+      group_of[i] = (int32_t)g;
+      order[pos++] = i;
+    }
+  *num_groups = (int32_t)groups.size();
+  return DMUON_OK;
+}
+
+int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
+  (void)ns_steps;
+  if (count <= 0 || !shapes) return 0;
+  const StepPlan P = make_step_plan(shapes, count);
+  return P.buffer_bytes * (P.overlap ? 2 : 1);
+}
+
+int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
+  if (count <= 0 || !shapes) return 0;
+  const StepPlan P = make_step_plan(shapes, count);
+  int64_t n = 0;
+  for (const ChunkRef& ck : P.chunks) n += chunk_launches_for(P.layouts[ck.cls], ns_steps);
+  return n;
+}
+
+
+
+dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
+                          const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
+                          int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
+                          dmuon_stream_t stream) {
+  return step_impl(params, grads, mom_bufs, shapes, count, lr, momentum, nesterov, ns_steps, coeffs, wd,
+                   nullptr, stream);
+}
+
+dmuon_status_t dmuon_step_clipped(void* const* params, const void* const* grads, void* const* mom_bufs,
+                                  const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
+                                  int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
+                                  float max_norm, float norm_type, double* total_norm,
+                                  dmuon_stream_t stream) {
+  ClipReq req{0, max_norm, total_norm};
+  dmuon_status_t rc = parse_clip(max_norm, norm_type, &req.p);
+  if (rc != DMUON_OK) return rc;
+  return step_impl(params, grads, mom_bufs, shapes, count, lr, momentum, nesterov, ns_steps, coeffs, wd,
+                   &req, stream);
+}
+
+dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* shapes, int32_t count,
+                                    float max_norm, float norm_type, double* total_norm,
+                                    dmuon_stream_t stream) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
+  ClipReq req{0, max_norm, total_norm};
+  dmuon_status_t rc = parse_clip(max_norm, norm_type, &req.p);
+  if (rc != DMUON_OK) return rc;
+  if (count == 0) return DMUON_OK;
+  if (!grads || !shapes) return fail(DMUON_ERR_INVALID_ARG, "null array argument");
+  std::vector<Interval> iv;
+  for (int32_t i = 0; i < count; ++i) {
+    rc = check_shape(shapes[i].rows, shapes[i].cols, "dmuon_clip_grad_norm");
+    if (rc != DMUON_OK) return rc;
+    if (!dtype_ok(shapes[i].dtype) || shapes[i].reserved != 0)
+      return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": bad dtype or reserved field");
+    if (!grads[i]) return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": null pointer");
+    const uintptr_t bytes = (uintptr_t)(shapes[i].rows * shapes[i].cols) * esize(shapes[i].dtype);
+    iv.push_back({(uintptr_t)grads[i], (uintptr_t)grads[i] + bytes, i});
+  }
+  if (any_overlap(iv)) return fail(DMUON_ERR_INVALID_ARG, "gradients must not overlap");
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  const std::vector<Group> groups = plan_groups(shapes, count);
+  const int64_t tiles = clip_tiles(groups);
+  void* ws = nullptr;
+  rc = get_workspace(clip_ws_bytes(tiles), st, &ws);
+  if (rc != DMUON_OK) return rc;
+  std::unique_ptr<ElemTable> tab(new ElemTable());
+  const void* const* cg = const_cast<const void* const*>(grads);
+  cudaError_t e = clip_norm_stage(groups, cg, req, ws, tiles, tab.get(), st);
+  if (e == cudaSuccess)
+    e = for_each_clip_table(groups, cg, tab.get(), [&](const ElemTable& t, int32_t dtype, int64_t, double bytes) {
+      Prof pr(kClipScale, st, 0.0, 2.0 * bytes);
+      cudaError_t r = launch_clip_scale(t, dtype, clip_coef_ptr(ws, tiles), st);
+      pr.done(st);
+      return r;
+    });
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_clip_grad_norm");
 }
 
 dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,

@@ -27,10 +27,13 @@ __device__ __forceinline__ int clamp8(int64_t v) { return v < 8 ? (int)v : 8; }
 
 // 8 resident blocks per SM (<= 32 registers): the extra block keeps more
 // loads in flight (measured +12 % bandwidth over the unbounded build).
-template <typename T, int MODE>
-__global__ void __launch_bounds__(kThreads, 8)
+// CLIP: the gradient is first scaled by the global clipping coefficient and
+// rounded to the storage type, exactly the value a separate in-place clip
+// would have stored, so a fused clipped step equals clip-then-step bit for bit.
+template <typename T, int MODE, bool CLIP>
+__global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
     k_momentum(const __grid_constant__ ElemTable tab, T* __restrict__ X, float* __restrict__ partials,
-               float mu, int nesterov, int dst_vec) {
+               float mu, int nesterov, int dst_vec, const float* __restrict__ clip_coef) {
   __shared__ float s[T64][T64 + 1];
   __shared__ float red[kThreads / 32];
   const int e = blockIdx.y;
@@ -63,6 +66,11 @@ __global__ void __launch_bounds__(kThreads, 8)
       const int64_t off = gr * C + gc;
       float gv[8];
       load8<T>(g + off, gv, v8, valid);
+      if (CLIP) {
+        const float k = *clip_coef;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) gv[i] = round_to<T>(__fmul_rn(gv[i], k));
+      }
       if (MODE == (int)ElemMode::kMomentum) {
         float bv[8], nb[8];
         load8<T>(buf + off, bv, v8, valid);
@@ -216,23 +224,28 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 cudaError_t launch_momentum(const ElemTable& t, int dtype, ElemMode mode, void* X, float* partials,
-                            float mu, int nesterov, cudaStream_t st) {
+                            float mu, int nesterov, cudaStream_t st, const float* clip_coef) {
   if (t.count == 0) return cudaSuccess;
+  if (clip_coef && mode != ElemMode::kMomentum) return cudaErrorInvalidValue;
   const size_t es = dtype == DMUON_BF16 ? 2 : 4;
   const int dst_vec = ((t.ldn * (int64_t)es) % 16 == 0) && aligned16(X);
   dim3 grid((unsigned)t.tiles_per_mat, (unsigned)t.count);
   if (dtype == DMUON_BF16) {
     auto* x = static_cast<__nv_bfloat16*>(X);
-    if (mode == ElemMode::kMomentum)
-      k_momentum<__nv_bfloat16, 0><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec);
+    if (clip_coef)
+      k_momentum<__nv_bfloat16, 0, true><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, clip_coef);
+    else if (mode == ElemMode::kMomentum)
+      k_momentum<__nv_bfloat16, 0, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
     else
-      k_momentum<__nv_bfloat16, 1><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec);
+      k_momentum<__nv_bfloat16, 1, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
   } else {
     auto* x = static_cast<float*>(X);
-    if (mode == ElemMode::kMomentum)
-      k_momentum<float, 0><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec);
+    if (clip_coef)
+      k_momentum<float, 0, true><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, clip_coef);
+    else if (mode == ElemMode::kMomentum)
+      k_momentum<float, 0, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
     else
-      k_momentum<float, 1><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec);
+      k_momentum<float, 1, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
   }
   return cudaGetLastError();
 }

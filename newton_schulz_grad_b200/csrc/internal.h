@@ -54,8 +54,10 @@ enum class Path : int {
 // Momentum (or load) stage: writes x0 into X (batch pitch m*ldn elements,
 // transposed where the entry says so) and one fp32 sum-of-squares partial per
 // 64x64 tile into `partials` (tiles_per_mat per matrix).
+// clip_coef (device float, kMomentum only): scale each gradient by it first.
 cudaError_t launch_momentum(const ElemTable& t, int dtype, ElemMode mode, void* X,
-                            float* partials, float mu, int nesterov, cudaStream_t st);
+                            float* partials, float mu, int nesterov, cudaStream_t st,
+                            const float* clip_coef = nullptr);
 // Sum the partials of each matrix in a fixed order; scale[i] = 1/(sqrt(sum)+eps).
 // sumsq (optional) receives the sums in fp64.
 cudaError_t launch_norm_finalize(const float* partials, int count, int tiles_per_mat,
@@ -78,6 +80,15 @@ cudaError_t simt_poly(const void* G, void* P, int batch, int m, int64_t ldg, int
 cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, int n,
                        int64_t ldp, int64_t ldx, int64_t ldy, float a, float alpha,
                        const float* scale, bool xbf16, cudaStream_t st);
+
+// ---- clip.cu --------------------------------------------------------------------
+// Global p-norm clipping (p = 0 means the infinity norm).  Tables hold
+// matrices of one source shape (m = rows, n = cols, not oriented); `src` is
+// read for the norm, `buf` scaled in place.
+cudaError_t launch_clip_partials(const ElemTable& t, int dtype, int p, float* partials, cudaStream_t st);
+cudaError_t launch_clip_coef(const float* partials, int64_t count, int p, float max_norm, float* coef,
+                             double* total, cudaStream_t st);
+cudaError_t launch_clip_scale(const ElemTable& t, int dtype, const float* coef, cudaStream_t st);
 
 // ---- small_ns.cu -------------------------------------------------------------
 // The whole chain for min side m <= 64 in one launch: one cluster of 8 CTAs per

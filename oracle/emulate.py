@@ -86,4 +86,5 @@ def update_fp32(p: np.ndarray, o: np.ndarray, lr: float, wd: float, dtype: str):
 def clip_scale_fp32(g: np.ndarray, coef: float, dtype: str) -> np.ndarray:
     """Stored g * coef: the coefficient rounded to fp32 once, one fp32 product."""
     g = np.asarray(g, dtype=np.float32)
-    return store((g * np.float32(coef)).astype(np.float32), dtype)
+    with np.errstate(invalid="ignore"):  # inf * 0
+        return store((g * np.float32(coef)).astype(np.float32), dtype)

@@ -170,12 +170,16 @@ def clip_grad_norm(grads: Sequence[np.ndarray], max_norm: float, norm_type: floa
     """
     gs = [np.asarray(g, dtype=np.float64) for g in grads]
     if norm_type == float("inf"):
-        total = max((float(np.max(np.abs(g))) if g.size else 0.0) for g in gs) if gs else 0.0
+        # np.max keeps a NaN wherever it sits (Python's max would drop it)
+        per = [np.max(np.abs(g)) for g in gs if g.size]
+        total = float(np.max(per)) if per else 0.0
     else:
         p = float(norm_type)
         total = sum(float(np.sum(np.abs(g) ** p)) for g in gs) ** (1.0 / p)
+    # a NaN total leaves coef at 1 (min(1, nan) keeps its first argument)
     coef = min(1.0, max_norm / (total + CLIP_EPS))
-    return [g * coef for g in gs], total, coef
+    with np.errstate(invalid="ignore"):
+        return [g * coef for g in gs], total, coef
 
 
 def shape_groups(shapes: Sequence[Tuple[int, int, int]]):

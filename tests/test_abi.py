@@ -137,3 +137,41 @@ def test_valid_call_without_device_reports_cuda_error():
     rc = _raw_step(1, [A], [A + 4096], [A + 8192], [(4, 8, 1)])
     assert rc in (nsg.DMUON_ERR_CUDA, nsg.DMUON_ERR_UNSUPPORTED)
     assert nsg.dmuon_get_last_error()
+
+
+def _raw_clip(count, ptrs, shapes, max_norm=1.0, norm_type=2.0):
+    lib = nsg.library()
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))(*ptrs)
+    return lib.dmuon_clip_grad_norm(arr, nsg._shape_array(shapes), count, max_norm, norm_type, None, None)
+
+
+def test_clip_validation_errors():
+    A = 1 << 40
+    ok = [(4, 8, 1)]
+    assert _raw_clip(0, [], []) == nsg.DMUON_OK
+    assert _raw_clip(-1, [A], ok) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_clip(1, [0], ok) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_clip(1, [A], [(4, 8, 5)]) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_clip(1, [A], [(0, 8, 1)]) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_clip(1, [A], ok, max_norm=float("nan")) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_clip(1, [A], ok, max_norm=-1.0) == nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_clip(1, [A], ok, norm_type=3.0) == nsg.DMUON_ERR_UNSUPPORTED
+    assert _raw_clip(1, [A], ok, norm_type=float("-inf")) == nsg.DMUON_ERR_UNSUPPORTED
+    # 4 x 8 bf16 = 64 bytes: the second gradient starts inside the first
+    assert _raw_clip(2, [A, A + 32], ok * 2) == nsg.DMUON_ERR_INVALID_ARG
+    assert "overlap" in nsg.dmuon_get_last_error()
+
+
+def test_step_clipped_validation_errors():
+    lib = nsg.library()
+    A = 1 << 40
+    vp = ctypes.c_void_p
+
+    def call(max_norm, norm_type, shapes=((4, 8, 1),)):
+        pa, ga, ba = (vp * 1)(A), (vp * 1)(A + 4096), (vp * 1)(A + 8192)
+        return lib.dmuon_step_clipped(pa, ga, ba, nsg._shape_array(list(shapes)), 1, 0.02, 0.95, 1, 5,
+                                      None, 0.0, max_norm, norm_type, None, None)
+    assert call(float("inf"), 2.0) == nsg.DMUON_ERR_INVALID_ARG
+    assert call(-0.5, 2.0) == nsg.DMUON_ERR_INVALID_ARG
+    assert call(1.0, 0.5) == nsg.DMUON_ERR_UNSUPPORTED
+    assert call(1.0, 2.0, ((4, 8, 9),)) == nsg.DMUON_ERR_INVALID_ARG

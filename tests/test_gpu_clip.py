@@ -1,0 +1,177 @@
+"""Global p-norm gradient clipping on the GPU against the fp64 oracle.
+
+DMuon Training Guide, "Gradient Clipping": the Muon gradients are clipped by
+their global p-norm after the reduce and before momentum + Newton-Schulz.
+The norm is compared with the oracle's fp64 norm (per-tile fp32 partials,
+then a fixed-order fp64 sum: relative error ~ sqrt(64*64) fp32 roundings at
+most, bounded here by 1e-5); the scaled values are compared bit for bit with
+the fp32 rounding contract fl(g * fl32(coef)), with the coefficient the GPU
+read back, and the coefficient itself with the oracle's to 1e-5.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_grad_b200 as nsg
+from oracle import emulate as em
+from oracle import muon as om
+from tests.gpu_util import bits, dtype_name, to64
+
+pytestmark = pytest.mark.gpu
+
+MIXED = [(64, 64), (100, 37), (4096, 11008), (257, 129), (1, 1), (33, 1000), (130, 136)]
+
+
+def make_grads(shapes, dtype, seed, scale=1.0):
+    gen = torch.Generator().manual_seed(seed)
+    out = []
+    for r, c in shapes:
+        t = torch.randn(r, c, generator=gen) * scale
+        out.append(t.to(dtype).cuda())
+    return out
+
+
+def check_clip(grads, max_norm, norm_type):
+    before = [g.clone() for g in grads]
+    total_dev = torch.zeros(1, dtype=torch.float64, device="cuda")
+    nsg.dmuon_clip_grad_norm(grads, max_norm, norm_type, total_dev)
+    torch.cuda.synchronize()
+    _, total, coef = om.clip_grad_norm([to64(g) for g in before], max_norm, norm_type)
+    got_total = float(total_dev.item())
+    assert math.isclose(got_total, total, rel_tol=1e-5), (got_total, total)
+    # the coefficient the kernel applied, recomputed from its own total as the
+    # kernel does (fp64, rounded once to fp32)
+    k = np.float32(min(1.0, max_norm / (got_total + om.CLIP_EPS)))
+    assert math.isclose(float(k), coef, rel_tol=1e-5)
+    for b, g in zip(before, grads):
+        want = em.clip_scale_fp32(b.float().cpu().numpy(), float(k), dtype_name(b))
+        want_t = torch.from_numpy(want).to(b.dtype)
+        assert np.array_equal(bits(g), bits(want_t))
+    return got_total, float(k)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("norm_type", [2.0, 1.0, float("inf")], ids=["l2", "l1", "linf"])
+def test_clip_mixed_shapes(dtype, norm_type):
+    grads = make_grads(MIXED, dtype, 11)
+    total, k = check_clip(grads, 1.0, norm_type)
+    assert k < 1.0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_clip_no_op_when_under_the_bound(dtype):
+    grads = make_grads(MIXED[:4], dtype, 12, scale=1e-3)
+    before = [bits(g) for g in grads]
+    _, k = check_clip(grads, 1e6, 2.0)
+    assert k == 1.0
+    for b, g in zip(before, grads):
+        assert np.array_equal(b, bits(g))
+
+
+def test_clip_zero_gradients_and_zero_max_norm():
+    grads = make_grads([(64, 128), (3, 5)], torch.float32, 13)
+    check_clip(grads, 0.0, 2.0)
+    assert all(float(g.abs().max()) == 0.0 for g in grads)
+    zeros = [torch.zeros(8, 8, device="cuda"), torch.zeros(5, 3, device="cuda")]
+    total, k = check_clip(zeros, 1.0, 2.0)
+    assert total == 0.0 and k == 1.0
+
+
+def test_clip_many_matrices_of_one_shape_spans_table_batches():
+    # more than one launch table per class (tables hold 256 matrices)
+    grads = make_grads([(16, 24)] * 300 + [(40, 8)] * 3, torch.bfloat16, 14)
+    check_clip(grads, 2.0, 2.0)
+
+
+def test_clip_unaligned_views_take_the_scalar_path():
+    base = torch.randn(1, 64 * 37 + 3, device="cuda")
+    g = base[0, 3:].view(64, 37)  # fp32 rows of 148 bytes, start 12 bytes off
+    assert g.is_contiguous()
+    check_clip([g], 0.5, 2.0)
+
+
+def test_clip_deterministic():
+    grads = make_grads([(1024, 2816), (300, 300)], torch.float32, 15)
+    a = [g.clone() for g in grads]
+    b = [g.clone() for g in grads]
+    ta = torch.zeros(1, dtype=torch.float64, device="cuda")
+    tb = torch.zeros(1, dtype=torch.float64, device="cuda")
+    nsg.dmuon_clip_grad_norm(a, 1.0, 2.0, ta)
+    nsg.dmuon_clip_grad_norm(b, 1.0, 2.0, tb)
+    torch.cuda.synchronize()
+    assert ta.item() == tb.item()
+    for x, y in zip(a, b):
+        assert np.array_equal(bits(x), bits(y))
+
+
+# ------------------------------------------------ clipping fused into the step
+import workloads  # noqa: E402
+
+
+def _clone(ts):
+    return [t.clone() for t in ts]
+
+
+@pytest.mark.parametrize("norm_type", [2.0, float("inf")], ids=["l2", "linf"])
+@pytest.mark.parametrize("name", ["small_layer_bf16", "single_256x512_f32"])
+def test_step_clipped_equals_clip_then_step(name, norm_type, monkeypatch):
+    # small workspace cap: several chunks, run overlapped on two streams
+    monkeypatch.setenv("DMUON_WS_CAP_MB", "20")
+    w = workloads.get(name)
+    ps, gs, bs = workloads.make_all(w, "cuda")
+    g_bits = [bits(g) for g in gs]
+    # reference order of operations: clip in place, then the plain step
+    p1, g1, b1 = _clone(ps), _clone(gs), _clone(bs)
+    t1 = torch.zeros(1, dtype=torch.float64, device="cuda")
+    if norm_type == 2.0:
+        max_norm = 0.25 * float(sum(float(g.double().norm()) ** 2 for g in gs)) ** 0.5
+    else:
+        max_norm = 0.5 * max(float(g.abs().max()) for g in gs)
+    nsg.dmuon_clip_grad_norm(g1, max_norm, norm_type, t1)
+    nsg.dmuon_step(p1, g1, b1, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov, wd=0.1)
+    # fused
+    p2, b2 = _clone(ps), _clone(bs)
+    t2 = torch.zeros(1, dtype=torch.float64, device="cuda")
+    nsg.dmuon_step(p2, gs, b2, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov, wd=0.1,
+                   max_norm=max_norm, norm_type=norm_type, total_norm=t2)
+    torch.cuda.synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    nsg.dmuon_release_workspace()
+    assert t1.item() == t2.item()
+    assert max_norm / t1.item() < 0.6  # clipping is active
+    for a, b in zip(p1 + b1, p2 + b2):
+        assert np.array_equal(bits(a), bits(b))
+    # the fused step leaves the gradients untouched
+    for before, g in zip(g_bits, gs):
+        assert np.array_equal(before, bits(g))
+
+
+@pytest.mark.parametrize("name", ["small_layer_bf16", "single_256x512_f32"])
+def test_step_clipped_matches_oracle(name):
+    w = workloads.get(name)
+    ps, gs, bs = workloads.make_all(w, "cuda")
+    p_old = [to64(p) for p in ps]
+    g_h = [to64(g) for g in gs]
+    b_h = [to64(b) for b in bs]
+    max_norm = 0.5
+    total = torch.zeros(1, dtype=torch.float64, device="cuda")
+    nsg.dmuon_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
+                   ns_steps=w.ns_steps, wd=w.wd, max_norm=max_norm, total_norm=total)
+    torch.cuda.synchronize()
+    clipped, want_total, coef = om.clip_grad_norm(g_h, max_norm, 2.0)
+    assert coef < 1.0
+    assert math.isclose(total.item(), want_total, rel_tol=1e-5)
+    p_new, b_new, _ = om.muon_step(p_old, clipped, b_h, w.lr, w.momentum, w.nesterov,
+                                   w.ns_steps, None, w.wd)
+    for k in range(w.count):
+        dn = dtype_name(ps[k])
+        step = np.linalg.norm(p_new[k] - p_old[k])
+        err = np.linalg.norm(to64(ps[k]) - p_new[k])
+        tol_rel = 2e-2 if dn == "bf16" else 1e-4
+        store = 2.0 ** -8 if dn == "bf16" else 1e-6
+        assert err <= tol_rel * step + store * np.linalg.norm(p_new[k]), (k, err, step)
+        # the buffer holds mu*buf + clipped g, rounded to its dtype
+        berr = np.linalg.norm(to64(bs[k]) - b_new[k])
+        assert berr <= (2.0 ** -8 if dn == "bf16" else 1e-6) * np.linalg.norm(b_new[k])

@@ -355,3 +355,23 @@ def test_clip_global_norm_couples_matrices():
     out, total, coef = om.clip_grad_norm([small, big], 1.0)
     assert abs(total - np.sqrt(4 * 1e-6 + 4 * 1e4)) < 1e-9
     assert np.allclose(out[0], small * coef) and coef < 0.01
+
+
+@pytest.mark.parametrize("norm_type", [1.0, 2.0, float("inf")])
+@pytest.mark.parametrize("where", [0, 1, 2])
+def test_clip_nan_anywhere_gives_nan_total(norm_type, where):
+    # PyTorch's clip_grad_norm_ (which the clipping section pairs the clip with)
+    # reduces with sum / max, both of which keep a NaN wherever it sits
+    gs = [gauss((3, 4), 20 + k) for k in range(3)]
+    gs[where][1, 2] = np.nan
+    out, total, coef = om.clip_grad_norm(gs, 1.0, norm_type)
+    assert np.isnan(total) and coef == 1.0
+    assert all(np.array_equal(a, b, equal_nan=True) for a, b in zip(out, gs))
+
+
+def test_clip_infinity_gives_zero_coefficient():
+    gs = [np.array([[1.0, np.inf]]), np.array([[2.0]])]
+    for norm_type in (1.0, 2.0, float("inf")):
+        out, total, coef = om.clip_grad_norm(gs, 1.0, norm_type)
+        assert total == np.inf and coef == 0.0
+        assert np.isnan(out[0][0, 1]) and out[0][0, 0] == 0.0 and out[1][0, 0] == 0.0

@@ -61,6 +61,8 @@ def parse_args(argv=None):
                     help="override the workload's Newton-Schulz iteration count")
     ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update"],
                     help="time one kernel through its stage call instead of the whole step")
+    ap.add_argument("--clip-norm", type=float, default=None,
+                    help="time dmuon_step_clipped: global 2-norm clipping of the gradients to this bound")
     ap.add_argument("--batch", type=int, default=8)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--n", type=int, default=4096)
@@ -296,10 +298,16 @@ def run_ours(args):
     # workspace per stream, so warm-up and capture use the same one
     run_stream = torch.cuda.Stream(dev) if args.graph else stream
     launches_per_step = nsg.dmuon_step_launches(shapes, w.ns_steps)
+    if args.clip_norm is not None:
+        # one norm launch per table of <= 256 matrices of one shape, plus the coefficient
+        groups = {}
+        for sh in shapes:
+            groups[sh] = groups.get(sh, 0) + 1
+        launches_per_step += sum((c + 255) // 256 for c in groups.values()) + 1
 
     def step():
         nsg.dmuon_step_ptrs(pp, gp, bp, shapes, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
-                            ns_steps=w.ns_steps, wd=w.wd, stream=run_stream)
+                            ns_steps=w.ns_steps, wd=w.wd, stream=run_stream, max_norm=args.clip_norm)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -373,7 +381,7 @@ def run_ours(args):
         peak = float(peaks["hbm_gbs"])
         bound, unit = "hbm", "GB/s"
     elem = {}
-    for k in ("momentum", "update"):
+    for k in ("momentum", "update", "clip_norm"):
         if k in kstats:
             v = kstats[k]
             elem[k] = {"GB/s": round(v["bytes"] / (v["total_ms"] / 1e3) / 1e9, 1),
@@ -414,6 +422,8 @@ def run_ours(args):
         "config": {"workload": w.name, "matrices": w.count,
                    "shapes": sorted({f"{r}x{c}" for r, c in w.shapes}),
                    "ns_steps": w.ns_steps, "nesterov": w.nesterov, "lr": w.lr, "wd": w.wd,
+                   **({"clip": {"max_norm": args.clip_norm, "norm_type": 2.0, "fused": "dmuon_step_clipped"}}
+                      if args.clip_norm is not None else {}),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"no flush: each step touches {w.elements() * 2 * 7 / 1e9:.1f} GB "
                          f"(inputs alone {w.elements() * 2 * 3 / 1e9:.1f} GB) >> 126 MB L2"},

@@ -168,6 +168,8 @@ DMUON_API dmuon_status_t dmuon_step_clipped(void* const* params, const void* con
  *   norm_type  1, 2 or INFINITY (others: DMUON_ERR_UNSUPPORTED)
  *   total_norm DEVICE double or NULL: receives `total`
  * Deterministic (fixed-order fp64 reduction of per-tile fp32 partials).
+ * Non-finite gradients: a NaN anywhere makes `total` NaN and coef 1 (nothing
+ * is scaled); an infinity (and no NaN) makes `total` inf and coef 0.
  */
 DMUON_API dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* shapes, int32_t count,
                                               float max_norm, float norm_type, double* total_norm,

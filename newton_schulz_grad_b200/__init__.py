@@ -251,15 +251,21 @@ def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
 def dmuon_step_ptrs(params: Sequence[int], grads: Sequence[int], mom_bufs: Sequence[int],
                     shapes: Sequence[Tuple[int, int, int]], lr: float = 0.02,
                     momentum: float = 0.95, nesterov: bool = True, ns_steps: int = 5,
-                    coeffs=None, wd: float = 0.0, stream=None) -> None:
-    """dmuon_step on raw device addresses (no per-tensor checks on the Python side)."""
+                    coeffs=None, wd: float = 0.0, stream=None, max_norm: Optional[float] = None,
+                    norm_type: float = 2.0) -> None:
+    """dmuon_step (dmuon_step_clipped with ``max_norm``) on raw device addresses."""
     n = len(params)
     vp = ctypes.c_void_p
     pa = (vp * max(1, n))(*params)
     ga = (vp * max(1, n))(*grads)
     ba = (vp * max(1, n))(*mom_bufs)
-    _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
-                           ns_steps, _coeffs(ns_steps, coeffs), wd, _stream(stream)))
+    if max_norm is None:
+        _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
+                               ns_steps, _coeffs(ns_steps, coeffs), wd, _stream(stream)))
+    else:
+        _check(_lib.dmuon_step_clipped(pa, ga, ba, _shape_array(shapes), n, lr, momentum,
+                                       int(bool(nesterov)), ns_steps, _coeffs(ns_steps, coeffs), wd,
+                                       float(max_norm), float(norm_type), None, _stream(stream)))
 
 
 def dmuon_clip_grad_norm(grads: Sequence[torch.Tensor], max_norm: float, norm_type: float = 2.0,

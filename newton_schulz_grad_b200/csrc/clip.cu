@@ -21,16 +21,23 @@ constexpr int kThreads = 256;
 
 __device__ __forceinline__ int clamp8(int64_t v) { return v < 8 ? (int)v : 8; }
 
+// max that keeps a NaN (fmaxf drops it), so a NaN gradient makes the
+// infinity norm NaN as it makes the sums NaN
+template <typename F>
+__device__ __forceinline__ F nan_max(F a, F b) {
+  return (a > b || a != a) ? a : b;
+}
+
 // P = 1, 2: sum of |g|^P; P = 0: max |g| (the infinity norm)
 template <int P>
 __device__ __forceinline__ float accum(float acc, float v) {
-  if (P == 0) return fmaxf(acc, fabsf(v));
+  if (P == 0) return nan_max(acc, fabsf(v));
   if (P == 1) return acc + fabsf(v);
   return fmaf(v, v, acc);
 }
 template <int P>
 __device__ __forceinline__ float combine(float a, float b) {
-  return P == 0 ? fmaxf(a, b) : a + b;
+  return P == 0 ? nan_max(a, b) : a + b;
 }
 
 template <typename T, int P>
@@ -78,17 +85,18 @@ __global__ void __launch_bounds__(kThreads)
   double acc = 0.0;
   for (int64_t i = threadIdx.x; i < count; i += kThreads) {
     const double v = (double)partials[i];
-    acc = p == 0 ? fmax(acc, v) : acc + v;
+    acc = p == 0 ? nan_max(acc, v) : acc + v;
   }
   red[threadIdx.x] = acc;
   __syncthreads();
   for (int w = kThreads / 2; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] = p == 0 ? fmax(red[threadIdx.x], red[threadIdx.x + w])
+    if (threadIdx.x < w) red[threadIdx.x] = p == 0 ? nan_max(red[threadIdx.x], red[threadIdx.x + w])
                                                    : red[threadIdx.x] + red[threadIdx.x + w];
     __syncthreads();
   }
   if (threadIdx.x == 0) {
     const double total = p == 0 ? red[0] : (p == 1 ? red[0] : sqrt(red[0]));
+    // a NaN total gives coef 1 (nothing scaled; the NaN total is reported)
     const double c = (double)max_norm / (total + 1e-6);
     *coef = (float)(c < 1.0 ? c : 1.0);
     if (total_out) *total_out = total;

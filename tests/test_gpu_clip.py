@@ -47,8 +47,12 @@ def check_clip(grads, max_norm, norm_type):
     assert math.isclose(float(k), coef, rel_tol=1e-5)
     for b, g in zip(before, grads):
         want = em.clip_scale_fp32(b.float().cpu().numpy(), float(k), dtype_name(b))
-        want_t = torch.from_numpy(want).to(b.dtype)
-        assert np.array_equal(bits(g), bits(want_t))
+        nan = np.isnan(want)
+        got = g.float().cpu().numpy()
+        assert np.array_equal(np.isnan(got), nan)  # NaN payloads differ between CPU and GPU
+        want_t = torch.from_numpy(np.where(nan, 0, want)).to(b.dtype)
+        got_t = torch.from_numpy(np.where(nan, 0, got)).to(b.dtype)
+        assert np.array_equal(bits(got_t), bits(want_t))
     return got_total, float(k)
 
 
@@ -175,3 +179,26 @@ def test_step_clipped_matches_oracle(name):
         # the buffer holds mu*buf + clipped g, rounded to its dtype
         berr = np.linalg.norm(to64(bs[k]) - b_new[k])
         assert berr <= (2.0 ** -8 if dn == "bf16" else 1e-6) * np.linalg.norm(b_new[k])
+
+
+def test_clip_non_finite_gradients():
+    for norm_type in (2.0, 1.0, float("inf")):
+        # a NaN: total NaN, coefficient 1, values unchanged (the oracle agrees)
+        a = make_grads([(64, 96), (10, 10)], torch.float32, 16)
+        a[1][3, 4] = float("nan")
+        _, want_total, want_coef = om.clip_grad_norm([to64(g) for g in a], 1.0, norm_type)
+        assert math.isnan(want_total) and want_coef == 1.0
+        before = [g.clone() for g in a]
+        t = torch.zeros(1, dtype=torch.float64, device="cuda")
+        nsg.dmuon_clip_grad_norm(a, 1.0, norm_type, t)
+        torch.cuda.synchronize()
+        assert math.isnan(t.item())
+        for x, g in zip(before, a):
+            nan = torch.isnan(x)
+            assert torch.equal(nan, torch.isnan(g))  # the GPU's NaN payload may differ
+            assert np.array_equal(bits(torch.where(nan, 0, x)), bits(torch.where(nan, 0, g)))
+        # an infinity: total inf, coefficient 0 (inf * 0 is NaN, the rest 0)
+        b = make_grads([(64, 96), (10, 10)], torch.bfloat16, 17)
+        b[0][5, 6] = float("inf")
+        total, k = check_clip(b, 1.0, norm_type)
+        assert math.isinf(total) and k == 0.0

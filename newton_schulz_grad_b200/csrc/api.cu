@@ -160,10 +160,11 @@ bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
 
 // ------------------------------------------------------------ kernel timing
 enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
-            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kNumKinds };
+            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kApplyUpdTc, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
                                            "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
-                                           "copy_out", "symm_tc", "chain_small", "clip_norm", "clip_scale"};
+                                           "copy_out", "symm_tc", "chain_small", "clip_norm", "clip_scale",
+                                           "apply_update_tc"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -234,9 +235,24 @@ bool any_overlap(std::vector<Interval>& v) {
 
 // The Newton-Schulz chain over a chunk of `b` oriented m x n matrices in the
 // workspace; returns the buffer that holds the result.
+// Thin matrices (m <= 64, FFMA path) whose chain runs as one clustered launch.
+bool thin_chain(const ChunkLayout& L, int64_t m, int64_t n, int32_t steps) {
+  return L.path != Path::kTensorBf16 && m <= kSmallM && steps >= 1 && steps <= 16 &&
+         n <= small_ns_max_n((int)m, L.path == Path::kSmallBf16 ? 2 : 4) && !env_is("DMUON_SMALL_CHAIN", '0');
+}
+
+// The tensor path ends with a tensor-core apply, whose epilogue can update
+// the parameters directly (DMUON_FUSED_UPDATE=0 keeps the separate pass).
+bool fuses_update(const ChunkLayout& L, int32_t steps) {
+  return L.path == Path::kTensorBf16 && steps >= 1 && !env_is("DMUON_FUSED_UPDATE", '0');
+}
+
+// upd (optional, only where fuses_update): the last apply updates the
+// parameters in its epilogue and stores no result (*result = nullptr).
 dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char* ws,
                          const ChunkOffsets& off, int32_t steps, const std::vector<float>& sched,
-                         const DeviceState& ds, cudaStream_t st, void** result) {
+                         const DeviceState& ds, cudaStream_t st, void** result,
+                         const UpdTable* upd = nullptr) {
   void* cur = ws + off.x0;
   void* nxt = ws + off.x1;
   void* G = ws + off.g;
@@ -257,7 +273,16 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
            : simt_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, xbf16, st);
     p.done(st);
   };
-  auto apply = [&](const void* Pm, const void* X, void* Y, float a, const float* sc) {
+  bool fused = false;
+  auto apply = [&](const void* Pm, const void* X, void* Y, float a, const float* sc, bool last) {
+    if (tc && last && upd) {
+      // update bytes: read and write p
+      Prof p(kApplyUpdTc, st, 2.0 * fb * fm * fm * fn, 4.0 * fb * fm * fn);
+      e = tc_apply_update(Pm, X, b, mi, ni, L.ldm, L.ldn, a, 1.f, sc, *upd, sw, sms, st);
+      p.done(st);
+      fused = true;
+      return;
+    }
     Prof p(tc ? kApplyTc : kApplyFfma, st, 2.0 * fb * fm * fm * fn, 0.0);
     e = tc ? tc_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, sw, sms, st)
            : simt_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st);
@@ -272,8 +297,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   const auto coef = [&](int k, int i) { return sched[3 * k + i]; };
 
   // thin matrices: the whole chain in one clustered launch, in place on X0
-  if (!tc && m <= kSmallM && steps >= 1 && steps <= 16 &&
-      n <= small_ns_max_n((int)m, xbf16 ? 2 : 4) && !env_is("DMUON_SMALL_CHAIN", '0')) {
+  if (thin_chain(L, m, n, steps)) {
     Prof p(kChainSmall, st, fb * (3.0 * fm * fm * fn + fm * fm * fm) * steps, 0.0);
     e = small_ns(cur, b, mi, ni, L.ldn, steps, sched.data(), scale, xbf16, st);
     p.done(st);
@@ -301,7 +325,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
         p.done(st);
       }
       if (e != cudaSuccess) break;
-      apply(P, cur, nxt, coef(k, 0), sc);
+      apply(P, cur, nxt, coef(k, 0), sc, k + 1 == steps);
       std::swap(cur, nxt);
       k += 1;
       continue;
@@ -325,20 +349,21 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
       if (e == cudaSuccess) symm(S1, S4, nullptr, S2, 0.f, 1.f, 0.f, kSymmTc);  // Q2 = P2 Q
       Q = S2;
     }
-    if (e == cudaSuccess) apply(Q, cur, nxt, 0.f, sc);  // X <- Q X (scaled by s when k == 0)
+    if (e == cudaSuccess) apply(Q, cur, nxt, 0.f, sc, k + len == steps);  // X <- Q X (scaled by s when k == 0)
     std::swap(cur, nxt);
     k += len;
   }
   if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
-  *result = cur;
+  *result = fused ? nullptr : cur;
   return DMUON_OK;
 }
 
-// Kernels one chunk launches: momentum, norm, the chain, update.
-int64_t chunk_launches_for(const ChunkLayout& L, int32_t steps) {
-  int64_t n = 3;
-  for (int len : chain_blocks(L, steps)) n += len == 1 ? 3 : (len == 2 ? 7 : 11);  // gram + products + apply
-  return n;
+// Kernels one chunk launches: momentum, norm, the chain, update (unless fused).
+int64_t chunk_launches_for(const ChunkLayout& L, int64_t m, int64_t n, int32_t steps) {
+  int64_t k = fuses_update(L, steps) ? 2 : 3;
+  if (thin_chain(L, m, n, steps)) return k + 1;
+  for (int len : chain_blocks(L, steps)) k += len == 1 ? 3 : (len == 2 ? 7 : 11);  // gram + products + apply
+  return k;
 }
 
 // ----------------------------------------------------------- gradient clipping
@@ -483,6 +508,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     if (e != cudaSuccess) return cuda_fail(e, "stream fork");
   }
   std::vector<void*> results(P.chunks.size(), nullptr);
+  std::unique_ptr<UpdTable> upd_tab(new UpdTable());
 
   auto fill_table = [&](const ChunkRef& ck, ElemTable& tab) {
     const LaunchClass& c = P.classes[ck.cls];
@@ -505,7 +531,9 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     }
   };
   auto buffer = [&](size_t i) { return static_cast<char*>(wsv) + (int64_t)(i % nbuf) * P.buffer_bytes; };
+  // the parameter update of chunk i, unless its last apply already did it
   auto update = [&](size_t i) -> dmuon_status_t {
+    if (!results[i]) return DMUON_OK;
     const ChunkRef& ck = P.chunks[i];
     const LaunchClass& c = P.classes[ck.cls];
     const ChunkOffsets off = chunk_offsets(P.layouts[ck.cls], ck.b);
@@ -552,7 +580,22 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
       drop();
       return cuda_fail(e, "norm launch / stream join");
     }
-    rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &results[i]);
+    const UpdTable* upd = nullptr;
+    if (fuses_update(L, ns_steps)) {
+      UpdTable& u = *upd_tab;
+      update_coeffs(lr, wd, c.n, &u.decay, &u.step_scale);
+      std::memset(u.tmask, 0, sizeof(u.tmask));
+      std::memset(u.vmask, 0, sizeof(u.vmask));
+      for (int j = 0; j < ck.b; ++j) {
+        const int32_t mi = c.members[ck.start + j];
+        u.p[j] = params[mi];
+        if (shapes[mi].rows > shapes[mi].cols) u.tmask[j >> 5] |= 1u << (j & 31);
+        if ((shapes[mi].cols * (int64_t)esize(c.dtype)) % 16 == 0 && aligned16(params[mi]))
+          u.vmask[j >> 5] |= 1u << (j & 31);
+      }
+      upd = &u;
+    }
+    rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &results[i], upd);
     if (rc != DMUON_OK) {
       drop();
       return rc;
@@ -639,7 +682,8 @@ int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t 
   if (count <= 0 || !shapes) return 0;
   const StepPlan P = make_step_plan(shapes, count);
   int64_t n = 0;
-  for (const ChunkRef& ck : P.chunks) n += chunk_launches_for(P.layouts[ck.cls], ns_steps);
+  for (const ChunkRef& ck : P.chunks)
+    n += chunk_launches_for(P.layouts[ck.cls], P.classes[ck.cls].m, P.classes[ck.cls].n, ns_steps);
   return n;
 }
 

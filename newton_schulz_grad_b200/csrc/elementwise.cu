@@ -257,16 +257,21 @@ cudaError_t launch_norm_finalize(const float* partials, int count, int tiles_per
   return cudaGetLastError();
 }
 
+void update_coeffs(float lr, float wd, int64_t scale_dim, float* decay, float* step_scale) {
+  // fp32, each operation rounded once, in this order (no contraction):
+  volatile float lw = lr * wd;
+  *decay = 1.0f - lw;
+  *step_scale = (float)((double)lr * 0.2 * sqrt((double)scale_dim));
+}
+
 cudaError_t launch_update(const ElemTable& t, int dtype, ElemMode mode, const void* O,
                           const float* scale, float lr, float wd, int64_t scale_dim,
                           cudaStream_t st) {
   if (t.count == 0) return cudaSuccess;
   const size_t es = dtype == DMUON_BF16 ? 2 : 4;
   const int o_vec = ((t.ldn * (int64_t)es) % 16 == 0) && aligned16(O);
-  // fp32, each operation rounded once, in this order (no contraction):
-  volatile float lw = lr * wd;
-  const float decay = 1.0f - lw;
-  const float step_scale = (float)((double)lr * 0.2 * sqrt((double)scale_dim));
+  float decay, step_scale;
+  update_coeffs(lr, wd, scale_dim, &decay, &step_scale);
   dim3 grid((unsigned)t.tiles_per_mat, (unsigned)t.count);
   if (dtype == DMUON_BF16) {
     auto* o = static_cast<const __nv_bfloat16*>(O);

@@ -114,6 +114,24 @@ cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int ba
 cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
                      int64_t ldx, int64_t ldy, float a, float alpha, const float* scale,
                      int* status, int num_sms, cudaStream_t st);
+
+// The parameter update fused into the last apply of the chain: for matrix b
+// of the launch, O = bf16(alpha (a X + P X)) (the value tc_apply would store)
+// and p_b <- bf16(p_b * decay - step_scale * O), p_b in its source layout
+// (n x m, i.e. O transposed, where the tmask bit is set).  Same arithmetic and
+// rounding as launch_update on the stored O, so the two paths agree bit for bit.
+struct UpdTable {
+  void* p[kMaxTable];
+  uint32_t tmask[kMaxTable / 32];  // source is n x m
+  uint32_t vmask[kMaxTable / 32];  // source rows allow 16-byte vectors
+  float decay, step_scale;
+};
+cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int n, int64_t ldp, int64_t ldx,
+                            float a, float alpha, const float* scale, const UpdTable& u, int* status,
+                            int num_sms, cudaStream_t st);
+// decay = 1 - lr wd and step_scale = fl32(lr 0.2 sqrt(scale_dim)), each rounded
+// as the update kernels use them.
+void update_coeffs(float lr, float wd, int64_t scale_dim, float* decay, float* step_scale);
 const char* tc_config_string();
 // One-thread kernel whose bounded wait runs out after limit_us (status word).
 cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st);

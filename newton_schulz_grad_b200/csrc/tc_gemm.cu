@@ -80,6 +80,12 @@ constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 256;
 
 enum { kGram = 0, kPoly = 1, kApply = 2 };
 
+// The update table is a kernel parameter only of the fused apply + update
+// instantiation; the others take an empty one.
+struct NoUpd {};
+template <bool UPD> struct UpdSel { using type = NoUpd; };
+template <> struct UpdSel<true> { using type = UpdTable; };
+
 struct TcArgs {
   __nv_bfloat16* C;
   const __nv_bfloat16* E;
@@ -320,11 +326,171 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* f) {
   return raw;
 }
 
+// Fused update, one 32-column chunk of oriented row r (< m), columns c0 ..
+// c0 + 31 (< n) of matrix b: p <- bf16(p * decay - step_scale * bf16(v)).
+// Non-transposed rows are contiguous runs of p; transposed ones are a column
+// of p, and across the warp (consecutive r) each j is one 64-byte run.  The
+// parameters (and the a X term) of a chunk are loaded one chunk ahead into
+// packed bf16 pairs, so their latency hides behind the previous chunk.
+struct UpdChunk {
+  uint32_t p[16];  // 32 bf16 parameters
+  uint32_t e[16];  // 32 bf16 of X (only when a != 0)
+};
+
+__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+__device__ __forceinline__ float half_of(const uint32_t* w, int j) {
+  const uint32_t x = w[j >> 1];
+  return __uint_as_float((j & 1) ? (x & 0xffff0000u) : (x << 16));
+}
+
+__device__ __forceinline__ void load_upd_chunk(const UpdTable& u, const TcArgs& a, int b, int r, int c0,
+                                               UpdChunk& k) {
+  const int m = a.m, n = a.n;
+  const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(u.p[b]);
+  const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
+  const bool full = c0 + 32 <= n;
+  if (tr) {
+    const __nv_bfloat16* q = p + (int64_t)c0 * m + r;
+    const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const __nv_bfloat16 lo = (c0 + j < n) ? *q : z;
+      q += m;
+      const __nv_bfloat16 hi = (c0 + j + 1 < n) ? *q : z;
+      q += m;
+      k.p[j >> 1] = pack2(lo, hi);
+    }
+  } else if (full && ((u.vmask[b >> 5] >> (b & 31)) & 1u)) {
+    const uint4* q = reinterpret_cast<const uint4*>(p + (int64_t)r * n + c0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(k.p)[i] = q[i];
+  } else {
+    const __nv_bfloat16* q = p + (int64_t)r * n + c0;
+    const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+    for (int j = 0; j < 32; j += 2)
+      k.p[j >> 1] = pack2((c0 + j < n) ? q[j] : z, (c0 + j + 1 < n) ? q[j + 1] : z);
+  }
+  if (a.p0 != 0.f) {
+    const __nv_bfloat16* ep = a.E + (int64_t)b * a.sE + (int64_t)r * a.lde + c0;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(k.e)[i] = __ldg(reinterpret_cast<const uint4*>(ep) + i);
+    } else {
+      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+      for (int j = 0; j < 32; j += 2)
+        k.e[j >> 1] = pack2((c0 + j < n) ? ep[j] : z, (c0 + j + 1 < n) ? ep[j + 1] : z);
+    }
+  }
+}
+
+// v: the accumulator chunk (fp32); applies alpha (a X + .), rounds the result
+// to bf16 as the plain apply would store it, and updates the parameters.
+__device__ __forceinline__ void store_upd_chunk(const UpdTable& u, const TcArgs& a, int b, int r, int c0,
+                                                float alpha, const UpdChunk& k, float* v) {
+  const int m = a.m, n = a.n;
+  if (a.p0 != 0.f) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = alpha * fmaf(a.p0, half_of(k.e, j), v[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = alpha * v[j];
+  }
+  float* pv = v;  // in place: v[j] becomes the new parameter
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float o = __bfloat162float(__float2bfloat16_rn(v[j]));
+    pv[j] = __fsub_rn(__fmul_rn(half_of(k.p, j), u.decay), __fmul_rn(u.step_scale, o));
+  }
+  __nv_bfloat16* p = static_cast<__nv_bfloat16*>(u.p[b]);
+  const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
+  if (tr) {
+    __nv_bfloat16* q = p + (int64_t)c0 * m + r;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (c0 + j < n) *q = __float2bfloat16_rn(pv[j]);
+      q += m;
+    }
+  } else if (c0 + 32 <= n && ((u.vmask[b >> 5] >> (b & 31)) & 1u)) {
+    uint4* q = reinterpret_cast<uint4*>(p + (int64_t)r * n + c0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = pack_bf16x8(pv + 8 * i);
+  } else {
+    __nv_bfloat16* q = p + (int64_t)r * n + c0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (c0 + j < n) q[j] = __float2bfloat16_rn(pv[j]);
+  }
+}
+
+// Epilogue of one apply tile with the fused update (see epilogue_row).
+__device__ __forceinline__ void epilogue_row_update(const TcArgs& a, const UpdTable& u, uint32_t taddr, int b,
+                                                    int r, int J) {
+  const bool row_ok = r < a.m;
+  const float alpha = a.p1 * (a.scale ? a.scale[b] : 1.f);
+  const int cbase = J * BN;
+  UpdChunk k0, k1;
+  if (row_ok) load_upd_chunk(u, a, b, r, cbase, k0);
+  // one chunk: load the next chunk's operands, then drain this one
+  auto chunk = [&](int ch, const UpdChunk& cur, UpdChunk& nxt) -> bool {
+    const int c0 = cbase + ch * 32;
+    if (c0 >= a.n) return false;  // warp-uniform
+    if (row_ok && ch + 1 < BN / 32 && c0 + 32 < a.n) load_upd_chunk(u, a, b, r, c0 + 32, nxt);
+    uint32_t raw[32];
+    tmem_ld32(taddr + (uint32_t)(ch * 32), raw);
+    tmem_ld_wait();
+    if (row_ok) store_upd_chunk(u, a, b, r, c0, alpha, cur, reinterpret_cast<float*>(raw));
+    return true;
+  };
+#pragma unroll 1
+  for (int ch = 0; ch < BN / 32; ch += 2) {
+    if (!chunk(ch, k0, k1)) break;
+    if (!chunk(ch + 1, k1, k0)) break;
+  }
+}
+
+// Before an update tile's accumulator is ready: pull the parameters it
+// rewrites into L2 (oriented rows [r0, r0 + 32) of this warp, columns
+// [col0, col0 + 256)), so the epilogue's loads do not wait on DRAM.
+__device__ __forceinline__ void prefetch_update_tile(const UpdTable& u, int b, int r0, int col0, int m, int n,
+                                                     int lane) {
+  const char* p = static_cast<const char*>(u.p[b]);
+  const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
+  if (r0 >= m) return;
+  if (tr) {
+    // source rows col0 .. col0 + 255, 64 bytes (32 columns from r0) each: 8 per lane
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = col0 + lane * 8 + i;
+      if (c < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + ((int64_t)c * m + r0) * 2));
+    }
+  } else {
+    // row r0 + lane, 512 bytes from col0: four 128-byte lines
+    const int r = r0 + lane;
+    if (r < m) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = col0 + i * 64;
+        if (c < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + ((int64_t)r * n + c) * 2));
+      }
+    }
+  }
+}
+
 // Epilogue of one tile for one accumulator row: TMEM lane quarter `wq` of
 // accumulator columns [col0, col0 + 256), output row r, output columns from
-// J * 256.  Warp-collective (tcgen05.ld).
-template <int MODE>
-__device__ __forceinline__ void epilogue_row(const TcArgs& a, uint32_t taddr, int b, int r, int J) {
+// J * 256.  Warp-collective (tcgen05.ld).  UPD (apply only): update the
+// parameters instead of storing the result.
+template <int MODE, bool UPD>
+__device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename UpdSel<UPD>::type& u, uint32_t taddr,
+                                             int b, int r, int J) {
+  if constexpr (UPD) {
+    epilogue_row_update(a, u, taddr, b, r, J);
+    return;
+  }
   const bool row_ok = r < a.m;
   float alpha = 1.f;
   if (MODE == kGram) {
@@ -424,10 +590,10 @@ __device__ __forceinline__ Bars bar_layout(uint64_t* bars) {
 }
 
 // ================================================================ one CTA
-template <int MODE>
+template <int MODE, bool UPD>
 __global__ void __launch_bounds__(kThreads, 1)
     k_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-         const TcArgs a) {
+         const TcArgs a, const __grid_constant__ typename UpdSel<UPD>::type u) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -555,9 +721,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
       int b, I, J;
       decode_tile<MODE>(a, t, b, I, J);
+      if constexpr (UPD) {
+        // this CTA's first tile now, then always the next one during this epilogue
+        if (t == (int)blockIdx.x) prefetch_update_tile(u, b, I * BM1 + wq * 32, J * BN, a.m, a.n, lane);
+        if (t + (int)gridDim.x < a.total_tiles) {
+          int b2, I2, J2;
+          decode_tile<MODE>(a, t + (int)gridDim.x, b2, I2, J2);
+          prefetch_update_tile(u, b2, I2 * BM1 + wq * 32, J2 * BN, a.m, a.n, lane);
+        }
+      }
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
-      epilogue_row<MODE>(a, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
+      epilogue_row<MODE, UPD>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
                          I * BM1 + wq * 32 + lane, J);
       tc_fence_before();
       __syncwarp();
@@ -576,10 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // =============================================================== CTA pair
-template <int MODE>
+template <int MODE, bool UPD>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const TcArgs a) {
+          const TcArgs a, const __grid_constant__ typename UpdSel<UPD>::type u) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -716,9 +891,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int t = pair; t < a.total_tiles; t += npairs) {
       int b, I, J;
       decode_tile<MODE>(a, t, b, I, J);
+      if constexpr (UPD) {
+        if (t == pair) prefetch_update_tile(u, b, I * BM2 + (int)rank * 128 + wq * 32, J * BN, a.m, a.n, lane);
+        if (t + npairs < a.total_tiles) {
+          int b2, I2, J2;
+          decode_tile<MODE>(a, t + npairs, b2, I2, J2);
+          prefetch_update_tile(u, b2, I2 * BM2 + (int)rank * 128 + wq * 32, J2 * BN, a.m, a.n, lane);
+        }
+      }
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
-      epilogue_row<MODE>(a, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
+      epilogue_row<MODE, UPD>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
                          I * BM2 + (int)rank * 128 + wq * 32 + lane, J);
       tc_fence_before();
       __syncwarp();
@@ -792,15 +975,15 @@ bool use_pair(int m) {
   return mode == 1 && m >= 256;
 }
 
-template <int MODE>
+template <int MODE, bool UPD = false>
 cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms, bool pair,
-                   cudaStream_t st) {
+                   cudaStream_t st, const typename UpdSel<UPD>::type& u = {}) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
+    attr_err = cudaFuncSetAttribute(k_tc<MODE, UPD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(k_tc2<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+      attr_err = cudaFuncSetAttribute(k_tc2<MODE, UPD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int64_t total = (int64_t)a.tiles_per_mat * batch;
@@ -809,10 +992,10 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int 
   a.total_tiles = (int)total;
   if (pair) {
     const int64_t pairs = total < num_sms / 2 ? total : num_sms / 2;
-    k_tc2<MODE><<<(int)(2 * pairs), kThreads, SMEM2_BYTES, st>>>(ma, mb, a);
+    k_tc2<MODE, UPD><<<(int)(2 * pairs), kThreads, SMEM2_BYTES, st>>>(ma, mb, a, u);
   } else {
     const int grid = (int)(total < num_sms ? total : num_sms);
-    k_tc<MODE><<<grid, kThreads, SMEM1_BYTES, st>>>(ma, mb, a);
+    k_tc<MODE, UPD><<<grid, kThreads, SMEM1_BYTES, st>>>(ma, mb, a, u);
   }
   return cudaGetLastError();
 }
@@ -903,6 +1086,33 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
   a.scale = scale;
   a.status = status;
   return launch<kApply>(ma, mb, a, batch, num_sms, pair, st);
+}
+
+cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int n, int64_t ldp, int64_t ldx,
+                            float a_coef, float alpha, const float* scale, const UpdTable& u, int* status,
+                            int num_sms, cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  if (batch > kMaxTable) return cudaErrorInvalidValue;
+  const bool pair = use_pair(m);
+  CUtensorMap ma, mb;
+  cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
+  if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
+  if (e != cudaSuccess) return e;
+  TcArgs a{};
+  a.C = nullptr;  // nothing stored but the parameters
+  a.E = static_cast<const __nv_bfloat16*>(X);
+  a.sE = (int64_t)m * ldx;
+  a.lde = ldx;
+  a.m = m; a.n = n; a.k = m;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
+  a.tiles_n = (n + BN - 1) / BN;
+  a.tiles_per_mat = a.tiles_m * a.tiles_n;
+  a.p0 = a_coef;
+  a.p1 = alpha;
+  a.scale = scale;
+  a.status = status;
+  return launch<kApply, true>(ma, mb, a, batch, num_sms, pair, st, u);
 }
 
 cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st) {

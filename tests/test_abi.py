@@ -64,14 +64,20 @@ def test_launch_count_and_workspace_llama7b():
     # 96 matrices; three iterations one at a time, then the last two as one
     # Gram-space block; five m x m slots: 340 MiB each).  Several chunks ->
     # overlapped execution with two buffers of half the 8 GiB cap: 5 chunks of
-    # <= 26 and 8 chunks of 12.  Per chunk: momentum + norm + update, plus 3 per
-    # single iteration and gram + 5 products + apply for the block of two.
-    assert nsg.dmuon_step_launches(shapes, 5) == 5 * (3 + 15) + 8 * (3 + 9 + 7)
+    # <= 26 and 8 chunks of 12.  Per chunk: momentum + norm (the update runs in
+    # the last apply's epilogue), plus 3 per single iteration and gram + 5
+    # products + apply for the block of two.
+    assert nsg.dmuon_step_launches(shapes, 5) == 5 * (2 + 15) + 8 * (2 + 9 + 7)
     os.environ["DMUON_GRAM_BLOCKS"] = "2"
     try:  # blocks of 2 and 3: gram + 5 products + apply, gram + 9 products + apply
-        assert nsg.dmuon_step_launches(shapes, 5) == 5 * (3 + 15) + 8 * (3 + 7 + 11)
+        assert nsg.dmuon_step_launches(shapes, 5) == 5 * (2 + 15) + 8 * (2 + 7 + 11)
     finally:
         del os.environ["DMUON_GRAM_BLOCKS"]
+    os.environ["DMUON_FUSED_UPDATE"] = "0"
+    try:  # a separate update pass per chunk
+        assert nsg.dmuon_step_launches(shapes, 5) == 5 * (3 + 15) + 8 * (3 + 9 + 7)
+    finally:
+        del os.environ["DMUON_FUSED_UPDATE"]
     ws = nsg.dmuon_workspace_bytes(shapes, 5)
     assert 5 << 30 < ws <= 8 << 30
 
@@ -81,8 +87,18 @@ def test_overlap_can_be_disabled(monkeypatch):
     shapes = [(r, c, 1) for r, c in w.shapes]
     monkeypatch.setenv("DMUON_OVERLAP", "0")
     monkeypatch.setenv("DMUON_GRAM_BLOCKS", "0")
-    assert nsg.dmuon_step_launches(shapes, 5) == 6 * (3 + 15)
+    assert nsg.dmuon_step_launches(shapes, 5) == 6 * (2 + 15)
     assert nsg.dmuon_workspace_bytes(shapes, 5) <= 8 << 30
+
+
+def test_launch_count_thin_and_fp32_chunks():
+    # fp32 and thin bf16 classes keep the separate update; thin bf16 chains
+    # (m <= 64) are one clustered launch
+    assert nsg.dmuon_step_launches([(256, 512, 0)], 5) == 3 + 5 * 3
+    assert nsg.dmuon_step_launches([(32, 4096, 1)] * 3, 5) == 3 + 1
+    assert nsg.dmuon_step_launches([(4096, 32, 1)], 5) == 3 + 1
+    assert nsg.dmuon_step_launches([(32, 4096, 1)], 0) == 3
+    assert nsg.dmuon_step_launches([(1024, 1024, 1)], 0) == 3
 
 
 def _raw_step(count, params, grads, bufs, shapes, ns_steps=5, nesterov=1, lr=0.02):

@@ -318,3 +318,57 @@ def test_thin_matrix_chain_matches_oracle_fused_and_unfused(shape, dtype, monkey
     tol = NS_TOL[dtype]
     assert rel_fro(to64(fused), want) < tol
     assert rel_fro(to64(plain), want) < tol
+
+
+@pytest.mark.parametrize("name,idx,env", [
+    ("small_layer_bf16", None, {}),
+    ("small_layer_bf16", None, {"DMUON_WS_CAP_MB": "20"}),        # several chunks, overlapped
+    ("small_layer_bf16", None, {"DMUON_GRAM_BLOCKS": "2"}),        # blocks of 2 and 3
+    ("small_layer_bf16", None, {"DMUON_GRAM_BLOCKS": "0"}),        # per-iteration form
+    ("llama3_2_3b_bf16", [0, 1, 4, 6], {}),
+    ("moe_skewed_bf16", [0, 2, 192, 240], {}),
+], ids=["small", "small-overlap", "small-blocks2", "small-periter", "3b", "moe"])
+def test_step_fused_update_equals_separate_pass(name, idx, env, monkeypatch):
+    # the last apply's epilogue updates the parameters (default) or a separate
+    # update kernel reads the stored result: same bits
+    w = workloads.get(name)
+    sk = workloads.skewed_indices(w)
+    idx = list(range(w.count)) if idx is None else idx
+    mats = [workloads.make_matrix(w, i, DEV, sk) for i in idx]
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+
+    def run(fused, steps=w.ns_steps):
+        monkeypatch.setenv("DMUON_FUSED_UPDATE", "1" if fused else "0")
+        ps = [m[0].clone() for m in mats]
+        gs = [m[1].clone() for m in mats]
+        bs = [m[2].clone() for m in mats]
+        nsg.dmuon_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
+                       ns_steps=steps, wd=0.1)
+        torch.cuda.synchronize()
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        nsg.dmuon_release_workspace()
+        return [bits(t) for t in ps + bs]
+
+    for steps in (w.ns_steps, 1, 2):
+        a, b = run(True, steps), run(False, steps)
+        assert all(np.array_equal(x, y) for x, y in zip(a, b)), steps
+
+
+def test_step_fused_update_unaligned_parameter():
+    # a parameter view 2 bytes off a 16-byte boundary takes the scalar path
+    # of the fused epilogue (both orientations)
+    for shape in ((256, 520), (520, 256)):
+        gen = torch.Generator().manual_seed(7)
+        base = (torch.randn(shape[0] * shape[1] + 1, generator=gen) * 0.02).to(torch.bfloat16).to(DEV)
+        p = base[1:].view(*shape)
+        g = torch.randn(*shape, generator=gen).to(torch.bfloat16).to(DEV)
+        b = torch.zeros(*shape, dtype=torch.bfloat16, device=DEV)
+        p_old = to64(p)
+        head = bits(base[:1])
+        nsg.dmuon_step([p], [g], [b], wd=0.1)
+        torch.cuda.synchronize()
+        want, _, _ = om.muon_step([p_old], [to64(g)], [np.zeros(shape)], 0.02, 0.95, True, 5, None, 0.1)
+        err = np.linalg.norm(to64(p) - want[0])
+        assert err <= 2e-2 * np.linalg.norm(want[0] - p_old) + 2 ** -8 * np.linalg.norm(want[0])
+        assert np.array_equal(head, bits(base[:1]))  # the element before the view is untouched

@@ -59,7 +59,7 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--ns-steps", type=int, default=None,
                     help="override the workload's Newton-Schulz iteration count")
-    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update"],
+    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update", "step"],
                     help="time one kernel through its stage call instead of the whole step")
     ap.add_argument("--clip-norm", type=float, default=None,
                     help="time dmuon_step_clipped: global 2-norm clipping of the gradients to this bound")
@@ -90,7 +90,10 @@ def launches_per_matrix(kernel: str, m: int, n: int, dtype: str, steps: int):
     blocked = mode != "0" and 4 * n >= 5 * m and steps >= 2
     if blocked and mode == "2":
         return None
-    return steps - 1 if blocked else steps
+    applies = steps - 1 if blocked else steps
+    # the last apply updates the parameters itself (apply_update_tc) unless disabled
+    fused = os.environ.get("DMUON_FUSED_UPDATE", "1")[:1] != "0" and steps >= 1
+    return applies - 1 if fused else applies
 
 
 def traffic_record(kernel: str, w, launches: int):
@@ -611,6 +614,16 @@ def run_stage(args):
         out = torch.empty_like(X)
         run = lambda: nsg.dmuon_poly_apply(P, X, out, 3.4445)  # noqa: E731
         flops, nbytes = 2 * b * m * m * n, 2 * b * (m * m + 2 * m * n)
+    elif args.stage == "step":
+        # a whole step over `batch` m x n matrices (rows x cols as given): the
+        # way to reach the apply with the fused update (its last launch)
+        steps = 1 if args.ns_steps is None else args.ns_steps
+        ps = [(torch.randn(m, n, generator=gen, device=dev) * 0.02).to(bf) for _ in range(b)]
+        gs = [torch.randn(m, n, generator=gen, device=dev).to(bf) for _ in range(b)]
+        bs = [torch.zeros(m, n, dtype=bf, device=dev) for _ in range(b)]
+        run = lambda: nsg.dmuon_step(ps, gs, bs, ns_steps=steps)  # noqa: E731
+        lo, hi = min(m, n), max(m, n)
+        flops, nbytes = b * steps * (3 * lo * lo * hi + lo ** 3), 0
     elif args.stage == "momentum":
         g = torch.randn(m, n, generator=gen, device=dev).to(bf)
         buf = torch.randn(m, n, generator=gen, device=dev).to(bf)
@@ -637,7 +650,7 @@ def run_stage(args):
         raise RuntimeError("stage call failed")
     print(json.dumps({"stage": args.stage, "batch": b, "m": m, "n": n, "ms": round(ms, 4),
                       "tflops": round(flops / (ms / 1e3) / 1e12, 1) if flops else None,
-                      "GB/s": round(nbytes / (ms / 1e3) / 1e9, 1)}), flush=True)
+                      "GB/s": round(nbytes / (ms / 1e3) / 1e9, 1) if nbytes else None}), flush=True)
 
 
 def main(argv=None):

@@ -59,7 +59,7 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--ns-steps", type=int, default=None,
                     help="override the workload's Newton-Schulz iteration count")
-    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update", "step"],
+    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update", "step", "clip"],
                     help="time one kernel through its stage call instead of the whole step")
     ap.add_argument("--clip-norm", type=float, default=None,
                     help="time dmuon_step_clipped: global 2-norm clipping of the gradients to this bound")
@@ -624,6 +624,11 @@ def run_stage(args):
         run = lambda: nsg.dmuon_step(ps, gs, bs, ns_steps=steps)  # noqa: E731
         lo, hi = min(m, n), max(m, n)
         flops, nbytes = b * steps * (3 * lo * lo * hi + lo ** 3), 0
+    elif args.stage == "clip":
+        # standalone clipping of `batch` m x n gradients: norm pass + in-place scale
+        gs = [torch.randn(m, n, generator=gen, device=dev).to(bf) for _ in range(b)]
+        run = lambda: nsg.dmuon_clip_grad_norm(gs, 1.0)  # noqa: E731
+        flops, nbytes = 0, 2 * b * m * n * 3
     elif args.stage == "momentum":
         g = torch.randn(m, n, generator=gen, device=dev).to(bf)
         buf = torch.randn(m, n, generator=gen, device=dev).to(bf)
@@ -640,15 +645,20 @@ def run_stage(args):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    nsg.dmuon_profile_start()
     e0.record()
     for _ in range(args.steps):
         run()
     e1.record()
     e1.synchronize()
+    kstats = nsg.dmuon_profile_stop()
     ms = e0.elapsed_time(e1) / args.steps
     if nsg.dmuon_stream_status() != nsg.DMUON_OK:
         raise RuntimeError("stage call failed")
-    print(json.dumps({"stage": args.stage, "batch": b, "m": m, "n": n, "ms": round(ms, 4),
+    kernels = {k: {"ms": round(v["total_ms"] / args.steps, 4),
+                   "GB/s": round(v["bytes"] / (v["total_ms"] / 1e3) / 1e9, 1) if v["bytes"] else None}
+               for k, v in kstats.items()}
+    print(json.dumps({"stage": args.stage, "batch": b, "m": m, "n": n, "ms": round(ms, 4), "kernels": kernels,
                       "tflops": round(flops / (ms / 1e3) / 1e12, 1) if flops else None,
                       "GB/s": round(nbytes / (ms / 1e3) / 1e9, 1) if nbytes else None}), flush=True)
 

@@ -383,9 +383,7 @@ dmuon_status_t parse_clip(float max_norm, float norm_type, int* p) {
   return DMUON_OK;
 }
 
-int64_t tiles_of(int64_t rows, int64_t cols) {
-  return ((rows + kElemTile - 1) / kElemTile) * ((cols + kElemTile - 1) / kElemTile);
-}
+int64_t tiles_of(int64_t rows, int64_t cols) { return (rows * cols + kClipChunk - 1) / kClipChunk; }
 
 int64_t clip_tiles(const std::vector<Group>& groups) {
   int64_t t = 0;
@@ -416,8 +414,7 @@ cudaError_t for_each_clip_table(const std::vector<Group>& groups, const void* co
       tab->tiles_per_mat = tpm;
       for (int j = 0; j < b; ++j) {
         const int32_t i = g.members[start + j];
-        const bool row16 = (g.cols * (int64_t)es) % 16 == 0 && aligned16(grads[i]);
-        tab->e[j] = MatEntry{grads[i], const_cast<void*>(grads[i]), nullptr, 0, row16 ? 1 : 0};
+        tab->e[j] = MatEntry{grads[i], const_cast<void*>(grads[i]), nullptr, 0, aligned16(grads[i]) ? 1 : 0};
       }
       cudaError_t e = fn(*tab, g.dtype, offset, (double)b * (double)g.rows * (double)g.cols * (double)es);
       if (e != cudaSuccess) return e;

@@ -5,19 +5,25 @@
 //   total = (sum over all matrices and elements of |g|^p)^(1/p)   (p = inf: max |g|)
 //   coef  = min(1, max_norm / (total + 1e-6));   g <- fl(g * fl32(coef))
 //
-// Three launches, all on the caller's stream: per 64 x 64 tile partials of
-// sum |g|^p (or max |g|) for every launch class of matrices; one block that
-// reduces all partials in a fixed order in fp64 and computes the coefficient;
-// an in-place scaling pass (a multiply by 1.0f when nothing is clipped, which
-// leaves every value unchanged).  Deterministic: no atomics.
+// Three launches, all on the caller's stream: per-chunk partials of sum |g|^p
+// (or max |g|) for every launch class of matrices; one block that reduces all
+// partials in a fixed order in fp64 and computes the coefficient; an in-place
+// scaling pass (a multiply by 1.0f when nothing is clipped, which leaves every
+// value unchanged).  Deterministic: no atomics.  The norm needs no 2D
+// structure, so each matrix is read as one flat array: a block covers a
+// contiguous chunk of 256 threads x 2 loads x 8 elements, and every warp load
+// is 32 consecutive 8-element vectors.  Measured on 128 x 4096^2 bf16 (norm +
+// scale, 3 passes): 2 loads per thread at 8 resident blocks per SM 5.79 TB/s;
+// 4 loads at 6 blocks 5.22; 8 loads (80 registers, 3 blocks) 3.74.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dmuon {
 namespace {
 
-constexpr int T64 = kElemTile;
 constexpr int kThreads = 256;
+constexpr int kLoads = 2;  // per thread, 8 elements each
+static_assert(kClipChunk == kThreads * kLoads * 8, "chunk size");
 
 __device__ __forceinline__ int clamp8(int64_t v) { return v < 8 ? (int)v : 8; }
 
@@ -41,31 +47,35 @@ __device__ __forceinline__ float combine(float a, float b) {
 }
 
 template <typename T, int P>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 8)
     k_clip_partials(const __grid_constant__ ElemTable tab, float* __restrict__ partials) {
   __shared__ float red[kThreads / 32];
   const int e = blockIdx.y;
   const MatEntry& me = tab.e[e];
-  const int64_t R = tab.m, C = tab.n;  // source layout, no orientation here
-  const int64_t tilesC = (C + T64 - 1) / T64;
-  const int64_t r0 = (blockIdx.x / tilesC) * T64;
-  const int64_t c0 = (blockIdx.x % tilesC) * T64;
+  const int64_t N = tab.m * tab.n;
+  const int64_t base = (int64_t)blockIdx.x * kClipChunk;
   const int tid = threadIdx.x;
-  const int cv = tid & 7, rr = tid >> 3;
   const bool vec = (me.pad & 1) != 0;
   const T* g = static_cast<const T*>(me.src);
+  float v[kLoads][8];
+  int valid[kLoads];
+#pragma unroll
+  for (int h = 0; h < kLoads; ++h) {
+    const int64_t i = base + ((int64_t)h * kThreads + tid) * 8;
+    valid[h] = i < N ? clamp8(N - i) : 0;
+    if (valid[h] > 0) {
+      load8<T>(g + i, v[h], vec && valid[h] == 8, valid[h]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[h][k] = 0.f;
+    }
+  }
   float acc = 0.f;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t gr = r0 + rr + 32 * h, gc = c0 + cv * 8;
-    if (gr >= R || gc >= C) continue;
-    const int valid = clamp8(C - gc);
-    float v[8];
-    load8<T>(g + gr * C + gc, v, vec && valid == 8, valid);
+  for (int h = 0; h < kLoads; ++h)
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (i < valid) acc = accum<P>(acc, v[i]);
-  }
+    for (int k = 0; k < 8; ++k)
+      if (k < valid[h]) acc = accum<P>(acc, v[h][k]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc = combine<P>(acc, __shfl_xor_sync(0xffffffffu, acc, o));
   if ((tid & 31) == 0) red[tid >> 5] = acc;
@@ -104,30 +114,30 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 8)
     k_clip_scale(const __grid_constant__ ElemTable tab, const float* __restrict__ coef) {
   const int e = blockIdx.y;
   const MatEntry& me = tab.e[e];
-  const int64_t R = tab.m, C = tab.n;
-  const int64_t tilesC = (C + T64 - 1) / T64;
-  const int64_t r0 = (blockIdx.x / tilesC) * T64;
-  const int64_t c0 = (blockIdx.x % tilesC) * T64;
+  const int64_t N = tab.m * tab.n;
+  const int64_t base = (int64_t)blockIdx.x * kClipChunk;
   const int tid = threadIdx.x;
-  const int cv = tid & 7, rr = tid >> 3;
   const bool vec = (me.pad & 1) != 0;
   T* g = static_cast<T*>(me.buf);
   const float k = *coef;
+  float v[kLoads][8];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t gr = r0 + rr + 32 * h, gc = c0 + cv * 8;
-    if (gr >= R || gc >= C) continue;
-    const int valid = clamp8(C - gc);
-    const bool v8 = vec && valid == 8;
-    float v[8];
-    load8<T>(g + gr * C + gc, v, v8, valid);
+  for (int h = 0; h < kLoads; ++h) {
+    const int64_t i = base + ((int64_t)h * kThreads + tid) * 8;
+    if (i < N) load8<T>(g + i, v[h], vec && N - i >= 8, clamp8(N - i));
+  }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], k);
-    store8<T>(g + gr * C + gc, v, v8, valid);
+  for (int h = 0; h < kLoads; ++h) {
+    const int64_t i = base + ((int64_t)h * kThreads + tid) * 8;
+    if (i < N) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[h][q] = __fmul_rn(v[h][q], k);
+      store8<T>(g + i, v[h], vec && N - i >= 8, clamp8(N - i));
+    }
   }
 }
 

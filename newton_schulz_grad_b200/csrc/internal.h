@@ -82,9 +82,13 @@ cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, 
                        const float* scale, bool xbf16, cudaStream_t st);
 
 // ---- clip.cu --------------------------------------------------------------------
+// Each matrix is read as a flat array of rows * cols elements; one partial per
+// chunk of kClipChunk elements (ceil(rows * cols / kClipChunk) per matrix).
+constexpr int kClipChunk = 4096;
 // Global p-norm clipping (p = 0 means the infinity norm).  Tables hold
-// matrices of one source shape (m = rows, n = cols, not oriented); `src` is
-// read for the norm, `buf` scaled in place.
+// matrices of one source shape (m = rows, n = cols, not oriented; tiles_per_mat
+// = chunks per matrix); `src` is read for the norm, `buf` scaled in place; pad
+// bit 0: the base is 16-byte aligned.
 cudaError_t launch_clip_partials(const ElemTable& t, int dtype, int p, float* partials, cudaStream_t st);
 cudaError_t launch_clip_coef(const float* partials, int64_t count, int p, float max_norm, float* coef,
                              double* total, cudaStream_t st);

@@ -2,9 +2,9 @@
 
 DMuon Training Guide, "Gradient Clipping": the Muon gradients are clipped by
 their global p-norm after the reduce and before momentum + Newton-Schulz.
-The norm is compared with the oracle's fp64 norm (per-tile fp32 partials,
-then a fixed-order fp64 sum: relative error ~ sqrt(64*64) fp32 roundings at
-most, bounded here by 1e-5); the scaled values are compared bit for bit with
+The norm is compared with the oracle's fp64 norm (fp32 partials of 4096
+elements, each a chain of at most 16 + 5 + 8 fp32 roundings, then a fixed-order
+fp64 sum: relative error below 29 * 2^-24 ~ 1.7e-6, bounded here by 1e-5); the scaled values are compared bit for bit with
 the fp32 rounding contract fl(g * fl32(coef)), with the coefficient the GPU
 read back, and the coefficient itself with the oracle's to 1e-5.
 """

@@ -1,8 +1,8 @@
-"""Parity at the full benchmark size: the 224-matrix Llama-7B projection set.
+"""Parity at the full benchmark sizes: the Llama-7B, Llama-3.2-3B and MoE sets.
 
-The whole set runs through one dmuon_step call, exactly as the benchmark
-launches it; the oracle then recomputes one sampled matrix per launch class
-(4096x4096, 11008x4096 transposed, 4096x11008) in fp64 on the host.
+Each whole set runs through one dmuon_step call, exactly as the benchmark
+launches it; the oracle then recomputes sampled matrices of every launch class
+(e.g. 4096x4096, 11008x4096 transposed, 4096x11008) in fp64 on the host.
 """
 import numpy as np
 import pytest
@@ -17,11 +17,8 @@ from tests.gpu_util import to64
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
-def test_llama7b_full_step_sampled_parity():
-    w = workloads.get("llama_7b_bf16")
+def full_step_sampled_parity(w, sample):
     ps, gs, bs = workloads.make_all(w, "cuda")
-    sample = [1, 4, 6]  # k_proj (4096x4096), gate_proj (11008x4096), down_proj (4096x11008)
-    sample += [w.count - 3]  # a last-layer gate_proj (last chunk of its class)
     saved = {i: (to64(ps[i]), gs[i].float().cpu().numpy(), bs[i].float().cpu().numpy())
              for i in sample}
     nsg.dmuon_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
@@ -37,9 +34,32 @@ def test_llama7b_full_step_sampled_parity():
         step = np.linalg.norm(p_new[0] - p0)
         err = np.linalg.norm(got - p_new[0])
         assert err <= 2e-2 * step + 2 ** -8 * np.linalg.norm(p_new[0]), (i, err / step)
-    # every parameter moved and stayed finite
+    # every parameter stayed finite
     for p in ps:
         assert torch.isfinite(p).all()
+
+
+def test_llama7b_full_step_sampled_parity():
+    w = workloads.get("llama_7b_bf16")
+    sample = [1, 4, 6]  # k_proj (4096x4096), gate_proj (11008x4096), down_proj (4096x11008)
+    sample += [w.count - 3]  # a last-layer gate_proj (last chunk of its class)
+    full_step_sampled_parity(w, sample)
+
+
+def test_llama3_2_3b_full_step_sampled_parity():
+    # 196 matrices, wd = 0.1; q (3072^2), k (1024x3072), gate (8192x3072,
+    # transposed), down (3072x8192), and the last layer's up_proj
+    w = workloads.get("llama3_2_3b_bf16")
+    full_step_sampled_parity(w, [0, 1, 4, 6, w.count - 2])
+
+
+def test_moe_full_step_sampled_parity():
+    # 248 matrices: expert gate (1408x2048) and down (2048x1408), the first and
+    # last of the seed-chosen 1e-4-scaled matrices, a thin 32x4096 GateDelta
+    # projection (clustered one-launch chain) and a tall 16384x2048 matrix
+    w = workloads.get("moe_skewed_bf16")
+    sk = workloads.skewed_indices(w)
+    full_step_sampled_parity(w, sorted({0, 2, sk[0], sk[-1], 192, w.count - 1}))
 
 
 @pytest.mark.parametrize("shape", [(16384, 24576), (24576, 16384)])

@@ -963,16 +963,31 @@ int tri_tiles(int tiles_m, int tiles_n, int tm) {
   return t;
 }
 
-// The CTA-pair kernel runs when the matrix fills 256-row tiles; setting
 // DMUON_TC_CTA_PAIR=0 forces the one-CTA kernel (for comparisons).
-bool use_pair(int m) {
+// CTA pair (256-row tiles) or one CTA (128-row tiles).  The pair runs about
+// 6 % faster per computed tile element (apply at 4096^2: 1378 vs 1300
+// TFLOP/s), so it is used unless the 128-row tiling computes enough less
+// area: m just above a multiple of 256 (e.g. 1408, 5.5 pair tiles).
+// Triangle kernels (gram, poly) compare their lower-triangle tile sets.
+bool use_pair(int m, bool triangle) {
   static int mode = -1;
   static std::once_flag once;
   std::call_once(once, [] {
     const char* e = std::getenv("DMUON_TC_CTA_PAIR");
     mode = (e && std::strcmp(e, "0") == 0) ? 0 : 1;
   });
-  return mode == 1 && m >= 256;
+  if (mode != 1 || m < 256) return false;
+  constexpr double kOneCtaCost = 1.06;
+  double pair_area, one_area;
+  if (triangle) {
+    const int tn = (m + BN - 1) / BN;
+    pair_area = tri_tiles((m + BM2 - 1) / BM2, tn, BM2) * (double)BM2;
+    one_area = tri_tiles((m + BM1 - 1) / BM1, tn, BM1) * (double)BM1;
+  } else {
+    pair_area = (double)((m + BM2 - 1) / BM2) * BM2;
+    one_area = (double)((m + BM1 - 1) / BM1) * BM1;
+  }
+  return one_area * kOneCtaCost >= pair_area;
 }
 
 template <int MODE, bool UPD = false>
@@ -1005,7 +1020,7 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int 
 cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg, float alpha,
                     const float* scale, int* status, int num_sms, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
-  const bool pair = use_pair(m);
+  const bool pair = use_pair(m, true);
   CUtensorMap ma, mb;
   // A: 128 rows per CTA; B: 256 rows (one CTA) or 128 rows per CTA (pair)
   cudaError_t e = make_map(&ma, X, n, m, batch, ldx, BK, 128);
@@ -1031,7 +1046,7 @@ cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int ba
                     int64_t ldb, int64_t lde, int64_t ldc, float p0, float p1, float p2, int* status, int num_sms,
                     cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
-  const bool pair = use_pair(m);
+  const bool pair = use_pair(m, true);
   CUtensorMap ma, mb;
   cudaError_t e = make_map(&ma, A, m, m, batch, lda, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, B, m, m, batch, ldb, BK, pair ? 128 : BN);
@@ -1064,7 +1079,7 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
                      int64_t ldx, int64_t ldy, float a_coef, float alpha, const float* scale, int* status,
                      int num_sms, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
-  const bool pair = use_pair(m);
+  const bool pair = use_pair(m, false);
   CUtensorMap ma, mb;
   cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
@@ -1093,7 +1108,7 @@ cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int 
                             int num_sms, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
   if (batch > kMaxTable) return cudaErrorInvalidValue;
-  const bool pair = use_pair(m);
+  const bool pair = use_pair(m, false);
   CUtensorMap ma, mb;
   cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);

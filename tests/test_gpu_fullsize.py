@@ -87,3 +87,67 @@ def test_large_diagonal_closed_form(shape):
     total = float(out.double().pow(2).sum().item())
     assert abs(total - float(np.sum(got ** 2))) <= 1e-12 * total   # nothing off the diagonal
     assert torch.isfinite(out).all()
+
+
+def _f5(s):
+    a, b, c = (float(np.float32(v)) for v in om.DEFAULT_COEFFS)
+    for _ in range(5):
+        s = a * s + b * s ** 3 + c * s ** 5
+    return s
+
+
+def _sumsq_rows(t, rows=2048):
+    return sum(float((t[i:i + rows].float() ** 2).sum(dtype=torch.float64)) for i in range(0, t.shape[0], rows))
+
+
+@pytest.mark.parametrize("shape", [(32768, 65535), (65535, 32768)])
+def test_max_elements_step_diagonal_closed_form(shape):
+    # The largest matrix the ABI takes (rows * cols < 2^31; 18 GiB of
+    # workspace, over the default cap, so a chunk of its own), through a whole
+    # dmuon_step: gradient [D | 0] (or its transpose), zero buffer and
+    # parameter.  The buffer becomes the gradient bit for bit, x0 = bf16(g +
+    # 0.95 g) stays diagonal, NS(x0) = diag(f^5(x0_i / ||x0||)) exactly in real
+    # arithmetic, and p' = -fl32(lr 0.2 sqrt(max side)) NS(x0) with nothing off
+    # the diagonal.  Runs the transposing momentum pass, every tile of the pair
+    # kernels, the Gram-space block and the fused update (column writes of p
+    # for the tall orientation) at the maximum size.
+    R, C = shape
+    m = min(R, C)
+    d = (1.0 + torch.arange(m, dtype=torch.float32) / m).to(torch.bfloat16)
+    g = torch.zeros(R, C, dtype=torch.bfloat16, device="cuda")
+    g.diagonal().copy_(d.cuda())
+    p = torch.zeros_like(g)
+    buf = torch.zeros_like(g)
+    lr = 0.02
+    nsg.dmuon_step([p], [g], [buf], lr=lr, momentum=0.95, nesterov=True, ns_steps=5, wd=0.0)
+    torch.cuda.synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    assert torch.equal(buf.diagonal(), g.diagonal()) and _sumsq_rows(buf) == _sumsq_rows(g)
+    dd = d.float().numpy()
+    _, x0 = em.momentum_fp32(np.zeros_like(dd), dd, 0.95, True, "bf16")
+    x0 = x0.astype(np.float64)
+    s = x0 / (np.linalg.norm(x0) + om.NORM_EPS)
+    want = -float(em.update_scale(lr, R, C)) * _f5(s)
+    got = p.diagonal().double().cpu().numpy()
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) < 2e-2
+    assert abs(_sumsq_rows(p) - float(np.sum(got ** 2))) <= 1e-9 * float(np.sum(got ** 2))
+    nsg.dmuon_release_workspace()
+
+
+@pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, 2e-2), (torch.float32, 1e-4)], ids=["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 1 << 20), (1 << 20, 1)])
+def test_longest_side_vector_closed_form(shape, dtype, tol):
+    # A vector has one singular value, ||x|| / (||x|| + eps) ~ 1 after the
+    # normalisation, so NS(x) = f^5(1) x / ||x|| (f^5(1) = 0.69644 for the
+    # default coefficients); 2^20 is the longest side the ABI takes
+    gen = torch.Generator().manual_seed(5)
+    x = torch.randn(*shape, generator=gen).to(dtype)
+    out = torch.empty_like(x).cuda()
+    nsg.dmuon_ns(x.cuda(), out, steps=5)
+    torch.cuda.synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    xv = x.double().numpy().ravel()
+    nx = np.linalg.norm(xv)
+    want = _f5(nx / (nx + om.NORM_EPS)) * xv / nx
+    got = out.double().cpu().numpy().ravel()
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) < tol

@@ -28,8 +28,20 @@
  *  - Arguments are validated on the host before anything is launched; on an
  *    error nothing is modified and the status says why (dmuon_get_last_error()
  *    holds a message, per host thread).
+ *  - A CUDA error after launches began (DMUON_ERR_CUDA) can leave a step
+ *    partly done (some buffers or parameters updated); the call still returns
+ *    with all of its work ordered before later work on `stream`, so the
+ *    caller can synchronise and restore its own copy.  DMUON_FAULT_INJECT=
+ *    launch makes dmuon_step report such a failure before its first chain
+ *    (momentum of the first chunk done, no parameter touched), for tests.
  *  - Device waits inside the kernels are bounded; a wait that runs out sets a
  *    per-device status word read by dmuon_stream_status() (DMUON_ERR_TIMEOUT).
+ *  - A debug build of the library (compiled with -DDMUON_DEBUG:
+ *    `build.py --debug` writes libdmuon_b200_debug.so) checks every global
+ *    access of its kernels against the extent of the buffer it belongs to,
+ *    computed on the host; an access outside is skipped and the status word
+ *    records DMUON_ERR_BOUNDS (no trap, no fault).  Release builds carry no
+ *    checks.
  *  - Results do not depend on how matrices are batched: a matrix gives the
  *    same bits alone, inside its group, or in a permuted list.
  */
@@ -57,7 +69,9 @@ typedef enum {
     DMUON_ERR_UNSUPPORTED = 2, /* no sm_100 device, or a size beyond a limit  */
     DMUON_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed             */
     DMUON_ERR_OOM = 4,         /* workspace allocation failed                   */
-    DMUON_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out            */
+    DMUON_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out            */
+    DMUON_ERR_BOUNDS = 6       /* debug builds: an access outside its buffer was
+                                  caught and skipped (see dmuon_stream_status)  */
 } dmuon_status_t;
 
 typedef enum {
@@ -295,7 +309,8 @@ DMUON_API const char* dmuon_get_last_error(void);
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device: DMUON_ERR_TIMEOUT if a device-side wait ran out since the
- * last call, DMUON_ERR_CUDA if the stream reports an error, else DMUON_OK. */
+ * last call, DMUON_ERR_BOUNDS if a debug build caught an access outside its
+ * buffer, DMUON_ERR_CUDA if the stream reports an error, else DMUON_OK. */
 DMUON_API dmuon_status_t dmuon_stream_status(dmuon_stream_t stream);
 
 /* Self-test of failure detection: launches one thread that waits on a device
@@ -305,6 +320,14 @@ DMUON_API dmuon_status_t dmuon_stream_status(dmuon_stream_t stream);
  * returns; the next dmuon_stream_status() reports DMUON_ERR_TIMEOUT and clears
  * the word, and the context stays usable. */
 DMUON_API dmuon_status_t dmuon_selftest_timeout(int32_t limit_us, dmuon_stream_t stream);
+
+/* Self-test of the debug build's bounds checks: launches one thread that
+ * evaluates a single check of an element offset just past a one-element
+ * extent, and touches no memory either way.  In a debug build the check fails
+ * and records DMUON_ERR_BOUNDS, which the next dmuon_stream_status() reports
+ * (and clears); in a release build there are no checks and the status stays
+ * DMUON_OK.  dmuon_build_info() names the build ("debug bounds checks"). */
+DMUON_API dmuon_status_t dmuon_selftest_bounds(dmuon_stream_t stream);
 
 /* Frees every cached workspace of the calling thread's current device after
  * synchronising the device.  Safe to call at any time between calls. */

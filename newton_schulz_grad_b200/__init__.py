@@ -25,8 +25,10 @@ DMUON_ERR_UNSUPPORTED = 2
 DMUON_ERR_CUDA = 3
 DMUON_ERR_OOM = 4
 DMUON_ERR_TIMEOUT = 5
+DMUON_ERR_BOUNDS = 6
 STATUS_NAMES = {0: "DMUON_OK", 1: "DMUON_ERR_INVALID_ARG", 2: "DMUON_ERR_UNSUPPORTED",
-                3: "DMUON_ERR_CUDA", 4: "DMUON_ERR_OOM", 5: "DMUON_ERR_TIMEOUT"}
+                3: "DMUON_ERR_CUDA", 4: "DMUON_ERR_OOM", 5: "DMUON_ERR_TIMEOUT",
+                6: "DMUON_ERR_BOUNDS"}
 DMUON_F32 = 0
 DMUON_BF16 = 1
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -36,7 +38,7 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_get_last_error", "dmuon_stream_status", "dmuon_release_workspace",
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
             "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout",
-            "dmuon_clip_grad_norm", "dmuon_step_clipped")
+            "dmuon_clip_grad_norm", "dmuon_step_clipped", "dmuon_selftest_bounds")
 
 
 class DmuonError(RuntimeError):
@@ -88,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
         "dmuon_selftest_timeout": ([i32, vp], i32),
         "dmuon_clip_grad_norm": ([ctypes.POINTER(vp), ctypes.POINTER(Shape), i32, f32, f32, vp, vp], i32),
+        "dmuon_selftest_bounds": ([vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -371,6 +374,11 @@ def dmuon_stream_status(stream=None) -> int:
 def dmuon_selftest_timeout(limit_us: int = 50000, stream=None) -> None:
     """Launch a kernel whose bounded device wait is made to run out (see dmuon.h)."""
     _check(_lib.dmuon_selftest_timeout(int(limit_us), _stream(stream)))
+
+
+def dmuon_selftest_bounds(stream=None) -> None:
+    """Evaluate one deliberately failing bounds check (see dmuon.h); touches no memory."""
+    _check(_lib.dmuon_selftest_bounds(_stream(stream)))
 
 
 def dmuon_get_last_error() -> str:

@@ -6,8 +6,11 @@ then linked into one shared library next to this file (the CUDA runtime is
 linked statically, so the library only needs the driver at run time).  Only
 symbols declared ``DMUON_API`` in ``include/dmuon.h`` are exported.
 
-Usage: ``python newton_schulz_grad_b200/build.py [--force] [--verbose]`` (run by path: importing
-the package loads the library this script produces).
+Usage: ``python newton_schulz_grad_b200/build.py [--force] [--verbose] [--debug]`` (run by
+path: importing the package loads the library this script produces).  ``--debug`` builds
+``libdmuon_b200_debug.so`` instead, with ``-DDMUON_DEBUG``: every global access of the
+kernels is checked against its buffer's extent and skipped, with DMUON_ERR_BOUNDS in the
+status word, when it falls outside (load it with DMUON_LIBRARY=<path>).
 """
 from __future__ import annotations
 
@@ -24,6 +27,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libdmuon_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
+DEBUG_LIB_PATH = os.path.join(HERE, "libdmuon_b200_debug.so")
 
 SOURCES = ["api.cu", "plan.cpp", "elementwise.cu", "simt_gemm.cu", "tc_gemm.cu", "noalloc.cu", "small_ns.cu", "clip.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -48,17 +52,20 @@ def _newest(paths) -> float:
     return max(os.path.getmtime(p) for p in paths if os.path.exists(p))
 
 
-def build(force: bool = False, verbose: bool = False, extra: List[str] = None) -> str:
+def build(force: bool = False, verbose: bool = False, extra: List[str] = None, debug: bool = False) -> str:
     """Compile and link if any source is newer than the library; return its path."""
-    extra = list(extra or [])
-    if (not force and not extra and os.path.exists(LIB_PATH)
-            and os.path.getmtime(LIB_PATH) >= _newest(_deps())):
-        return LIB_PATH
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    user_extra = list(extra or [])
+    lib = DEBUG_LIB_PATH if debug else LIB_PATH
+    build_dir = os.path.join(BUILD_DIR, "debug") if debug else BUILD_DIR
+    if (not force and not user_extra and os.path.exists(lib)
+            and os.path.getmtime(lib) >= _newest(_deps())):
+        return lib
+    extra = user_extra + (["-DDMUON_DEBUG"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     objs = []
     for src in SOURCES:
-        obj = os.path.join(BUILD_DIR, src + ".o")
+        obj = os.path.join(build_dir, src + ".o")
         cmd = [cc] + ARCH + COMMON + extra + ["-c", os.path.join(CSRC, src), "-o", obj]
         if src.endswith(".cpp"):
             cmd = ["g++", "-O3", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-I", INCLUDE,
@@ -68,17 +75,18 @@ def build(force: bool = False, verbose: bool = False, extra: List[str] = None) -
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB_PATH + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [cc] + ARCH + ["-shared", "-Xcompiler", "-fvisibility=hidden", "-o", tmp] + objs
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     force = "--force" in sys.argv
     verbose = "--verbose" in sys.argv
-    extra = [a for a in sys.argv[1:] if a not in ("--force", "--verbose")]
-    print(build(force=force, verbose=verbose, extra=extra))
+    debug = "--debug" in sys.argv
+    extra = [a for a in sys.argv[1:] if a not in ("--force", "--verbose", "--debug")]
+    print(build(force=force, verbose=verbose, extra=extra, debug=debug))

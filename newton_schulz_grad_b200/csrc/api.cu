@@ -17,8 +17,12 @@
 // (per-iteration form | Gram-space blocks of 2, 3, 3, ...),
 // DMUON_TC_CTA_PAIR=0 (one-CTA tensor-core kernel only, read once),
 // DMUON_SMALL_CHAIN=0 (thin matrices on the per-product FFMA kernels),
-// DMUON_FAULT_INJECT=alloc (workspace allocation fails, for tests).
+// DMUON_FAULT_INJECT=alloc (workspace allocation fails) or =launch (dmuon_step
+// reports a failed launch before its first chain), for tests;
+// DMUON_NVTX=1 (NVTX ranges per step, chunk chain and clip stage, for
+// profilers: `ncu --nvtx --nvtx-include "dmuon_step/"`).
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -32,6 +36,7 @@
 #include <utility>
 #include <vector>
 
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace dmuon {
@@ -87,6 +92,21 @@ bool env_is(const char* name, char first) {
   const char* e = std::getenv(name);
   return e && e[0] == first;
 }
+
+// An NVTX range for the scope when DMUON_NVTX=1 (a no-op without a tool attached).
+struct NvtxRange {
+  bool on;
+  explicit NvtxRange(const std::string& name) : on(env_is("DMUON_NVTX", '1')) {
+    if (on) nvtxRangePushA(name.c_str());
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+};
+
+// One check of element offset 1 in a one-element extent; no memory is
+// touched in either build (release: the check is the constant true).
+__global__ void k_bounds_selftest(int* status) { (void)DMUON_IN(status, 1, 1, 1); }
 
 bool fault_injected(const char* what) {
   const char* e = std::getenv("DMUON_FAULT_INJECT");
@@ -270,7 +290,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   auto gram = [&](const void* X, void* out, const float* sc) {
     Prof p(tc ? kGramTc : kGramFfma, st, fb * fm * fm * fn, 0.0);
     e = tc ? tc_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, sw, sms, st)
-           : simt_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, xbf16, st);
+           : simt_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, xbf16, st, sw);
     p.done(st);
   };
   bool fused = false;
@@ -285,7 +305,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
     }
     Prof p(tc ? kApplyTc : kApplyFfma, st, 2.0 * fb * fm * fm * fn, 0.0);
     e = tc ? tc_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, sw, sms, st)
-           : simt_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st);
+           : simt_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st, sw);
     p.done(st);
   };
   // C = p1 (A B) + p0 E + p2 I on the tensor path (A, B symmetric and commuting)
@@ -299,7 +319,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   // thin matrices: the whole chain in one clustered launch, in place on X0
   if (thin_chain(L, m, n, steps)) {
     Prof p(kChainSmall, st, fb * (3.0 * fm * fm * fn + fm * fm * fm) * steps, 0.0);
-    e = small_ns(cur, b, mi, ni, L.ldn, steps, sched.data(), scale, xbf16, st);
+    e = small_ns(cur, b, mi, ni, L.ldn, steps, sched.data(), scale, xbf16, st, sw);
     p.done(st);
     if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
     *result = cur;
@@ -321,7 +341,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
       {
         Prof p(tc ? kPolyTc : kPolyFfma, st, fb * fm * fm * fm, 0.0);
         e = tc ? tc_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), sw, sms, st)
-               : simt_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), st);
+               : simt_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), st, sw);
         p.done(st);
       }
       if (e != cudaSuccess) break;
@@ -427,6 +447,7 @@ cudaError_t for_each_clip_table(const std::vector<Group>& groups, const void* co
 // The norm pass and the coefficient: coef = min(1, max_norm / (total + 1e-6)).
 cudaError_t clip_norm_stage(const std::vector<Group>& groups, const void* const* grads, const ClipReq& req,
                             void* ws, int64_t tiles, ElemTable* tab, cudaStream_t st) {
+  NvtxRange range("clip norm");
   float* partials = static_cast<float*>(ws);
   cudaError_t e = for_each_clip_table(groups, grads, tab, [&](const ElemTable& t, int32_t dtype, int64_t off, double bytes) {
     Prof pr(kClipNorm, st, 0.0, bytes);
@@ -443,6 +464,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
                          const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
                          int32_t nesterov, int32_t ns_steps, const float* coeffs, float wd,
                          const ClipReq* clip, dmuon_stream_t stream) {
+  NvtxRange range(clip ? "dmuon_step_clipped" : "dmuon_step");
   // ---------------------------------------------------------- validation
   if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
   if (ns_steps < 0 || ns_steps > 1000) return fail(DMUON_ERR_INVALID_ARG, "ns_steps must be in 0..1000");
@@ -489,6 +511,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
   rc = get_workspace(clip ? clip_off + clip_ws_bytes(clip_tile_count) : (size_t)(P.buffer_bytes * nbuf), st, &wsv);
   if (rc != DMUON_OK) return rc;
   std::unique_ptr<ElemTable[]> tabs(new ElemTable[2]);
+  tabs[0].status = tabs[1].status = ds.status_word;
   const float* clip_coef = nullptr;
   if (clip) {
     void* cws = static_cast<char*>(wsv) + clip_off;
@@ -504,6 +527,15 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     cudaError_t e = stream_after(aux, st);
     if (e != cudaSuccess) return cuda_fail(e, "stream fork");
   }
+  // Every return after the fork leaves the caller's stream ordered after aux,
+  // so a call that fails part-way leaves none of its work unordered.
+  struct JoinAux {
+    cudaStream_t st, aux;
+    bool on;
+    ~JoinAux() {
+      if (on) stream_after(st, aux);
+    }
+  } join{st, aux, P.overlap};
   std::vector<void*> results(P.chunks.size(), nullptr);
   std::unique_ptr<UpdTable> upd_tab(new UpdTable());
 
@@ -592,7 +624,14 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
       }
       upd = &u;
     }
-    rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &results[i], upd);
+    if (i == 0 && fault_injected("launch")) {
+      drop();
+      return cuda_fail(cudaErrorLaunchFailure, "first chain launch (injected failure)");
+    }
+    {
+      NvtxRange r("chain " + std::to_string(c.m) + "x" + std::to_string(c.n) + " x" + std::to_string(ck.b));
+      rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &results[i], upd);
+    }
     if (rc != DMUON_OK) {
       drop();
       return rc;
@@ -628,6 +667,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     if (e != cudaSuccess) return cuda_fail(e, "stream fork");
     rc = update(P.chunks.size() - 1);
     if (rc != DMUON_OK) return rc;
+    join.on = false;
     e = stream_after(st, aux);
     if (e != cudaSuccess) return cuda_fail(e, "stream join");
   }
@@ -648,7 +688,12 @@ const char* dmuon_get_last_error(void) { return g_last_error.c_str(); }
 
 const char* dmuon_build_info(void) {
   static std::string s = std::string("dmuon-b200 0.1.0; sm_100a; ") + tc_config_string() +
-                         "; FFMA chain for fp32 and min side <= 64; elementwise 64x64 tiles";
+                         "; FFMA chain for fp32 and min side <= 64; elementwise 64x64 tiles" +
+#ifdef DMUON_DEBUG
+                         "; debug bounds checks";
+#else
+                         "; release";
+#endif
   return s.c_str();
 }
 
@@ -737,6 +782,7 @@ dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* sha
   rc = get_workspace(clip_ws_bytes(tiles), st, &ws);
   if (rc != DMUON_OK) return rc;
   std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->status = ds.status_word;
   const void* const* cg = const_cast<const void* const*>(grads);
   cudaError_t e = clip_norm_stage(groups, cg, req, ws, tiles, tab.get(), st);
   if (e == cudaSuccess)
@@ -774,6 +820,7 @@ dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int64_t cols,
   if (rc != DMUON_OK) return rc;
   char* ws = static_cast<char*>(wsv);
   std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->status = ds.status_word;
   tab->m = m;
   tab->n = n;
   tab->ldn = L.ldn;
@@ -846,7 +893,7 @@ dmuon_status_t dmuon_gram(const void* X, void* G, int64_t batch, int64_t m, int6
   cudaError_t e = dtype == DMUON_BF16
                       ? tc_gram(X, G, (int)batch, (int)m, (int)n, ldx, ldg, alpha, nullptr, ds.status_word,
                                 ds.sm_count, st)
-                      : simt_gram(X, G, (int)batch, (int)m, (int)n, ldx, ldg, alpha, nullptr, false, st);
+                      : simt_gram(X, G, (int)batch, (int)m, (int)n, ldx, ldg, alpha, nullptr, false, st, ds.status_word);
   return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_gram");
 }
 
@@ -863,7 +910,7 @@ dmuon_status_t dmuon_gram_poly(const void* G, void* P, int64_t batch, int64_t m,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = dtype == DMUON_BF16
                       ? tc_poly(G, P, (int)batch, (int)m, ldg, ldp, b, c, ds.status_word, ds.sm_count, st)
-                      : simt_poly(G, P, (int)batch, (int)m, ldg, ldp, b, c, st);
+                      : simt_poly(G, P, (int)batch, (int)m, ldg, ldp, b, c, st, ds.status_word);
   return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_gram_poly");
 }
 
@@ -883,7 +930,7 @@ dmuon_status_t dmuon_poly_apply(const void* P, const void* X, void* Y, int64_t b
                       ? tc_apply(P, X, Y, (int)batch, (int)m, (int)n, ldp, ldx, ldy, a, alpha, nullptr,
                                  ds.status_word, ds.sm_count, st)
                       : simt_apply(P, X, Y, (int)batch, (int)m, (int)n, ldp, ldx, ldy, a, alpha, nullptr, false,
-                                   st);
+                                   st, ds.status_word);
   return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_poly_apply");
 }
 
@@ -899,6 +946,7 @@ dmuon_status_t dmuon_momentum(void* buf, const void* grad, void* x0, int64_t row
   if (rc != DMUON_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->status = ds.status_word;
   tab->m = rows;
   tab->n = cols;
   tab->ldn = cols;
@@ -928,6 +976,7 @@ dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, int64_t co
   if (rc != DMUON_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->status = ds.status_word;
   // not oriented: the table's (m, n) is the matrix itself
   const int64_t n = std::max(rows, cols);
   tab->m = rows;
@@ -1001,6 +1050,15 @@ dmuon_status_t dmuon_selftest_timeout(int32_t limit_us, dmuon_stream_t stream) {
   return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "self-test launch");
 }
 
+dmuon_status_t dmuon_selftest_bounds(dmuon_stream_t stream) {
+  DeviceState ds;
+  dmuon_status_t rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  k_bounds_selftest<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ds.status_word);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "self-test launch");
+}
+
 dmuon_status_t dmuon_stream_status(dmuon_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);
@@ -1013,7 +1071,9 @@ dmuon_status_t dmuon_stream_status(dmuon_stream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (word != 0) {
     cudaMemset(ds.status_word, 0, sizeof(int));
-    return fail((dmuon_status_t)word, "a device-side wait ran out (kernel gave up and returned)");
+    return fail((dmuon_status_t)word, word == DMUON_ERR_BOUNDS
+                                          ? "a kernel access fell outside its buffer (debug build: skipped)"
+                                          : "a device-side wait ran out (kernel gave up and returned)");
   }
   return DMUON_OK;
 }

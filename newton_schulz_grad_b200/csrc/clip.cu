@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads, 8)
   for (int h = 0; h < kLoads; ++h) {
     const int64_t i = base + ((int64_t)h * kThreads + tid) * 8;
     valid[h] = i < N ? clamp8(N - i) : 0;
-    if (valid[h] > 0) {
+    if (valid[h] > 0 && DMUON_IN(tab.status, i, valid[h], N)) {
       load8<T>(g + i, v[h], vec && valid[h] == 8, valid[h]);
     } else {
 #pragma unroll
@@ -128,12 +128,12 @@ __global__ void __launch_bounds__(kThreads, 8)
 #pragma unroll
   for (int h = 0; h < kLoads; ++h) {
     const int64_t i = base + ((int64_t)h * kThreads + tid) * 8;
-    if (i < N) load8<T>(g + i, v[h], vec && N - i >= 8, clamp8(N - i));
+    if (i < N && DMUON_IN(tab.status, i, clamp8(N - i), N)) load8<T>(g + i, v[h], vec && N - i >= 8, clamp8(N - i));
   }
 #pragma unroll
   for (int h = 0; h < kLoads; ++h) {
     const int64_t i = base + ((int64_t)h * kThreads + tid) * 8;
-    if (i < N) {
+    if (i < N && DMUON_IN(tab.status, i, clamp8(N - i), N)) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[h][q] = __fmul_rn(v[h][q], k);
       store8<T>(g + i, v[h], vec && N - i >= 8, clamp8(N - i));

@@ -5,7 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bounds.cuh"
+
 namespace dmuon {
+
 
 template <typename T>
 struct Elt;

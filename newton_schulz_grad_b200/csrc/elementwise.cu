@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
     int valid = 0;
     if (gr < R && gc < C) valid = clamp8(C - gc);
     float x[8];
-    if (valid > 0) {
+    if (valid > 0 && DMUON_IN(tab.status, gr * C + gc, valid, R * C)) {
       const bool v8 = src_vec && valid == 8;
       const int64_t off = gr * C + gc;
       float gv[8];
@@ -88,7 +88,10 @@ __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
         x[i] = (i < valid) ? round_to<T>(x[i]) : 0.f;
         ss = fmaf(x[i], x[i], ss);
       }
-      if (!tr) store8<T>(Xm + gr * tab.ldn + gc, x, dst_vec && valid == 8, valid);
+      if (!tr && DMUON_IN(tab.status, gc, valid, tab.ldn) &&
+          DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + gr * tab.ldn + gc, valid,
+                   (int64_t)tab.count * tab.m * tab.ldn))
+        store8<T>(Xm + gr * tab.ldn + gc, x, dst_vec && valid == 8, valid);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = 0.f;
@@ -110,7 +113,10 @@ __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
         float y[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) y[k] = s[j0 + k][i];
-        store8<T>(Xm + (c0 + i) * tab.ldn + r0 + j0, y, dst_vec && valid == 8, valid);
+        if (DMUON_IN(tab.status, r0 + j0, valid, tab.ldn) &&
+            DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + (c0 + i) * tab.ldn + r0 + j0, valid,
+                     (int64_t)tab.count * tab.m * tab.ldn))
+          store8<T>(Xm + (c0 + i) * tab.ldn + r0 + j0, y, dst_vec && valid == 8, valid);
       }
     }
   }
@@ -173,8 +179,10 @@ __global__ void __launch_bounds__(kThreads)
       const int i = rr + 32 * h;
       const int j0 = cv * 8;
       float y[8];
-      if (c0 + i < C && r0 + j0 < R) {
-        const int valid = clamp8(R - (r0 + j0));
+      const int valid = (c0 + i < C && r0 + j0 < R) ? clamp8(R - (r0 + j0)) : 0;
+      if (valid > 0 && DMUON_IN(tab.status, r0 + j0, valid, tab.ldn) &&
+          DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + (c0 + i) * tab.ldn + r0 + j0, valid,
+                   (int64_t)tab.count * tab.m * tab.ldn)) {
         load8<T>(Om + (c0 + i) * tab.ldn + r0 + j0, y, o_vec && valid == 8, valid);
       } else {
 #pragma unroll
@@ -192,12 +200,17 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t gc = c0 + cv * 8;
     if (gr >= R || gc >= C) continue;
     const int valid = clamp8(C - gc);
+    if (!DMUON_IN(tab.status, gr * C + gc, valid, R * C)) continue;
     float o[8];
     if (tr) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) o[i] = s[r][cv * 8 + i];
-    } else {
+    } else if (DMUON_IN(tab.status, gc, valid, tab.ldn) &&
+               DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + gr * tab.ldn + gc, valid,
+                        (int64_t)tab.count * tab.m * tab.ldn)) {
       load8<T>(Om + gr * tab.ldn + gc, o, o_vec && valid == 8, valid);
+    } else {
+      continue;
     }
     if (scale) {
 #pragma unroll

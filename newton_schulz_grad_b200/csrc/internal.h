@@ -38,6 +38,7 @@ struct ElemTable {
   int64_t m, n, ldn;
   int32_t count;
   int32_t tiles_per_mat;  // ceil(m/64) * ceil(n/64)
+  int* status = nullptr;  // device status word (debug builds record bounds errors)
   MatEntry e[kMaxTable];
 };
 
@@ -73,13 +74,14 @@ cudaError_t launch_update(const ElemTable& t, int dtype, ElemMode mode, const vo
 // FFMA chain kernels, batched over `batch` matrices with element batch strides.
 // xbf16: X is bf16 (else fp32); G and P are bf16 only when gbf16 (stage calls
 // of the bf16 dtype never come here; gbf16 is always false in practice).
+// status: device status word (debug builds record bounds errors there).
 cudaError_t simt_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,
-                      float alpha, const float* scale, bool xbf16, cudaStream_t st);
+                      float alpha, const float* scale, bool xbf16, cudaStream_t st, int* status);
 cudaError_t simt_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp,
-                      float b, float c, cudaStream_t st);
+                      float b, float c, cudaStream_t st, int* status);
 cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, int n,
                        int64_t ldp, int64_t ldx, int64_t ldy, float a, float alpha,
-                       const float* scale, bool xbf16, cudaStream_t st);
+                       const float* scale, bool xbf16, cudaStream_t st, int* status);
 
 // ---- clip.cu --------------------------------------------------------------------
 // Each matrix is read as a flat array of rows * cols elements; one partial per
@@ -102,7 +104,7 @@ cudaError_t launch_clip_scale(const ElemTable& t, int dtype, const float* coef, 
 // Valid for steps <= 16 and n <= small_ns_max_n(m, element size).
 int small_ns_max_n(int m, size_t es);
 cudaError_t small_ns(void* X, int batch, int m, int n, int64_t ld, int steps, const float* coeffs,
-                     const float* scale, bool xbf16, cudaStream_t st);
+                     const float* scale, bool xbf16, cudaStream_t st, int* status);
 
 // ---- tc_gemm.cu -------------------------------------------------------------
 // tcgen05 chain kernels (bf16 in/out, fp32 accumulation in TMEM).

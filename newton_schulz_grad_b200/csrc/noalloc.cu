@@ -114,6 +114,7 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
 
   // ------------------------------------------------- the dmuon_ns_ex kernels
   ElemTable tab;  // on the stack: no host or device allocation
+  tab.status = status_word;
   tab.m = m;
   tab.n = n;
   tab.ldn = L.ldn;
@@ -141,9 +142,9 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
                      st);
     } else {
       const bool xbf16 = L.path == Path::kSmallBf16;
-      e = simt_gram(cur, G, 1, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, xbf16, st);
-      if (e == cudaSuccess) e = simt_poly(G, P, 1, (int)m, L.ldm, L.ldm, b, c, st);
-      if (e == cudaSuccess) e = simt_apply(P, cur, nxt, 1, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st);
+      e = simt_gram(cur, G, 1, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, xbf16, st, status_word);
+      if (e == cudaSuccess) e = simt_poly(G, P, 1, (int)m, L.ldm, L.ldm, b, c, st, status_word);
+      if (e == cudaSuccess) e = simt_apply(P, cur, nxt, 1, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st, status_word);
     }
     std::swap(cur, nxt);
   }

@@ -39,6 +39,8 @@ struct SimtArgs {
   float p0, p1;     // gram: alpha; poly: b, c; apply: a, alpha
   const float* scale;
   int tiles_n, tiles_per_mat;
+  int batch;
+  int* status;      // device status word (bounds errors of debug builds)
 };
 
 template <typename T>
@@ -86,7 +88,11 @@ __global__ void __launch_bounds__(kThreads) k_simt(const SimtArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int gr = i0 + row, gk = k0 + kq + e;
-        As[kq + e][row] = (gr < a.m && gk < a.k) ? ld(A, (int64_t)gr * a.lda + gk) : 0.f;
+        As[kq + e][row] = (gr < a.m && gk < a.k &&
+                           DMUON_IN(a.status, (int64_t)b * a.sA + (int64_t)gr * a.lda + gk, 1, a.batch * a.sA) &&
+                           DMUON_IN(a.status, gk, 1, a.lda))
+                              ? ld(A, (int64_t)gr * a.lda + gk)
+                              : 0.f;
       }
     }
     if (MODE == kApply) {  // B is k x n row-major: Bs[k][j]
@@ -94,14 +100,22 @@ __global__ void __launch_bounds__(kThreads) k_simt(const SimtArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int gk = k0 + kk, gj = j0 + jq + e;
-        Bs[kk][jq + e] = (gk < a.k && gj < a.n) ? ld(B, (int64_t)gk * a.ldb + gj) : 0.f;
+        Bs[kk][jq + e] = (gk < a.k && gj < a.n &&
+                          DMUON_IN(a.status, (int64_t)b * a.sB + (int64_t)gk * a.ldb + gj, 1, a.batch * a.sB) &&
+                          DMUON_IN(a.status, gj, 1, a.ldb))
+                             ? ld(B, (int64_t)gk * a.ldb + gj)
+                             : 0.f;
       }
     } else {  // B rows j0.. (k-major, like A)
       const int row = tid / 4, kq = (tid % 4) * 4;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int gr = j0 + row, gk = k0 + kq + e;
-        Bs[kq + e][row] = (gr < a.n && gk < a.k) ? ld(B, (int64_t)gr * a.ldb + gk) : 0.f;
+        Bs[kq + e][row] = (gr < a.n && gk < a.k &&
+                           DMUON_IN(a.status, (int64_t)b * a.sB + (int64_t)gr * a.ldb + gk, 1, a.batch * a.sB) &&
+                           DMUON_IN(a.status, gk, 1, a.ldb))
+                              ? ld(B, (int64_t)gr * a.ldb + gk)
+                              : 0.f;
       }
     }
     __syncthreads();
@@ -149,6 +163,9 @@ __global__ void __launch_bounds__(kThreads) k_simt(const SimtArgs a) {
     for (int j = 0; j < 4; ++j) {
       const int c = j0 + tx * 4 + j;
       if (c >= a.n) continue;
+      if (MODE != kGram && (!DMUON_IN(a.status, (int64_t)b * a.sE + (int64_t)r * a.lde + c, 1, a.batch * a.sE) ||
+                            !DMUON_IN(a.status, c, 1, a.lde)))
+        continue;
       float v;
       if (MODE == kGram) {
         v = alpha * acc[i][j];
@@ -157,11 +174,15 @@ __global__ void __launch_bounds__(kThreads) k_simt(const SimtArgs a) {
       } else {
         v = alpha * fmaf(a.p0, ld(Em, (int64_t)r * a.lde + c), acc[i][j]);
       }
+      const bool here = DMUON_IN(a.status, (int64_t)b * a.sC + (int64_t)r * a.ldc + c, 1, a.batch * a.sC) &&
+                        DMUON_IN(a.status, c, 1, a.ldc);
       if (MODE == kApply) {
-        Cm[(int64_t)r * a.ldc + c] = Elt<TC>::from_f(v);
+        if (here) Cm[(int64_t)r * a.ldc + c] = Elt<TC>::from_f(v);
       } else {
-        if (r >= c) Cm[(int64_t)r * a.ldc + c] = Elt<TC>::from_f(v);
-        if (r > c) Cm[(int64_t)c * a.ldc + r] = Elt<TC>::from_f(v);
+        if (r >= c && here) Cm[(int64_t)r * a.ldc + c] = Elt<TC>::from_f(v);
+        if (r > c && DMUON_IN(a.status, (int64_t)b * a.sC + (int64_t)c * a.ldc + r, 1, a.batch * a.sC) &&
+            DMUON_IN(a.status, r, 1, a.ldc))
+          Cm[(int64_t)c * a.ldc + r] = Elt<TC>::from_f(v);
       }
     }
   }
@@ -175,9 +196,10 @@ int tri_tiles(int m) {
 }  // namespace
 
 cudaError_t simt_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,
-                      float alpha, const float* scale, bool xbf16, cudaStream_t st) {
+                      float alpha, const float* scale, bool xbf16, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
   SimtArgs a{};
+  a.batch = batch; a.status = status;
   a.A = X; a.B = X; a.E = nullptr; a.C = G;
   a.sA = a.sB = (int64_t)m * ldx; a.sC = (int64_t)m * ldg;
   a.lda = a.ldb = ldx; a.ldc = ldg;
@@ -193,9 +215,10 @@ cudaError_t simt_gram(const void* X, void* G, int batch, int m, int n, int64_t l
 }
 
 cudaError_t simt_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b,
-                      float c, cudaStream_t st) {
+                      float c, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
   SimtArgs a{};
+  a.batch = batch; a.status = status;
   a.A = G; a.B = G; a.E = G; a.C = P;
   a.sA = a.sB = a.sE = (int64_t)m * ldg; a.sC = (int64_t)m * ldp;
   a.lda = a.ldb = a.lde = ldg; a.ldc = ldp;
@@ -209,9 +232,10 @@ cudaError_t simt_poly(const void* G, void* P, int batch, int m, int64_t ldg, int
 
 cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
                        int64_t ldx, int64_t ldy, float a_coef, float alpha, const float* scale,
-                       bool xbf16, cudaStream_t st) {
+                       bool xbf16, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
   SimtArgs a{};
+  a.batch = batch; a.status = status;
   a.A = P; a.B = X; a.E = X; a.C = Y;
   a.sA = (int64_t)m * ldp; a.sB = a.sE = (int64_t)m * ldx; a.sC = (int64_t)m * ldy;
   a.lda = ldp; a.ldb = a.lde = ldx; a.ldc = ldy;

@@ -38,6 +38,8 @@ struct SmallArgs {
   int steps;
   const float* scale;  // per matrix 1/(||x0|| + eps)
   float coeffs[3 * 16];  // a, b, c per iteration (at most 16 here)
+  int batch;
+  int* status;         // device status word (bounds errors of debug builds)
 };
 
 // Two consecutive elements of a shared row as fp32 (c even).
@@ -74,7 +76,11 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   // rows >= m and columns >= cw are zero, so they add nothing below
   for (int i = tid; i < m4 * w; i += kThreads) {
     const int r = i / w, c = i % w;
-    Xs[r * lw + c] = (r < m && c < cw) ? Xg[(int64_t)r * a.ld + c0 + c] : Elt<T>::from_f(0.f);
+    Xs[r * lw + c] = (r < m && c < cw &&
+                      DMUON_IN(a.status, (int64_t)mat * a.sX + (int64_t)r * a.ld + c0 + c, 1, a.batch * a.sX) &&
+                      DMUON_IN(a.status, c0 + c, 1, a.ld))
+                         ? Xg[(int64_t)r * a.ld + c0 + c]
+                         : Elt<T>::from_f(0.f);
   }
   for (int i = tid; i < kMaxM * kMaxM; i += kThreads) Pt[i] = 0.f;
   const float s = a.scale[mat];
@@ -165,7 +171,9 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   }
   for (int i = tid; i < m * w; i += kThreads) {
     const int r = i / w, c = i % w;
-    if (c < cw) Xg[(int64_t)r * a.ld + c0 + c] = Xs[r * lw + c];
+    if (c < cw && DMUON_IN(a.status, (int64_t)mat * a.sX + (int64_t)r * a.ld + c0 + c, 1, a.batch * a.sX) &&
+        DMUON_IN(a.status, c0 + c, 1, a.ld))
+      Xg[(int64_t)r * a.ld + c0 + c] = Xs[r * lw + c];
   }
 }
 
@@ -186,10 +194,12 @@ int small_ns_max_n(int m, size_t es) {
 }
 
 cudaError_t small_ns(void* X, int batch, int m, int n, int64_t ld, int steps, const float* coeffs,
-                     const float* scale, bool xbf16, cudaStream_t st) {
+                     const float* scale, bool xbf16, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
   if (m > kMaxM || steps > 16) return cudaErrorInvalidValue;
   SmallArgs a{};
+  a.batch = batch;
+  a.status = status;
   a.X = X;
   a.ld = ld;
   a.sX = (int64_t)m * ld;

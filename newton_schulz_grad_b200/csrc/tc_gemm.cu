@@ -48,6 +48,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace dmuon {
@@ -97,6 +98,9 @@ struct TcArgs {
   const float* scale;
   int* status;
 };
+
+// Matrices in the launch (extent checks of debug builds).
+[[maybe_unused]] __device__ __forceinline__ int64_t batch_of(const TcArgs& a) { return a.total_tiles / a.tiles_per_mat; }
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -351,17 +355,24 @@ __device__ __forceinline__ void load_upd_chunk(const UpdTable& u, const TcArgs& 
   const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(u.p[b]);
   const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
   const bool full = c0 + 32 <= n;
+  [[maybe_unused]] const int len = full ? 32 : n - c0;
+  [[maybe_unused]] const int64_t pext = (int64_t)m * n;
   if (tr) {
     const __nv_bfloat16* q = p + (int64_t)c0 * m + r;
     const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
-      const __nv_bfloat16 lo = (c0 + j < n) ? *q : z;
+      const __nv_bfloat16 lo =
+          (c0 + j < n && DMUON_IN(a.status, (int64_t)(c0 + j) * m + r, 1, pext)) ? *q : z;
       q += m;
-      const __nv_bfloat16 hi = (c0 + j + 1 < n) ? *q : z;
+      const __nv_bfloat16 hi =
+          (c0 + j + 1 < n && DMUON_IN(a.status, (int64_t)(c0 + j + 1) * m + r, 1, pext)) ? *q : z;
       q += m;
       k.p[j >> 1] = pack2(lo, hi);
     }
+  } else if (!DMUON_IN(a.status, (int64_t)r * n + c0, len, pext) || !DMUON_IN(a.status, c0, len, n)) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) k.p[j] = 0u;
   } else if (full && ((u.vmask[b >> 5] >> (b & 31)) & 1u)) {
     const uint4* q = reinterpret_cast<const uint4*>(p + (int64_t)r * n + c0);
 #pragma unroll
@@ -375,7 +386,11 @@ __device__ __forceinline__ void load_upd_chunk(const UpdTable& u, const TcArgs& 
   }
   if (a.p0 != 0.f) {
     const __nv_bfloat16* ep = a.E + (int64_t)b * a.sE + (int64_t)r * a.lde + c0;
-    if (full) {
+    if (!DMUON_IN(a.status, (int64_t)b * a.sE + (int64_t)r * a.lde + c0, len, batch_of(a) * a.sE) ||
+        !DMUON_IN(a.status, c0, len, a.lde)) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) k.e[j] = 0u;
+    } else if (full) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(k.e)[i] = __ldg(reinterpret_cast<const uint4*>(ep) + i);
     } else {
@@ -407,13 +422,16 @@ __device__ __forceinline__ void store_upd_chunk(const UpdTable& u, const TcArgs&
   }
   __nv_bfloat16* p = static_cast<__nv_bfloat16*>(u.p[b]);
   const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
+  [[maybe_unused]] const int64_t pext = (int64_t)m * n;
   if (tr) {
     __nv_bfloat16* q = p + (int64_t)c0 * m + r;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      if (c0 + j < n) *q = __float2bfloat16_rn(pv[j]);
+      if (c0 + j < n && DMUON_IN(a.status, (int64_t)(c0 + j) * m + r, 1, pext)) *q = __float2bfloat16_rn(pv[j]);
       q += m;
     }
+  } else if (!DMUON_IN(a.status, (int64_t)r * n + c0, c0 + 32 <= n ? 32 : n - c0, pext)) {
+    return;
   } else if (c0 + 32 <= n && ((u.vmask[b >> 5] >> (b & 31)) & 1u)) {
     uint4* q = reinterpret_cast<uint4*>(p + (int64_t)r * n + c0);
 #pragma unroll
@@ -513,10 +531,15 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename Upd
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]);
     const bool full_chunk = c0 + 32 <= a.n;
+    [[maybe_unused]] const int len = full_chunk ? 32 : a.n - c0;
     if ((MODE == kApply && a.p0 != 0.f) || (MODE == kPoly && Em != nullptr)) {
       float e[32];
       const __nv_bfloat16* ep = Em + (int64_t)r * a.lde + c0;
-      if (full_chunk) {
+      if (!DMUON_IN(a.status, (int64_t)b * a.sE + (int64_t)r * a.lde + c0, len, batch_of(a) * a.sE) ||
+          !DMUON_IN(a.status, c0, len, a.lde)) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) e[j] = 0.f;
+      } else if (full_chunk) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
       } else {
@@ -543,6 +566,9 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename Upd
         if (c0 + j == r) v[j] += a.p2;
     }
     __nv_bfloat16* rowp = Cm + (int64_t)r * a.ldc + c0;
+    if (!DMUON_IN(a.status, (int64_t)b * a.sC + (int64_t)r * a.ldc + c0, len, batch_of(a) * a.sC) ||
+        !DMUON_IN(a.status, c0, len, a.ldc))
+      continue;
     if (MODE == kApply) {
       if (full_chunk) {
 #pragma unroll
@@ -561,14 +587,19 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename Upd
 #pragma unroll
         for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(rowp)[q] = pack_bf16x8(v + 8 * q);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) Cm[(int64_t)(c0 + j) * a.ldc + r] = h[j];
+        for (int j = 0; j < 32; ++j)
+          if (DMUON_IN(a.status, (int64_t)b * a.sC + (int64_t)(c0 + j) * a.ldc + r, 1, batch_of(a) * a.sC) &&
+              DMUON_IN(a.status, r, 1, a.ldc))
+            Cm[(int64_t)(c0 + j) * a.ldc + r] = h[j];
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int c = c0 + j;
           if (c < a.n && r >= c) {
             rowp[j] = h[j];
-            if (r > c) Cm[(int64_t)c * a.ldc + r] = h[j];
+            if (r > c && DMUON_IN(a.status, (int64_t)b * a.sC + (int64_t)c * a.ldc + r, 1, batch_of(a) * a.sC) &&
+                DMUON_IN(a.status, r, 1, a.ldc))
+              Cm[(int64_t)c * a.ldc + r] = h[j];
           }
         }
       }

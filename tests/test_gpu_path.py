@@ -7,6 +7,7 @@ Tolerances (per matrix, relative Frobenius):
 * momentum buffers: bit for bit against the fp32 rounding-contract emulation.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -372,3 +373,82 @@ def test_step_fused_update_unaligned_parameter():
         err = np.linalg.norm(to64(p) - want[0])
         assert err <= 2e-2 * np.linalg.norm(want[0] - p_old) + 2 ** -8 * np.linalg.norm(want[0])
         assert np.array_equal(head, bits(base[:1]))  # the element before the view is untouched
+
+
+def test_step_injected_launch_failure_is_ordered_and_recoverable(monkeypatch):
+    # A launch failure part-way through an overlapped step: the status says so,
+    # the parameters are untouched (the chain never ran), all of the call's
+    # work is ordered before later work on the caller's stream, and the next
+    # step gives the same bits as a step that never saw the failure.
+    monkeypatch.setenv("DMUON_WS_CAP_MB", "20")
+    w = workloads.get("small_layer_bf16")
+    mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
+    ref_p = [m[0].clone() for m in mats]
+    ref_b = [m[2].clone() for m in mats]
+    nsg.dmuon_step(ref_p, [m[1] for m in mats], ref_b)
+    torch.cuda.synchronize()
+    ps = [m[0].clone() for m in mats]
+    bs = [m[2].clone() for m in mats]
+    p_bits = [bits(p) for p in ps]
+    monkeypatch.setenv("DMUON_FAULT_INJECT", "launch")
+    with pytest.raises(nsg.DmuonError) as ei:
+        nsg.dmuon_step(ps, [m[1] for m in mats], bs)
+    assert ei.value.status == nsg.DMUON_ERR_CUDA and "injected" in str(ei.value)
+    monkeypatch.delenv("DMUON_FAULT_INJECT")
+    torch.cuda.current_stream().synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    assert all(np.array_equal(a, bits(p)) for a, p in zip(p_bits, ps))
+    # restore the buffers (the first chunk's momentum ran) and step again
+    bs = [m[2].clone() for m in mats]
+    nsg.dmuon_step(ps, [m[1] for m in mats], bs)
+    torch.cuda.synchronize()
+    assert all(np.array_equal(bits(a), bits(b)) for a, b in zip(ref_p + ref_b, ps + bs))
+    nsg.dmuon_release_workspace()
+
+
+def test_step_resumes_bitwise_in_a_new_process(tmp_path):
+    # checkpoint / resume: the library keeps no state between steps beyond the
+    # caller's parameters and momentum buffers, so two steps in one process
+    # equal one step, torch.save, and a second step in a fresh process
+    import subprocess
+    import sys
+    w = workloads.get("small_layer_bf16")
+    ps, gs, bs = workloads.make_all(w, DEV)
+    g2 = [torch.flip(g, dims=[0]).contiguous() for g in gs]
+    nsg.dmuon_step(ps, gs, bs, wd=0.1)
+    torch.cuda.synchronize()
+    ck = tmp_path / "ck.pt"
+    torch.save({"p": [p.cpu() for p in ps], "b": [b.cpu() for b in bs], "g2": [g.cpu() for g in g2]}, ck)
+    nsg.dmuon_step(ps, g2, bs, wd=0.1)
+    torch.cuda.synchronize()
+    out = tmp_path / "out.pt"
+    code = (
+        "import torch, newton_schulz_grad_b200 as nsg\n"
+        f"d = torch.load({str(ck)!r})\n"
+        "ps = [t.cuda() for t in d['p']]; bs = [t.cuda() for t in d['b']]; gs = [t.cuda() for t in d['g2']]\n"
+        "nsg.dmuon_step(ps, gs, bs, wd=0.1)\n"
+        "torch.cuda.synchronize()\n"
+        f"torch.save({{'p': [p.cpu() for p in ps], 'b': [b.cpu() for b in bs]}}, {str(out)!r})\n"
+    )
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    subprocess.run([sys.executable, "-c", code], check=True, cwd=root, timeout=600)
+    r = torch.load(out)
+    assert all(np.array_equal(bits(a), bits(b)) for a, b in zip(ps + bs, r["p"] + r["b"]))
+
+
+def test_step_with_nvtx_ranges_gives_the_same_bits(monkeypatch):
+    w = workloads.get("small_layer_bf16")
+    mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
+
+    def run():
+        ps = [m[0].clone() for m in mats]
+        bs = [m[2].clone() for m in mats]
+        nsg.dmuon_step(ps, [m[1] for m in mats], bs, max_norm=1.0)
+        torch.cuda.synchronize()
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        return [bits(t) for t in ps + bs]
+
+    plain = run()
+    monkeypatch.setenv("DMUON_NVTX", "1")
+    with_ranges = run()
+    assert all(np.array_equal(a, b) for a, b in zip(plain, with_ranges))

@@ -464,15 +464,27 @@ def run_ours(args):
         pg.destroy_process_group()
 
 
-def e2e_groups(w, size: int = 16):
-    """Matrix indices in groups of one oriented shape, at most `size` each."""
+def e2e_groups(w, size: int = 16, edge: int = 2):
+    """Matrix indices in groups of one oriented shape, at most `size` each.
+
+    The first group's host-to-device copy and the last group's read-back
+    overlap no compute, so both are `edge` matrices of the class with the
+    smallest matrices (when it has enough members); the rest follow in groups
+    of `size`."""
     by_class = {}
     for i, (r, c) in enumerate(w.shapes):
         by_class.setdefault((min(r, c), max(r, c)), []).append(i)
-    groups = []
+    small = min(by_class, key=lambda k: k[0] * k[1])
+    head, tail = [], []
+    if len(by_class[small]) > 2 * edge:
+        head, tail = by_class[small][:edge], by_class[small][-edge:]
+        by_class[small] = by_class[small][edge:-edge]
+    groups = [head] if head else []
     for idx in by_class.values():
         for k in range(0, len(idx), size):
             groups.append(idx[k:k + size])
+    if tail:
+        groups.append(tail)
     return groups
 
 
@@ -484,7 +496,8 @@ def run_e2e(args, w, ps, gs, bs, shapes, stream, dev, world):
     group j's gradients travel on a copy stream while earlier groups compute,
     its dmuon_step call runs on the compute stream, and its parameters return
     on a second copy stream, so PCIe traffic in both directions overlaps the
-    tensor-core work.
+    tensor-core work (only the small first group's copy in and the small last
+    group's copy out overlap nothing).
     """
     import newton_schulz_grad_b200 as nsg
     try:

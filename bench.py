@@ -422,14 +422,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded low-rank + noise gradients, random-init parameters)",
-        "config": {"workload": w.name, "matrices": w.count,
-                   "shapes": sorted({f"{r}x{c}" for r, c in w.shapes}),
-                   "ns_steps": w.ns_steps, "nesterov": w.nesterov, "lr": w.lr, "wd": w.wd,
-                   **({"clip": {"max_norm": args.clip_norm, "norm_type": 2.0, "fused": "dmuon_step_clipped"}}
-                      if args.clip_norm is not None else {}),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"no flush: each step touches {w.elements() * 2 * 7 / 1e9:.1f} GB "
-                         f"(inputs alone {w.elements() * 2 * 3 / 1e9:.1f} GB) >> 126 MB L2"},
+        "config": workload_config(w, args, world),
         "ns_tflops": round(ns_tflops_step, 1),
         "ns_frac_of_peak": round(ns_tflops_step / float(peaks.get("bf16_tflops_sustained",
                                                                peaks["bf16_tflops"])), 4),
@@ -462,6 +455,18 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if pg:
         pg.destroy_process_group()
+
+
+def workload_config(w, args, world: int) -> dict:
+    """The `config` of the JSON line: the workload, the same for both arms."""
+    return {"workload": w.name, "matrices": w.count,
+            "shapes": sorted({f"{r}x{c}" for r, c in w.shapes}),
+            "ns_steps": w.ns_steps, "nesterov": w.nesterov, "lr": w.lr, "wd": w.wd,
+            **({"clip": {"max_norm": args.clip_norm, "norm_type": 2.0, "fused": "dmuon_step_clipped"}}
+               if getattr(args, "clip_norm", None) is not None else {}),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"no flush: each step touches {w.elements() * 2 * 7 / 1e9:.1f} GB "
+                  f"(inputs alone {w.elements() * 2 * 3 / 1e9:.1f} GB) >> 126 MB L2"}
 
 
 def e2e_groups(w, size: int = 16, edge: int = 2):
@@ -592,7 +597,7 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total * 1e3, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "matrices": w.count, "ns_steps": w.ns_steps},
+            "config": workload_config(w, args, world),
             "cpu_baseline": {"value": round(value, 5), "unit": "matrices/s", "cores": blas_threads(),
                              "kind": "oracle",
                              "sample": "each step one matrix, rotating over the launch classes; "

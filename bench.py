@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama_7b_bf16")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-group", type=int, default=16,
+                    help="matrices per dmuon_step call in the end-to-end pipeline")
     ap.add_argument("--cpu-budget-s", type=float, default=30.0,
                     help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -514,7 +516,7 @@ def run_e2e(args, w, ps, gs, bs, shapes, stream, dev, world):
         gh.copy_(g)
     h2d = sum(g.numel() * g.element_size() for g in gs)
     d2h = sum(p.numel() * p.element_size() for p in ps)
-    groups = e2e_groups(w)
+    groups = e2e_groups(w, size=args.e2e_group)
     s_in = torch.cuda.Stream(dev)
     s_out = torch.cuda.Stream(dev)
     done_compute = [None] * len(groups)  # last step's compute of group j (frees its gradients)

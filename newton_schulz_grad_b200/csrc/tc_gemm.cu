@@ -1168,8 +1168,9 @@ cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st) {
 
 const char* tc_config_string() {
   return "tcgen05 bf16->fp32: CTA-pair kernel (cta_group::2, M256xN256xK16, 6 x 32 KB stages per CTA) for "
-         "m >= 256, one-CTA kernel (cta_group::1, M128xN256xK16, 4 x 48 KB stages) otherwise; BK=64 SW128, 2 TMEM "
-         "accumulators, persistent 192-thread CTAs (TMA warp, MMA warp, 4 epilogue warps)";
+         "m >= 256 unless 128-row tiles compute over 6 % less area, one-CTA kernel (cta_group::1, "
+         "M128xN256xK16, 4 x 48 KB stages) otherwise; BK=64 SW128, 2 TMEM accumulators, persistent "
+         "192-thread CTAs (TMA warp, MMA warp, 4 epilogue warps); last apply of a chain fused with the update";
 }
 
 }  // namespace dmuon

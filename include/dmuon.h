@@ -138,8 +138,10 @@ DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int
  * Matrices are grouped by shape (dmuon_plan_groups) and each group runs as
  * batched launches.  The library's workspace (cached per device and stream,
  * at most DMUON_WS_CAP_MB, default 8 GiB) is allocated stream-ordered on
- * first use or growth; after one call with the same shapes, a call allocates
- * nothing and can be captured in a CUDA graph.  With several chunks the
+ * first use or growth; after one call with the same shapes on the same
+ * stream, a call allocates nothing and can be captured in a CUDA graph (a
+ * call that would grow the workspace while its stream is capturing returns
+ * DMUON_ERR_INVALID_ARG instead).  With several chunks the
  * momentum and update stages run on an internal stream underneath the
  * Newton-Schulz chain and are joined back into `stream` before the call's
  * work ends; the results do not depend on that schedule.

@@ -126,6 +126,17 @@ dmuon_status_t get_workspace(size_t bytes, cudaStream_t st, void** out) {
     *out = slot.first;
     return DMUON_OK;
   }
+  // growing inside a stream capture would make the cached workspace memory
+  // owned by the graph: the first call with these shapes must run uncaptured
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) {
+    cudaGetLastError();
+    cap = cudaStreamCaptureStatusNone;
+  }
+  if (cap != cudaStreamCaptureStatusNone)
+    return fail(DMUON_ERR_INVALID_ARG, "the stream is capturing and its workspace needs " + std::to_string(bytes) +
+                                           " bytes it does not have yet: make one call with these shapes on this "
+                                           "stream before capturing");
   if (slot.first) {
     cudaFreeAsync(slot.first, st);
     slot = {nullptr, 0};

@@ -270,24 +270,29 @@ def test_bounded_device_wait_reports_timeout_and_context_survives():
     assert rel_fro(to64(out), om.newton_schulz(to64(X), 5)) < 2e-2
 
 
+@pytest.mark.parametrize("clip", [None, 0.5], ids=["plain", "clipped"])
 @pytest.mark.parametrize("name", ["small_layer_bf16", "single_256x512_f32"])
-def test_step_replays_from_a_cuda_graph(name):
-    # after one eager call (workspace and internal stream exist) a step can be
-    # captured into a CUDA graph; replays give the eager step's bits
+def test_step_replays_from_a_cuda_graph(name, clip):
+    # after one eager call on the capture stream (workspace and internal stream
+    # exist) a step can be captured into a CUDA graph; replays give the eager
+    # step's bits
     w = workloads.get(name)
     mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
     eager = [[t.clone() for t in m] for m in mats]
     graphed = [[t.clone() for t in m] for m in mats]
+    scratch = [[t.clone() for t in m] for m in mats]
 
     def step(sets, stream=None):
         nsg.dmuon_step([m[0] for m in sets], [m[1] for m in sets], [m[2] for m in sets],
-                       lr=w.lr, wd=0.05, stream=stream)
+                       lr=w.lr, wd=0.05, stream=stream, max_norm=clip)
 
-    step(eager)                    # warm-up: allocations happen here
     step(eager)
-    torch.cuda.synchronize()
+    step(eager)
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
+    step(scratch, stream=side)     # warm-up on the capture stream: allocations happen here
+    side.synchronize()
+    torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=side):
         step(graphed, stream=side)
@@ -452,3 +457,56 @@ def test_step_with_nvtx_ranges_gives_the_same_bits(monkeypatch):
     monkeypatch.setenv("DMUON_NVTX", "1")
     with_ranges = run()
     assert all(np.array_equal(a, b) for a, b in zip(plain, with_ranges))
+
+
+@pytest.mark.filterwarnings("ignore:The CUDA Graph is empty")
+def test_step_refuses_to_grow_its_workspace_while_capturing():
+    w = workloads.get("single_256x512_f32")
+    ps, gs, bs = workloads.make_all(w, DEV)
+    side = torch.cuda.Stream()          # never used: no workspace yet
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with pytest.raises(nsg.DmuonError) as ei:
+        with torch.cuda.graph(g, stream=side):
+            nsg.dmuon_step(ps, gs, bs, stream=side)
+    assert ei.value.status == nsg.DMUON_ERR_INVALID_ARG and "capturing" in str(ei.value)
+    torch.cuda.synchronize()
+    nsg.dmuon_step(ps, gs, bs, stream=side)   # uncaptured, it allocates and runs
+    side.synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+
+
+def test_concurrent_host_threads_on_their_own_streams():
+    # two host threads step disjoint sets on their own streams at the same time
+    # (the binding releases the GIL inside the library): each gets the bits of
+    # a step run alone
+    import threading
+    w = workloads.get("small_layer_bf16")
+    sets = [[[t.clone() for t in workloads.make_matrix(w, i, DEV)] for i in range(w.count)] for _ in range(2)]
+    alone = [[[t.clone() for t in m] for m in s] for s in sets]
+    for s in alone:
+        nsg.dmuon_step([m[0] for m in s], [m[1] for m in s], [m[2] for m in s], wd=0.1)
+    torch.cuda.synchronize()
+    errors = []
+
+    def worker(s):
+        try:
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.current_stream())
+            for _ in range(1):
+                nsg.dmuon_step([m[0] for m in s], [m[1] for m in s], [m[2] for m in s], wd=0.1, stream=st)
+            st.synchronize()
+        except Exception as exc:  # reported below
+            errors.append(exc)
+
+    threads = [threading.Thread(target=worker, args=(s,)) for s in sets]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    for s, a in zip(sets, alone):
+        for m, n in zip(s, a):
+            for x, y in zip(m, n):
+                assert np.array_equal(bits(x), bits(y))

@@ -61,10 +61,13 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--ns-steps", type=int, default=None,
                     help="override the workload's Newton-Schulz iteration count")
-    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update", "step", "clip"],
+    ap.add_argument("--stage", choices=["gram", "poly", "apply", "momentum", "update", "step", "clip",
+                                        "lib_chain", "lib_apply"],
                     help="time one kernel through its stage call instead of the whole step")
     ap.add_argument("--clip-norm", type=float, default=None,
                     help="time dmuon_step_clipped: global 2-norm clipping of the gradients to this bound")
+    ap.add_argument("--lib", choices=["torch", "quack"], default="torch",
+                    help="--stage lib_chain / lib_apply: the library whose GEMMs run the comparison")
     ap.add_argument("--batch", type=int, default=8)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--n", type=int, default=4096)
@@ -609,6 +612,71 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_lib_chain(args):
+    """Comparison only: the workload's Newton-Schulz chain (5 iterations of
+    G = X X^T, P = b G + c G G, X <- a X + P X on the oriented, normalised
+    matrices, batches of 16 per shape) through a library's bf16 GEMMs, timed
+    with CUDA events.  `torch`: torch.bmm / baddbmm (cuBLAS); `quack`: quack's
+    symmetric and add GEMMs (the kernels the DMuon pages name for SM90 and
+    later).  Nothing here is on the library's path and nothing is checked for
+    parity; the line sets the chain's time beside this library's chain
+    (the `ns_chain_tflops` of the default run counts the same flops)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workloads.get(args.workload)
+    steps = w.ns_steps if args.ns_steps is None else args.ns_steps
+    a, b, c = 3.4445, -4.7750, 2.0315
+    gen = torch.Generator(device=dev).manual_seed(11)
+    by_class = {}
+    for r, cc in w.shapes:
+        key = (min(r, cc), max(r, cc))
+        by_class[key] = by_class.get(key, 0) + 1
+    batches = []
+    for (m, n), cnt in by_class.items():
+        for k in range(0, cnt, 16):
+            X = torch.randn(min(16, cnt - k), m, n, generator=gen, device=dev)
+            X = (X / X.flatten(1).norm(dim=1).view(-1, 1, 1)).to(torch.bfloat16)
+            batches.append(X)
+    if args.lib == "quack":
+        from quack.gemm_interface import gemm_add, gemm_symmetric
+
+        def chain(X):
+            for _ in range(steps):
+                G = gemm_symmetric(X, X.mT)
+                P = gemm_symmetric(G, G, C=G, alpha=c, beta=b)
+                X = gemm_add(P, X, C=X, alpha=1.0, beta=a, tuned=False)
+            return X
+    else:
+        def chain(X):
+            for _ in range(steps):
+                G = torch.bmm(X, X.mT)
+                P = torch.baddbmm(G, G, G, beta=b, alpha=c)
+                X = torch.baddbmm(X, P, X, beta=a, alpha=1.0)
+            return X
+    for X in batches:                 # warm-up (and compilation, for quack)
+        chain(X)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.steps)
+    clocks = ClockSampler(0)
+    clocks.start()
+    e0.record()
+    for _ in range(reps):
+        for X in batches:
+            chain(X)
+    e1.record()
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / reps
+    flops = w.ns_flops() * steps / max(1, w.ns_steps)
+    print(json.dumps({"stage": "lib_chain", "lib": args.lib, "workload": w.name, "ns_steps": steps,
+                      "chain_ms": round(ms, 3), "matrices_per_s": round(w.count / (ms / 1e3), 2),
+                      "ns_tflops": round(flops / (ms / 1e3) / 1e12, 1), "reps": reps, "clocks": clk,
+                      "note": "Newton-Schulz chain only (no momentum, normalisation or update); "
+                              "flops counted as 3 m^2 n + m^3 per matrix and iteration"}), flush=True)
+
+
 def run_stage(args):
     """One kernel through its stage call (bf16), e.g. for an ncu capture of a small case."""
     import newton_schulz_grad_b200 as nsg
@@ -628,11 +696,17 @@ def run_stage(args):
         out = torch.empty_like(G)
         run = lambda: nsg.dmuon_gram_poly(G, out, -4.775, 2.0315)  # noqa: E731
         flops, nbytes = b * m ** 3, 2 * b * 2 * m * m
-    elif args.stage == "apply":
+    elif args.stage in ("apply", "lib_apply"):
         P = (torch.randn(b, m, m, generator=gen, device=dev) / math.sqrt(m)).to(bf)
         X = torch.randn(b, m, n, generator=gen, device=dev).to(bf)
         out = torch.empty_like(X)
-        run = lambda: nsg.dmuon_poly_apply(P, X, out, 3.4445)  # noqa: E731
+        if args.stage == "apply":
+            run = lambda: nsg.dmuon_poly_apply(P, X, out, 3.4445)  # noqa: E731
+        elif args.lib == "quack":  # comparison only: the same product through quack
+            from quack.gemm_interface import gemm_add
+            run = lambda: gemm_add(P, X, C=X, out=out, alpha=1.0, beta=3.4445, tuned=False)  # noqa: E731
+        else:  # comparison only: the same product through torch (cuBLAS)
+            run = lambda: torch.baddbmm(X, P, X, beta=3.4445, alpha=1.0, out=out)  # noqa: E731
         flops, nbytes = 2 * b * m * m * n, 2 * b * (m * m + 2 * m * n)
     elif args.stage == "step":
         # a whole step over `batch` m x n matrices (rows x cols as given): the
@@ -685,6 +759,9 @@ def run_stage(args):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.stage == "lib_chain":
+        run_lib_chain(args)
+        return
     if args.stage:
         run_stage(args)
     elif args.impl == "reference":

@@ -165,7 +165,10 @@ __device__ __noinline__ bool wait_bar_limit(uint32_t bar, uint32_t parity, int* 
     }
   }
 }
+// The common case (the phase already completed) stays inline: one poll, no
+// call; only a wait that has to spin goes to the bounded loop.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
   return wait_bar_limit(bar, parity, status, kTimeoutNs);
 }
 
@@ -702,6 +705,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ----------------------------------------------------------------- MMA
       constexpr uint32_t idesc = make_idesc(MODE == kApply, BM1);
+      // stage 0, k-step 0; every other descriptor adds an offset to these
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t b_desc0 = (MODE == kApply) ? sdesc_sw128(smem_u32(smem) + A1_BYTES, 8192, 1024)
+                                                : sdesc_sw128(smem_u32(smem) + A1_BYTES, 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -717,13 +724,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE1_BYTES);
-          const uint32_t sb = sa + A1_BYTES;
+          // descriptors of this stage: the bases plus the stage offset (16-byte units)
+          const uint64_t soff = (uint64_t)((stage * STAGE1_BYTES) >> 4);
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k) {
-            const uint64_t ad = sdesc_sw128(sa + k * (UK * 2), 16, 1024);
-            const uint64_t bd = (MODE == kApply) ? sdesc_sw128(sb + k * (UK * 128), 8192, 1024)
-                                                 : sdesc_sw128(sb + k * (UK * 2), 16, 1024);
+            const uint64_t ad = a_desc0 + soff + (uint64_t)(k * (UK * 2 / 16));
+            const uint64_t bd = b_desc0 + soff + (uint64_t)(k * ((MODE == kApply ? UK * 128 : UK * 2) / 16));
             tc_mma<1>(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit<1>(B.empty0 + 8 * stage);
@@ -871,6 +877,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       // ------------------------------------------------------ MMA (leader)
       constexpr uint32_t idesc = make_idesc(MODE == kApply, BM2);
+      // stage 0, k-step 0; every other descriptor adds an offset to these
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t b_desc0 = (MODE == kApply) ? sdesc_sw128(smem_u32(smem) + A2_BYTES, 8192, 1024)
+                                                : sdesc_sw128(smem_u32(smem) + A2_BYTES, 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -886,13 +896,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
-          const uint32_t sb = sa + A2_BYTES;
+          // descriptors of this stage: the bases plus the stage offset (16-byte units)
+          const uint64_t soff = (uint64_t)((stage * STAGE2_BYTES) >> 4);
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k) {
-            const uint64_t ad = sdesc_sw128(sa + k * (UK * 2), 16, 1024);
-            const uint64_t bd = (MODE == kApply) ? sdesc_sw128(sb + k * (UK * 128), 8192, 1024)
-                                                 : sdesc_sw128(sb + k * (UK * 2), 16, 1024);
+            const uint64_t ad = a_desc0 + soff + (uint64_t)(k * (UK * 2 / 16));
+            const uint64_t bd = b_desc0 + soff + (uint64_t)(k * ((MODE == kApply ? UK * 128 : UK * 2) / 16));
             tc_mma<2>(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit_pair(B.empty0 + 8 * stage, 0x3);

@@ -6,7 +6,6 @@ Tolerances (per matrix, relative Frobenius):
   (the update is small next to p, and bf16 storage of p rounds at 2^-9);
 * momentum buffers: bit for bit against the fp32 rounding-contract emulation.
 """
-import math
 import os
 
 import numpy as np

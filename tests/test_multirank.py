@@ -7,8 +7,6 @@ max over ranks of the timed region.  These run here without a GPU.
 import os
 import socket
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

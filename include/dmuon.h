@@ -141,10 +141,13 @@ DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int
  * first use or growth; after one call with the same shapes on the same
  * stream, a call allocates nothing and can be captured in a CUDA graph (a
  * call that would grow the workspace while its stream is capturing returns
- * DMUON_ERR_INVALID_ARG instead).  With several chunks the
- * momentum and update stages run on an internal stream underneath the
- * Newton-Schulz chain and are joined back into `stream` before the call's
- * work ends; the results do not depend on that schedule.
+ * DMUON_ERR_INVALID_ARG instead).  On the bf16 tensor-core path the update
+ * runs inside the chain's last product (its epilogue writes the parameters;
+ * DMUON_FUSED_UPDATE=0 runs it as a separate pass, with the same bits).  With
+ * several chunks the momentum stage (and any separate update) runs on an
+ * internal stream underneath the Newton-Schulz chain and is joined back into
+ * `stream` before the call returns, on error paths too; the results do not
+ * depend on that schedule.
  */
 DMUON_API dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
                           const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,

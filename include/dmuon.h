@@ -137,7 +137,9 @@ DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int
  *   wd     decoupled weight decay: p <- p (1 - lr wd) - ...
  * Matrices are grouped by shape (dmuon_plan_groups) and each group runs as
  * batched launches.  The library's workspace (cached per device and stream,
- * at most DMUON_WS_CAP_MB, default 8 GiB) is allocated stream-ordered on
+ * at most DMUON_WS_CAP_MB, default 8 GiB, unless one matrix alone needs more:
+ * it then runs as a chunk of its own and the step runs without the
+ * double-buffered overlap) is allocated stream-ordered on
  * first use or growth; after one call with the same shapes on the same
  * stream, a call allocates nothing and can be captured in a CUDA graph (a
  * call that would grow the workspace while its stream is capturing returns

@@ -107,6 +107,7 @@ StepPlan make_step_plan(const dmuon_shape_t* shapes, int32_t count) {
   const char* ov = std::getenv("DMUON_OVERLAP");
   const bool allow = !(ov && ov[0] == '0');
   const int64_t cap = workspace_cap_bytes();
+  StepPlan serial;
   for (int pass = 0; pass < 2; ++pass) {
     // pass 0: one buffer with the whole cap; pass 1: two buffers of half the cap
     const int64_t cap_b = pass == 0 ? cap : cap / 2;
@@ -123,7 +124,11 @@ StepPlan make_step_plan(const dmuon_shape_t* shapes, int32_t count) {
     }
     P.overlap = pass == 1;
     if (pass == 0 && (!allow || P.chunks.size() < 2)) break;
+    if (pass == 0) serial = P;
   }
+  // a matrix whose workspace alone exceeds half the cap would make the two
+  // overlapped buffers exceed the cap: run serially in one buffer instead
+  if (P.overlap && 2 * P.buffer_bytes > cap) return serial;
   return P;
 }
 

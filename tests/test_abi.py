@@ -191,3 +191,37 @@ def test_step_clipped_validation_errors():
     assert call(-0.5, 2.0) == nsg.DMUON_ERR_INVALID_ARG
     assert call(1.0, 0.5) == nsg.DMUON_ERR_UNSUPPORTED
     assert call(1.0, 2.0, ((4, 8, 9),)) == nsg.DMUON_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_workspace_stays_under_the_cap(seed, monkeypatch):
+    # random shape sets: the planned workspace fits the cap unless one matrix
+    # alone needs more (that matrix then runs as a chunk of its own), and more
+    # iterations never mean fewer launches
+    rng = random.Random(100 + seed)
+    cap_mb = rng.choice([64, 256, 1024, 8192])
+    monkeypatch.setenv("DMUON_WS_CAP_MB", str(cap_mb))
+    shapes = [(rng.choice([32, 256, 1000, 1408, 2048, 4096]), rng.choice([64, 512, 2816, 4096, 11008]),
+               rng.randint(0, 1)) for _ in range(rng.randint(1, 40))]
+    ws = nsg.dmuon_workspace_bytes(shapes, 5)
+    single = max(nsg.dmuon_workspace_bytes([s], 5) for s in shapes)
+    assert 0 < ws <= max(cap_mb << 20, single)
+    assert nsg.dmuon_step_launches(shapes, 6) >= nsg.dmuon_step_launches(shapes, 5) >= nsg.dmuon_step_launches(shapes, 1)
+
+
+def test_overlap_only_when_both_buffers_fit_the_cap(monkeypatch):
+    # small layer: its largest matrix needs about 21 MB of workspace.  Under a
+    # 20 MB cap two overlapped buffers would exceed the cap, so the plan runs
+    # serially in one buffer; under 64 MB it overlaps with two buffers
+    w = workloads.get("small_layer_bf16")
+    shapes = [(r, c, 1) for r, c in w.shapes]
+
+    def plan(cap, overlap):
+        monkeypatch.setenv("DMUON_WS_CAP_MB", str(cap))
+        monkeypatch.setenv("DMUON_OVERLAP", overlap)
+        return nsg.dmuon_workspace_bytes(shapes, 5), nsg.dmuon_step_launches(shapes, 5)
+
+    assert plan(20, "1") == plan(20, "0")
+    ws_over, launches_over = plan(64, "1")
+    ws_serial, launches_serial = plan(64, "0")
+    assert ws_over <= 64 << 20 and launches_over > launches_serial

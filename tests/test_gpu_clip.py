@@ -122,7 +122,7 @@ def _clone(ts):
 @pytest.mark.parametrize("name", ["small_layer_bf16", "single_256x512_f32"])
 def test_step_clipped_equals_clip_then_step(name, norm_type, monkeypatch):
     # small workspace cap: several chunks, run overlapped on two streams
-    monkeypatch.setenv("DMUON_WS_CAP_MB", "20")
+    monkeypatch.setenv("DMUON_WS_CAP_MB", "64")
     w = workloads.get(name)
     ps, gs, bs = workloads.make_all(w, "cuda")
     g_bits = [bits(g) for g in gs]

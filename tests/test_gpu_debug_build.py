@@ -46,7 +46,7 @@ for r, c in [(1, 37), (37, 1), (100, 37), (257, 129), (130, 136), (300, 520), (5
         done(f"ns {r}x{c} {dt}")
         res[f"ns {r}x{c} {dt}"] = out.cpu()
 
-os.environ["DMUON_WS_CAP_MB"] = "20"   # several chunks, overlapped
+os.environ["DMUON_WS_CAP_MB"] = "64"   # several chunks, overlapped
 w = workloads.get("small_layer_bf16")
 ps, gs, bs = workloads.make_all(w, dev)
 nsg.dmuon_step(ps, gs, bs, wd=0.1)

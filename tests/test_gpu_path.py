@@ -212,9 +212,9 @@ def test_step_overlapped_equals_serial(monkeypatch):
         assert nsg.dmuon_stream_status() == nsg.DMUON_OK
         return [bits(t) for t in ps + bs]
 
-    serial = run({"DMUON_OVERLAP": "0", "DMUON_WS_CAP_MB": "20"})
+    serial = run({"DMUON_OVERLAP": "0", "DMUON_WS_CAP_MB": "64"})
     nsg.dmuon_release_workspace()
-    over = run({"DMUON_OVERLAP": "1", "DMUON_WS_CAP_MB": "20"})
+    over = run({"DMUON_OVERLAP": "1", "DMUON_WS_CAP_MB": "64"})
     nsg.dmuon_release_workspace()
     monkeypatch.delenv("DMUON_WS_CAP_MB")
     monkeypatch.delenv("DMUON_OVERLAP")
@@ -327,7 +327,7 @@ def test_thin_matrix_chain_matches_oracle_fused_and_unfused(shape, dtype, monkey
 
 @pytest.mark.parametrize("name,idx,env", [
     ("small_layer_bf16", None, {}),
-    ("small_layer_bf16", None, {"DMUON_WS_CAP_MB": "20"}),        # several chunks, overlapped
+    ("small_layer_bf16", None, {"DMUON_WS_CAP_MB": "64"}),        # several chunks, overlapped
     ("small_layer_bf16", None, {"DMUON_GRAM_BLOCKS": "2"}),        # blocks of 2 and 3
     ("small_layer_bf16", None, {"DMUON_GRAM_BLOCKS": "0"}),        # per-iteration form
     ("llama3_2_3b_bf16", [0, 1, 4, 6], {}),
@@ -384,7 +384,7 @@ def test_step_injected_launch_failure_is_ordered_and_recoverable(monkeypatch):
     # the parameters are untouched (the chain never ran), all of the call's
     # work is ordered before later work on the caller's stream, and the next
     # step gives the same bits as a step that never saw the failure.
-    monkeypatch.setenv("DMUON_WS_CAP_MB", "20")
+    monkeypatch.setenv("DMUON_WS_CAP_MB", "64")
     w = workloads.get("small_layer_bf16")
     mats = [workloads.make_matrix(w, i, DEV) for i in range(w.count)]
     ref_p = [m[0].clone() for m in mats]

@@ -3,7 +3,8 @@
 // momentum + Newton-Schulz; the default strategy is global p-norm clipping).
 //
 //   total = (sum over all matrices and elements of |g|^p)^(1/p)   (p = inf: max |g|)
-//   coef  = min(1, max_norm / (total + 1e-6));   g <- fl(g * fl32(coef))
+//   coef  = min(1, max_norm / (total + 1e-6)), NaN if total is NaN;
+//   g <- fl(g * fl32(coef))
 //
 // Three launches, all on the caller's stream: per-chunk partials of sum |g|^p
 // (or max |g|) for every launch class of matrices; one block that reduces all
@@ -106,9 +107,10 @@ __global__ void __launch_bounds__(kThreads)
   }
   if (threadIdx.x == 0) {
     const double total = p == 0 ? red[0] : (p == 1 ? red[0] : sqrt(red[0]));
-    // a NaN total gives coef 1 (nothing scaled; the NaN total is reported)
+    // clamped to 1 by a comparison that keeps a NaN: a NaN total gives a NaN
+    // coefficient, so every gradient becomes NaN (PyTorch's clip_grad_norm_)
     const double c = (double)max_norm / (total + 1e-6);
-    *coef = (float)(c < 1.0 ? c : 1.0);
+    *coef = (float)((c < 1.0 || c != c) ? c : 1.0);
     if (total_out) *total_out = total;
   }
 }

@@ -156,17 +156,22 @@ def muon_step(params: Sequence[np.ndarray], grads: Sequence[np.ndarray],
 
 
 # Reading (the Training Guide's "Gradient Clipping" section names global p-norm
-# clipping of the Muon gradients and pairs it with PyTorch's clip_grad_norm_):
-# the same formula, 1e-6 added to the norm, coefficient clamped to 1.
+# clipping of the Muon gradients, gives DMuon's clip the name and max_norm
+# argument of PyTorch's clip_grad_norm_ and uses the two side by side):
+# PyTorch's formula, 1e-6 added to the norm, coefficient clamped to 1 by a
+# clamp that keeps a NaN.
 CLIP_EPS: float = 1e-6
 
 
 def clip_grad_norm(grads: Sequence[np.ndarray], max_norm: float, norm_type: float = 2.0):
     """Global p-norm clipping of a list of gradients.
 
-    total = (sum_i sum |g|^p)^(1/p) (p = inf: max |g|); coef = min(1, max_norm /
-    (total + 1e-6)); returns (clipped gradients, total, coef).  Training Guide,
-    "Gradient Clipping": after the reduce, before momentum + Newton-Schulz.
+    total = (sum_i sum |g|^p)^(1/p) (p = inf: max |g|); coef = clamp(max_norm /
+    (total + 1e-6), max=1), NaN when total is NaN (so every gradient becomes
+    NaN, as with PyTorch's clip_grad_norm_; the returned total is what a
+    caller checks for non-finite values); returns (clipped gradients, total,
+    coef).  Training Guide, "Gradient Clipping": after the reduce, before
+    momentum + Newton-Schulz.
     """
     gs = [np.asarray(g, dtype=np.float64) for g in grads]
     if norm_type == float("inf"):
@@ -176,8 +181,9 @@ def clip_grad_norm(grads: Sequence[np.ndarray], max_norm: float, norm_type: floa
     else:
         p = float(norm_type)
         total = sum(float(np.sum(np.abs(g) ** p)) for g in gs) ** (1.0 / p)
-    # a NaN total leaves coef at 1 (min(1, nan) keeps its first argument)
-    coef = min(1.0, max_norm / (total + CLIP_EPS))
+    coef = max_norm / (total + CLIP_EPS)
+    if not math.isnan(coef):
+        coef = min(1.0, coef)
     with np.errstate(invalid="ignore"):
         return [g * coef for g in gs], total, coef
 

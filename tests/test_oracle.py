@@ -12,6 +12,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from oracle import muon as om
@@ -360,13 +361,41 @@ def test_clip_global_norm_couples_matrices():
 @pytest.mark.parametrize("norm_type", [1.0, 2.0, float("inf")])
 @pytest.mark.parametrize("where", [0, 1, 2])
 def test_clip_nan_anywhere_gives_nan_total(norm_type, where):
-    # PyTorch's clip_grad_norm_ (which the clipping section pairs the clip with)
-    # reduces with sum / max, both of which keep a NaN wherever it sits
+    # PyTorch's clip_grad_norm_ (whose name and max_norm argument the clipping
+    # section gives DMuon's clip) reduces with sum / max, both of which keep a
+    # NaN wherever it sits, and its clamp keeps the NaN coefficient: every
+    # gradient becomes NaN
     gs = [gauss((3, 4), 20 + k) for k in range(3)]
     gs[where][1, 2] = np.nan
     out, total, coef = om.clip_grad_norm(gs, 1.0, norm_type)
-    assert np.isnan(total) and coef == 1.0
-    assert all(np.array_equal(a, b, equal_nan=True) for a, b in zip(out, gs))
+    assert np.isnan(total) and np.isnan(coef)
+    assert all(np.isnan(a).all() for a in out)
+
+
+@pytest.mark.parametrize("norm_type", [1.0, 2.0, float("inf")], ids=["l1", "l2", "linf"])
+@pytest.mark.parametrize("case", ["clipped", "below", "nan", "inf", "zero"])
+def test_clip_matches_pytorch_clip_grad_norm(norm_type, case):
+    # the reading is PyTorch's formula: its own routine (CPU, fp64) pins the
+    # total, the coefficient and the clipped values, non-finite cases included
+    gs = [gauss((5, 7), 40), gauss((3, 11), 41) * 3.0, gauss((1, 4), 42)]
+    max_norm = 2.5 if case != "below" else 1e6
+    if case == "nan":
+        gs[1][2, 3] = np.nan
+    elif case == "inf":
+        gs[2][0, 1] = -np.inf
+    elif case == "zero":
+        gs = [np.zeros_like(g) for g in gs]
+    ts = [torch.nn.Parameter(torch.zeros(g.shape, dtype=torch.float64)) for g in gs]
+    for t, g in zip(ts, gs):
+        t.grad = torch.from_numpy(g.copy())
+    want_total = float(torch.nn.utils.clip_grad_norm_(ts, max_norm, norm_type=norm_type))
+    out, total, coef = om.clip_grad_norm(gs, max_norm, norm_type)
+    assert (np.isnan(total) and np.isnan(want_total)) or total == pytest.approx(want_total, rel=1e-12, abs=0)
+    for o, t in zip(out, ts):
+        w = t.grad.numpy()
+        assert np.array_equal(np.isnan(o), np.isnan(w))
+        ok = ~np.isnan(w)
+        assert np.allclose(o[ok], w[ok], rtol=1e-12, atol=0)
 
 
 def test_clip_infinity_gives_zero_coefficient():

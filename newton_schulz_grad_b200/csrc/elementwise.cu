@@ -14,6 +14,8 @@
 // moving two 8-element (16-byte for bf16) vectors.  Arithmetic is fp32 with
 // every operation rounded separately (__fmul_rn/__fadd_rn), so the stored
 // results are fixed bit for bit.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -30,9 +32,11 @@ __device__ __forceinline__ int clamp8(int64_t v) { return v < 8 ? (int)v : 8; }
 // CLIP: the gradient is first scaled by the global clipping coefficient and
 // rounded to the storage type, exactly the value a separate in-place clip
 // would have stored, so a fused clipped step equals clip-then-step bit for bit.
-template <typename T, int MODE, bool CLIP>
+// XT: element type of X in the workspace (T, or fp32 for bf16 matrices whose
+// chain keeps X in fp32; x0 is rounded to T first either way).
+template <typename T, typename XT, int MODE, bool CLIP>
 __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
-    k_momentum(const __grid_constant__ ElemTable tab, T* __restrict__ X, float* __restrict__ partials,
+    k_momentum(const __grid_constant__ ElemTable tab, XT* __restrict__ X, float* __restrict__ partials,
                float mu, int nesterov, int dst_vec, const float* __restrict__ clip_coef) {
   __shared__ float s[T64][T64 + 1];
   __shared__ float red[kThreads / 32];
@@ -50,7 +54,7 @@ __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
   const int rr = tid >> 3;
   const T* g = static_cast<const T*>(me.src);
   T* buf = static_cast<T*>(me.buf);
-  T* Xm = X + (int64_t)e * tab.m * tab.ldn;
+  XT* Xm = X + (int64_t)e * tab.m * tab.ldn;
 
   float ss = 0.f;
 #pragma unroll
@@ -91,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
       if (!tr && DMUON_IN(tab.status, gc, valid, tab.ldn) &&
           DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + gr * tab.ldn + gc, valid,
                    (int64_t)tab.count * tab.m * tab.ldn))
-        store8<T>(Xm + gr * tab.ldn + gc, x, dst_vec && valid == 8, valid);
+        store8<XT>(Xm + gr * tab.ldn + gc, x, dst_vec && valid == 8, valid);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = 0.f;
@@ -116,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, CLIP ? 6 : 8)
         if (DMUON_IN(tab.status, r0 + j0, valid, tab.ldn) &&
             DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + (c0 + i) * tab.ldn + r0 + j0, valid,
                      (int64_t)tab.count * tab.m * tab.ldn))
-          store8<T>(Xm + (c0 + i) * tab.ldn + r0 + j0, y, dst_vec && valid == 8, valid);
+          store8<XT>(Xm + (c0 + i) * tab.ldn + r0 + j0, y, dst_vec && valid == 8, valid);
       }
     }
   }
@@ -151,9 +155,11 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-template <typename T, int MODE>
+// XT: element type of O in the workspace; an fp32 O of a bf16 matrix is
+// rounded to bf16 first, the value dmuon_ns would return for it.
+template <typename T, typename XT, int MODE>
 __global__ void __launch_bounds__(kThreads)
-    k_update(const __grid_constant__ ElemTable tab, const T* __restrict__ O,
+    k_update(const __grid_constant__ ElemTable tab, const XT* __restrict__ O,
              const float* __restrict__ scale, float decay, float step_scale, int o_vec) {
   __shared__ float s[T64][T64 + 1];
   const int e = blockIdx.y;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x;
   const int cv = tid & 7;
   const int rr = tid >> 3;
-  const T* Om = O + (int64_t)e * tab.m * tab.ldn;
+  const XT* Om = O + (int64_t)e * tab.m * tab.ldn;
   T* p = static_cast<T*>(me.dst);
   const float sc = scale ? scale[e] : 1.f;
 
@@ -183,7 +189,11 @@ __global__ void __launch_bounds__(kThreads)
       if (valid > 0 && DMUON_IN(tab.status, r0 + j0, valid, tab.ldn) &&
           DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + (c0 + i) * tab.ldn + r0 + j0, valid,
                    (int64_t)tab.count * tab.m * tab.ldn)) {
-        load8<T>(Om + (c0 + i) * tab.ldn + r0 + j0, y, o_vec && valid == 8, valid);
+        load8<XT>(Om + (c0 + i) * tab.ldn + r0 + j0, y, o_vec && valid == 8, valid);
+        if (!std::is_same<T, XT>::value) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) y[k] = round_to<T>(y[k]);
+        }
       } else {
 #pragma unroll
         for (int k = 0; k < 8; ++k) y[k] = 0.f;
@@ -208,7 +218,11 @@ __global__ void __launch_bounds__(kThreads)
     } else if (DMUON_IN(tab.status, gc, valid, tab.ldn) &&
                DMUON_IN(tab.status, (int64_t)e * tab.m * tab.ldn + gr * tab.ldn + gc, valid,
                         (int64_t)tab.count * tab.m * tab.ldn)) {
-      load8<T>(Om + gr * tab.ldn + gc, o, o_vec && valid == 8, valid);
+      load8<XT>(Om + gr * tab.ldn + gc, o, o_vec && valid == 8, valid);
+      if (!std::is_same<T, XT>::value) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = round_to<T>(o[i]);
+      }
     } else {
       continue;
     }
@@ -236,30 +250,34 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+template <typename T, typename XT>
+void momentum_kernels(const ElemTable& t, ElemMode mode, XT* x, float* partials, float mu, int nesterov,
+                      int dst_vec, const float* clip_coef, cudaStream_t st) {
+  dim3 grid((unsigned)t.tiles_per_mat, (unsigned)t.count);
+  if (clip_coef)
+    k_momentum<T, XT, 0, true><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, clip_coef);
+  else if (mode == ElemMode::kMomentum)
+    k_momentum<T, XT, 0, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
+  else
+    k_momentum<T, XT, 1, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
+}
+
 cudaError_t launch_momentum(const ElemTable& t, int dtype, ElemMode mode, void* X, float* partials,
-                            float mu, int nesterov, cudaStream_t st, const float* clip_coef) {
+                            float mu, int nesterov, cudaStream_t st, const float* clip_coef, int xdtype) {
   if (t.count == 0) return cudaSuccess;
   if (clip_coef && mode != ElemMode::kMomentum) return cudaErrorInvalidValue;
-  const size_t es = dtype == DMUON_BF16 ? 2 : 4;
+  if (xdtype < 0) xdtype = dtype;
+  if (dtype == DMUON_F32 && xdtype != DMUON_F32) return cudaErrorInvalidValue;
+  const size_t es = xdtype == DMUON_BF16 ? 2 : 4;
   const int dst_vec = ((t.ldn * (int64_t)es) % 16 == 0) && aligned16(X);
-  dim3 grid((unsigned)t.tiles_per_mat, (unsigned)t.count);
-  if (dtype == DMUON_BF16) {
-    auto* x = static_cast<__nv_bfloat16*>(X);
-    if (clip_coef)
-      k_momentum<__nv_bfloat16, 0, true><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, clip_coef);
-    else if (mode == ElemMode::kMomentum)
-      k_momentum<__nv_bfloat16, 0, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
-    else
-      k_momentum<__nv_bfloat16, 1, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
-  } else {
-    auto* x = static_cast<float*>(X);
-    if (clip_coef)
-      k_momentum<float, 0, true><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, clip_coef);
-    else if (mode == ElemMode::kMomentum)
-      k_momentum<float, 0, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
-    else
-      k_momentum<float, 1, false><<<grid, kThreads, 0, st>>>(t, x, partials, mu, nesterov, dst_vec, nullptr);
-  }
+  if (dtype == DMUON_BF16 && xdtype == DMUON_BF16)
+    momentum_kernels<__nv_bfloat16>(t, mode, static_cast<__nv_bfloat16*>(X), partials, mu, nesterov, dst_vec,
+                                    clip_coef, st);
+  else if (dtype == DMUON_BF16)
+    momentum_kernels<__nv_bfloat16>(t, mode, static_cast<float*>(X), partials, mu, nesterov, dst_vec, clip_coef,
+                                    st);
+  else
+    momentum_kernels<float>(t, mode, static_cast<float*>(X), partials, mu, nesterov, dst_vec, clip_coef, st);
   return cudaGetLastError();
 }
 
@@ -277,28 +295,33 @@ void update_coeffs(float lr, float wd, int64_t scale_dim, float* decay, float* s
   *step_scale = (float)((double)lr * 0.2 * sqrt((double)scale_dim));
 }
 
+template <typename T, typename XT>
+void update_kernels(const ElemTable& t, ElemMode mode, const XT* o, const float* scale, float decay,
+                    float step_scale, int o_vec, cudaStream_t st) {
+  dim3 grid((unsigned)t.tiles_per_mat, (unsigned)t.count);
+  if (mode == ElemMode::kUpdate)
+    k_update<T, XT, 2><<<grid, kThreads, 0, st>>>(t, o, scale, decay, step_scale, o_vec);
+  else
+    k_update<T, XT, 3><<<grid, kThreads, 0, st>>>(t, o, scale, decay, step_scale, o_vec);
+}
+
 cudaError_t launch_update(const ElemTable& t, int dtype, ElemMode mode, const void* O,
                           const float* scale, float lr, float wd, int64_t scale_dim,
-                          cudaStream_t st) {
+                          cudaStream_t st, int xdtype) {
   if (t.count == 0) return cudaSuccess;
-  const size_t es = dtype == DMUON_BF16 ? 2 : 4;
+  if (xdtype < 0) xdtype = dtype;
+  if (dtype == DMUON_F32 && xdtype != DMUON_F32) return cudaErrorInvalidValue;
+  const size_t es = xdtype == DMUON_BF16 ? 2 : 4;
   const int o_vec = ((t.ldn * (int64_t)es) % 16 == 0) && aligned16(O);
   float decay, step_scale;
   update_coeffs(lr, wd, scale_dim, &decay, &step_scale);
-  dim3 grid((unsigned)t.tiles_per_mat, (unsigned)t.count);
-  if (dtype == DMUON_BF16) {
-    auto* o = static_cast<const __nv_bfloat16*>(O);
-    if (mode == ElemMode::kUpdate)
-      k_update<__nv_bfloat16, 2><<<grid, kThreads, 0, st>>>(t, o, scale, decay, step_scale, o_vec);
-    else
-      k_update<__nv_bfloat16, 3><<<grid, kThreads, 0, st>>>(t, o, scale, decay, step_scale, o_vec);
-  } else {
-    auto* o = static_cast<const float*>(O);
-    if (mode == ElemMode::kUpdate)
-      k_update<float, 2><<<grid, kThreads, 0, st>>>(t, o, scale, decay, step_scale, o_vec);
-    else
-      k_update<float, 3><<<grid, kThreads, 0, st>>>(t, o, scale, decay, step_scale, o_vec);
-  }
+  if (dtype == DMUON_BF16 && xdtype == DMUON_BF16)
+    update_kernels<__nv_bfloat16>(t, mode, static_cast<const __nv_bfloat16*>(O), scale, decay, step_scale, o_vec,
+                                  st);
+  else if (dtype == DMUON_BF16)
+    update_kernels<__nv_bfloat16>(t, mode, static_cast<const float*>(O), scale, decay, step_scale, o_vec, st);
+  else
+    update_kernels<float>(t, mode, static_cast<const float*>(O), scale, decay, step_scale, o_vec, st);
   return cudaGetLastError();
 }
 

@@ -20,6 +20,14 @@ constexpr int kMaxTable = 256;
 // the bf16 path (bf16 rounding of G and p(G) is too coarse for such thin
 // matrices to meet the 2e-2 budget).
 constexpr int kSmallM = 64;
+// Below this min(rows, cols), bf16 matrices that are also near-square
+// (max < kNearSquare * min) keep X in fp32 as well: their many tiny singular
+// values are not resolved by bf16 storage of X (measured: the tensor-core
+// chain exceeds 2e-2 on low-rank-plus-noise inputs there, e.g. 96 x 200 and
+// 128 x 160), and at these sizes the FFMA chain costs well under a
+// millisecond.
+constexpr int kF32XBelowM = 256;
+constexpr int kNearSquare = 3;
 
 // One matrix of an elementwise launch.  `src` is the gradient (momentum
 // stage) or the input matrix (load stage); `buf` the momentum buffer or NULL;
@@ -48,7 +56,8 @@ enum class ElemMode : int { kMomentum = 0, kLoad = 1, kUpdate = 2, kCopyOut = 3 
 enum class Path : int {
   kTensorBf16 = 0,   // bf16 X, G, P on tcgen05 tensor cores
   kSmallBf16 = 1,    // bf16 X, fp32 G, P on FFMA
-  kF32 = 2           // fp32 X, G, P on FFMA
+  kF32 = 2,          // fp32 X, G, P on FFMA
+  kBf16F32 = 3       // bf16 matrix, fp32 X, G, P on FFMA (small, near-square)
 };
 
 // ---- elementwise.cu --------------------------------------------------------
@@ -56,9 +65,11 @@ enum class Path : int {
 // transposed where the entry says so) and one fp32 sum-of-squares partial per
 // 64x64 tile into `partials` (tiles_per_mat per matrix).
 // clip_coef (device float, kMomentum only): scale each gradient by it first.
+// xdtype: storage type of X in the workspace (-1: dtype; DMUON_F32 for a bf16
+// matrix whose chain keeps X in fp32, see Path::kBf16F32).
 cudaError_t launch_momentum(const ElemTable& t, int dtype, ElemMode mode, void* X,
                             float* partials, float mu, int nesterov, cudaStream_t st,
-                            const float* clip_coef = nullptr);
+                            const float* clip_coef = nullptr, int xdtype = -1);
 // Sum the partials of each matrix in a fixed order; scale[i] = 1/(sqrt(sum)+eps).
 // sumsq (optional) receives the sums in fp64.
 cudaError_t launch_norm_finalize(const float* partials, int count, int tiles_per_mat,
@@ -66,9 +77,11 @@ cudaError_t launch_norm_finalize(const float* partials, int count, int tiles_per
 // Update (or copy-out) stage.  O is the oriented m x n result in the
 // workspace (pitch ldn); `scale` (optional, per matrix) multiplies O first.
 // The update uses lr * 0.2 * sqrt(scale_dim) (scale_dim = max(rows, cols)).
+// xdtype as for launch_momentum; an fp32 O of a bf16 matrix is rounded to
+// bf16 before it is used.
 cudaError_t launch_update(const ElemTable& t, int dtype, ElemMode mode, const void* O,
                           const float* scale, float lr, float wd, int64_t scale_dim,
-                          cudaStream_t st);
+                          cudaStream_t st, int xdtype = -1);
 
 // ---- simt_gemm.cu -----------------------------------------------------------
 // FFMA chain kernels, batched over `batch` matrices with element batch strides.
@@ -145,6 +158,17 @@ cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st);
 // ---- api.cu -------------------------------------------------------------------
 // Sets the message returned by dmuon_get_last_error on this thread; returns s.
 dmuon_status_t record_error(dmuon_status_t s, const std::string& msg);
+struct ChunkLayout;
+struct ChunkOffsets;
+// The Newton-Schulz chain that dmuon_ns_ex and dmuon_step run, over a chunk of
+// `b` oriented m x n matrices whose x0 is in the workspace `ws` (laid out by
+// chunk_offsets, per-matrix scales filled in); sched holds 3 * steps
+// coefficients (a, b, c per iteration); *result receives the buffer holding
+// the result.  `status` is the device status word the kernels'
+// bounded waits report to; `sms` the device's SM count.
+dmuon_status_t ns_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char* ws, const ChunkOffsets& off,
+                        int32_t steps, const float* sched, int* status, int sms, cudaStream_t st,
+                        void** result);
 
 // ---- plan.cpp -----------------------------------------------------------------
 struct Group {
@@ -175,6 +199,10 @@ struct ChunkLayout {
 };
 // allow_blocked = false keeps the per-iteration form (two m x m buffers).
 ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype, bool allow_blocked = true);
+// Storage type of X in the workspace of a layout.
+inline int32_t x_dtype(const ChunkLayout& L, int32_t dtype) {
+  return L.path == Path::kBf16F32 ? (int32_t)DMUON_F32 : dtype;
+}
 // Iteration blocks of the chain for `steps` iterations: all 1 in the
 // per-iteration form; otherwise the Gram-space schedule of DMUON_GRAM_BLOCKS
 // (default: per-iteration steps, then the last two iterations as one block;

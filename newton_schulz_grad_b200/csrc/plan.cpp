@@ -63,13 +63,23 @@ ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype, bool allow_blocked
   ChunkLayout L{};
   if (dtype == DMUON_F32)
     L.path = Path::kF32;
+  else if (m <= kSmallM)
+    L.path = Path::kSmallBf16;
+  else if (m < kF32XBelowM && n < kNearSquare * m)
+    L.path = Path::kBf16F32;
   else
-    L.path = (m <= kSmallM) ? Path::kSmallBf16 : Path::kTensorBf16;
+    L.path = Path::kTensorBf16;
   // Gram-space blocks cost 3 m^2 n + (4L - 3) m^3 per block of L iterations
-  // against L (3 m^2 n + m^3) iteration by iteration: fewer flops once n > m.
-  L.blocked = allow_blocked && gram_block_mode() != 0 && L.path == Path::kTensorBf16 && 4 * n >= 5 * m;
+  // against L (3 m^2 n + m^3) iteration by iteration: fewer flops once n > m,
+  // but Gram space squares the singular values, so bf16 rounding there costs
+  // accuracy, the more the closer to square the matrix is and the smaller it
+  // is (measured 1.5-1.8e-2 against 1.0-1.2e-2 at n = 1.25 m, m = 256..384, for
+  // 3 % fewer flops).  Used where n >= 2 m (8.6 % fewer flops or more), or
+  // n >= 1.25 m once m >= 512.
+  const bool wide = n >= 2 * m || (m >= 512 && 4 * n >= 5 * m);
+  L.blocked = allow_blocked && gram_block_mode() != 0 && L.path == Path::kTensorBf16 && wide;
   L.gslots = L.blocked ? 5 : 2;
-  const int64_t xs = dtype == DMUON_BF16 ? 2 : 4;
+  const int64_t xs = (dtype == DMUON_BF16 && L.path != Path::kBf16F32) ? 2 : 4;
   const int64_t gs = L.path == Path::kTensorBf16 ? 2 : 4;
   // 16-byte row pitch: the TMA descriptors need it, vector loads like it
   L.ldn = round_up(n, 8);

@@ -8,9 +8,9 @@
 //   (ns_steps x (gram, poly, apply); wide matrices on the tensor path run
 //   their last two iterations as one Gram-space block) -> update
 // With several chunks the elementwise stages run on an internal stream
-// underneath the chains of neighbouring chunks (two workspace buffers),
-// ordered by events and joined back into the caller's stream; there is no
-// host synchronisation.
+// underneath the chains of neighbouring chunks (two workspace buffers), the
+// chains on a second, higher-priority internal stream, ordered by events and
+// joined back into the caller's stream; there is no host synchronisation.
 //
 // Environment switches (read per call): DMUON_WS_CAP_MB (workspace cap,
 // default 8 GiB), DMUON_OVERLAP=0 (serial schedule), DMUON_GRAM_BLOCKS=0|2
@@ -153,22 +153,36 @@ dmuon_status_t get_workspace(size_t bytes, cudaStream_t st, void** out) {
   return DMUON_OK;
 }
 
-// Auxiliary stream per (device, caller stream) for the elementwise stages of
-// an overlapped step.
-std::map<std::pair<int, uintptr_t>, cudaStream_t> g_aux;
+// Internal streams per (device, caller stream) of an overlapped step: `aux`
+// (least priority) for the elementwise stages, `chain` (greatest priority) for
+// the Newton-Schulz chains.  The priorities matter when a chain kernel is
+// launched while a momentum kernel still has blocks waiting: the block
+// scheduler then places the chain kernel's persistent CTAs first, instead of
+// letting the waiting momentum blocks take the SMs as they free up (which
+// delayed the chain kernel by about the momentum kernel's whole duration).
+struct SideStreams {
+  cudaStream_t aux = nullptr, chain = nullptr;
+};
+std::map<std::pair<int, uintptr_t>, SideStreams> g_side;
 
-dmuon_status_t get_aux_stream(cudaStream_t st, cudaStream_t* out) {
+dmuon_status_t get_side_streams(cudaStream_t st, SideStreams* out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_mu);
   auto key = std::make_pair(dev, reinterpret_cast<uintptr_t>(st));
-  auto it = g_aux.find(key);
-  if (it == g_aux.end()) {
-    cudaStream_t aux = nullptr;
-    e = cudaStreamCreateWithFlags(&aux, cudaStreamNonBlocking);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
-    it = g_aux.emplace(key, aux).first;
+  auto it = g_side.find(key);
+  if (it == g_side.end()) {
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    SideStreams ss;
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.aux, cudaStreamNonBlocking, least);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.chain, cudaStreamNonBlocking, greatest);
+    if (e != cudaSuccess) {
+      if (ss.aux) cudaStreamDestroy(ss.aux);
+      return cuda_fail(e, "cudaStreamCreateWithPriority");
+    }
+    it = g_side.emplace(key, ss).first;
   }
   *out = it->second;
   return DMUON_OK;
@@ -281,8 +295,8 @@ bool fuses_update(const ChunkLayout& L, int32_t steps) {
 // upd (optional, only where fuses_update): the last apply updates the
 // parameters in its epilogue and stores no result (*result = nullptr).
 dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char* ws,
-                         const ChunkOffsets& off, int32_t steps, const std::vector<float>& sched,
-                         const DeviceState& ds, cudaStream_t st, void** result,
+                         const ChunkOffsets& off, int32_t steps, const float* sched,
+                         int* sw, int sms, cudaStream_t st, void** result,
                          const UpdTable* upd = nullptr) {
   void* cur = ws + off.x0;
   void* nxt = ws + off.x1;
@@ -293,8 +307,6 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   const bool xbf16 = L.path == Path::kSmallBf16;
   const double fm = (double)m, fn = (double)n, fb = (double)b;
   const int mi = (int)m, ni = (int)n;
-  int* sw = ds.status_word;
-  const int sms = ds.sm_count;
   cudaError_t e = cudaSuccess;
   // m x m slot s of the chunk (slot 0 is G, the rest follow P)
   auto slot = [&](int s) -> char* { return s == 0 ? (char*)G : (char*)P + (int64_t)(s - 1) * ((off.p - off.g)); };
@@ -330,7 +342,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   // thin matrices: the whole chain in one clustered launch, in place on X0
   if (thin_chain(L, m, n, steps)) {
     Prof p(kChainSmall, st, fb * (3.0 * fm * fm * fn + fm * fm * fm) * steps, 0.0);
-    e = small_ns(cur, b, mi, ni, L.ldn, steps, sched.data(), scale, xbf16, st, sw);
+    e = small_ns(cur, b, mi, ni, L.ldn, steps, sched, scale, xbf16, st, sw);
     p.done(st);
     if (e != cudaSuccess) return cuda_fail(e, "Newton-Schulz launch");
     *result = cur;
@@ -530,23 +542,35 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     if (e != cudaSuccess) return cuda_fail(e, "clip norm launch");
     clip_coef = clip_coef_ptr(cws, clip_tile_count);
   }
-  // elementwise stages run on `aux` when overlapping, else on the caller's stream
-  cudaStream_t aux = st;
+  // when overlapping, the elementwise stages run on `aux` and the chains on
+  // `cs`; otherwise everything runs on the caller's stream
+  cudaStream_t aux = st, cs = st;
   if (P.overlap) {
-    rc = get_aux_stream(st, &aux);
+    SideStreams ss;
+    rc = get_side_streams(st, &ss);
     if (rc != DMUON_OK) return rc;
+    aux = ss.aux;
+    cs = ss.chain;
     cudaError_t e = stream_after(aux, st);
-    if (e != cudaSuccess) return cuda_fail(e, "stream fork");
-  }
-  // Every return after the fork leaves the caller's stream ordered after aux,
-  // so a call that fails part-way leaves none of its work unordered.
-  struct JoinAux {
-    cudaStream_t st, aux;
-    bool on;
-    ~JoinAux() {
-      if (on) stream_after(st, aux);
+    if (e == cudaSuccess) e = stream_after(cs, st);
+    if (e != cudaSuccess) {
+      stream_after(st, aux);
+      return cuda_fail(e, "stream fork");
     }
-  } join{st, aux, P.overlap};
+  }
+  // Every return after the fork leaves the caller's stream ordered after both
+  // internal streams, so a call that fails part-way leaves none of its work
+  // unordered.
+  struct JoinSide {
+    cudaStream_t st, aux, cs;
+    bool on;
+    ~JoinSide() {
+      if (on) {
+        stream_after(st, aux);
+        stream_after(st, cs);
+      }
+    }
+  } join{st, aux, cs, P.overlap};
   std::vector<void*> results(P.chunks.size(), nullptr);
   std::unique_ptr<UpdTable> upd_tab(new UpdTable());
 
@@ -581,14 +605,17 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     const double elems = (double)ck.b * (double)c.m * (double)c.n;
     Prof pu(kUpdate, aux, 0.0, 3.0 * elems * (double)esize(c.dtype));
     cudaError_t e = launch_update(tabs[i % 2], c.dtype, ElemMode::kUpdate, results[i], ns_steps == 0 ? scale : nullptr,
-                                  lr, wd, c.n, aux);
+                                  lr, wd, c.n, aux, x_dtype(P.layouts[ck.cls], c.dtype));
     pu.done(aux);
     return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "update launch");
   };
 
   // ------------------------------------------------------------ execution
-  // aux: M0 N0 | M1 N1 U0 | M2 N2 U1 | ...   caller: chain0 | chain1 | ...
-  // U(i-1) waits only for chain(i-1) (event recorded when it was enqueued).
+  // aux: M0 N0 | M1 N1 U0 | M2 N2 U1 | ...   cs: chain0 | chain1 | ...
+  // U(i-1) waits only for chain(i-1) (event recorded when it was enqueued);
+  // M(i+1) comes after that wait, so it overwrites buffer (i+1) % 2 only once
+  // chain(i-1), which used it, is done.  Without overlap, cs and aux are the
+  // caller's stream.
   cudaEvent_t chain_done = nullptr;
   auto drop = [&]() {
     if (chain_done) cudaEventDestroy(chain_done);  // released once complete
@@ -606,7 +633,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     const double elems = (double)ck.b * (double)c.m * (double)c.n;
     Prof pm(kMomentum, aux, 0.0, 4.0 * elems * (double)esize(c.dtype));
     cudaError_t e = launch_momentum(tabs[i % 2], c.dtype, ElemMode::kMomentum, ws + off.x0, partials, momentum,
-                                    nesterov, aux, clip_coef);
+                                    nesterov, aux, clip_coef, x_dtype(L, c.dtype));
     pm.done(aux);
     if (e != cudaSuccess) {
       drop();
@@ -615,7 +642,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     Prof pn(kNorm, aux, 0.0, 4.0 * (double)ck.b * (double)L.tiles_per_mat);
     e = launch_norm_finalize(partials, ck.b, (int)L.tiles_per_mat, scale, nullptr, aux);
     pn.done(aux);
-    if (e == cudaSuccess && P.overlap) e = stream_after(st, aux);
+    if (e == cudaSuccess && P.overlap) e = stream_after(cs, aux);
     if (e != cudaSuccess) {
       drop();
       return cuda_fail(e, "norm launch / stream join");
@@ -641,7 +668,8 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     }
     {
       NvtxRange r("chain " + std::to_string(c.m) + "x" + std::to_string(c.n) + " x" + std::to_string(ck.b));
-      rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched, ds, st, &results[i], upd);
+      rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched.data(), ds.status_word, ds.sm_count, cs, &results[i],
+                     upd);
     }
     if (rc != DMUON_OK) {
       drop();
@@ -666,7 +694,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     }
     drop();
     e = cudaEventCreateWithFlags(&chain_done, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventRecord(chain_done, st);
+    if (e == cudaSuccess) e = cudaEventRecord(chain_done, cs);
     if (e != cudaSuccess) {
       drop();
       return cuda_fail(e, "chain event");
@@ -680,6 +708,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     if (rc != DMUON_OK) return rc;
     join.on = false;
     e = stream_after(st, aux);
+    if (e == cudaSuccess) e = stream_after(st, cs);
     if (e != cudaSuccess) return cuda_fail(e, "stream join");
   }
   return DMUON_OK;
@@ -688,6 +717,12 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
 }  // namespace
 
 dmuon_status_t record_error(dmuon_status_t s, const std::string& msg) { return fail(s, msg); }
+
+dmuon_status_t ns_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char* ws, const ChunkOffsets& off,
+                        int32_t steps, const float* sched, int* status, int sms, cudaStream_t st,
+                        void** result) {
+  return run_chain(L, b, m, n, ws, off, steps, sched, status, sms, st, result);
+}
 
 }  // namespace dmuon
 
@@ -848,7 +883,8 @@ dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int64_t cols,
   float* scale = reinterpret_cast<float*>(ws + off.scale);
   const double elems = (double)m * (double)n, es = (double)esize(dtype);
   Prof pl(kLoad, st, 0.0, 2.0 * elems * es);
-  cudaError_t e = launch_momentum(*tab, dtype, ElemMode::kLoad, ws + off.x0, partials, 0.f, 0, st);
+  cudaError_t e = launch_momentum(*tab, dtype, ElemMode::kLoad, ws + off.x0, partials, 0.f, 0, st, nullptr,
+                                  x_dtype(L, dtype));
   pl.done(st);
   if (e != cudaSuccess) return cuda_fail(e, "load launch");
   Prof pn(kNorm, st, 0.0, 4.0 * (double)L.tiles_per_mat);
@@ -856,10 +892,11 @@ dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int64_t cols,
   pn.done(st);
   if (e != cudaSuccess) return cuda_fail(e, "norm launch");
   void* result = nullptr;
-  rc = run_chain(L, 1, m, n, ws, off, steps, sched, ds, st, &result);
+  rc = run_chain(L, 1, m, n, ws, off, steps, sched.data(), ds.status_word, ds.sm_count, st, &result);
   if (rc != DMUON_OK) return rc;
   Prof pc(kCopyOut, st, 0.0, 2.0 * elems * es);
-  e = launch_update(*tab, dtype, ElemMode::kCopyOut, result, steps == 0 ? scale : nullptr, 0.f, 0.f, n, st);
+  e = launch_update(*tab, dtype, ElemMode::kCopyOut, result, steps == 0 ? scale : nullptr, 0.f, 0.f, n, st,
+                    x_dtype(L, dtype));
   pc.done(st);
   if (e != cudaSuccess) return cuda_fail(e, "copy-out launch");
   return DMUON_OK;
@@ -1011,6 +1048,40 @@ dmuon_status_t dmuon_profile_start(void) {
   return DMUON_OK;
 }
 
+int32_t dmuon_profile_stop_launches(dmuon_launch_record_t* recs, int32_t max_recs) {
+  g_prof_on = false;
+  bool ok = true;
+  if (!g_prof.empty() && cudaEventSynchronize(g_prof.back().b) != cudaSuccess) ok = false;
+  int32_t n = 0;
+  for (size_t i = 0; i < g_prof.size(); ++i) {
+    ProfRec& r = g_prof[i];
+    float t = 0.f, t0 = 0.f;
+    if (ok && (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess ||
+               cudaEventElapsedTime(&t0, g_prof.front().a, r.a) != cudaSuccess))
+      ok = false;
+    if (ok && recs && n < max_recs) {
+      dmuon_launch_record_t& o = recs[n];
+      std::memset(&o, 0, sizeof(o));
+      std::strncpy(o.name, kKindNames[r.kind], sizeof(o.name) - 1);
+      o.start_ms = t0;
+      o.ms = t;
+      o.flops = r.flops;
+      o.bytes = r.bytes;
+    }
+    ++n;
+  }
+  for (ProfRec& r : g_prof) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof.clear();
+  if (!ok) {
+    fail(DMUON_ERR_CUDA, "profile events failed");
+    return -1;
+  }
+  return n;
+}
+
 int32_t dmuon_profile_stop(dmuon_kernel_stat_t* stats, int32_t max_stats) {
   g_prof_on = false;
   double ms[kNumKinds] = {0}, fl[kNumKinds] = {0}, by[kNumKinds] = {0};
@@ -1102,10 +1173,11 @@ void dmuon_release_workspace(void) {
       ++it;
     }
   }
-  for (auto it = g_aux.begin(); it != g_aux.end();) {
+  for (auto it = g_side.begin(); it != g_side.end();) {
     if (it->first.first == dev) {
-      cudaStreamDestroy(it->second);
-      it = g_aux.erase(it);
+      cudaStreamDestroy(it->second.aux);
+      cudaStreamDestroy(it->second.chain);
+      it = g_side.erase(it);
     } else {
       ++it;
     }

@@ -30,30 +30,37 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DMUON_NOALLOC_SCRATCH_BYTES];
 constexpr size_t kHeader = 256;
 
-// Per-device set-up, done once with that device current: the device address
-// of the array (host code only holds a stand-in for it) and the SM count.
+// Per-device set-up with that device current: the device address of the array
+// (host code only holds a stand-in for it) and the SM count.  It is marked done
+// only once it succeeded, so a failed first attempt (for instance one made
+// while a stream was capturing) is retried by the next call.
 constexpr int kMaxDevices = 64;
 struct DeviceSetup {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
+  bool done = false;
   void* scratch = nullptr;
   int sm_count = 0;
   int major = 0;
 };
+std::mutex g_setup_mu;
 DeviceSetup g_setup[kMaxDevices];
 
-cudaError_t setup_device(int dev, DeviceSetup** out) {
-  DeviceSetup* d = &g_setup[dev];
-  std::call_once(d->once, [d, dev]() {
-    d->err = cudaGetSymbolAddress(&d->scratch, g_noalloc_scratch);
-    if (d->err == cudaSuccess)
-      d->err = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
-    if (d->err == cudaSuccess)
-      d->err = cudaDeviceGetAttribute(&d->major, cudaDevAttrComputeCapabilityMajor, dev);
-    if (d->err != cudaSuccess) d->scratch = nullptr;
-  });
+cudaError_t setup_device(int dev, DeviceSetup* out) {
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  DeviceSetup& d = g_setup[dev];
+  if (!d.done) {
+    DeviceSetup t;
+    cudaError_t e = cudaGetSymbolAddress(&t.scratch, g_noalloc_scratch);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&t.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&t.major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // not sticky: the next call tries again
+      return e;
+    }
+    t.done = true;
+    d = t;
+  }
   *out = d;
-  return d->err;
+  return cudaSuccess;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -81,7 +88,8 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
   const uintptr_t bytes = (uintptr_t)(rows * cols * es), x = (uintptr_t)X, o = (uintptr_t)out;
   if (x < o + bytes && o < x + bytes) return record_error(DMUON_ERR_INVALID_ARG, "out may not overlap X");
   const int64_t m = std::min(rows, cols), n = std::max(rows, cols);
-  const ChunkLayout L = chunk_layout(m, n, dtype, /*allow_blocked=*/false);
+  // the layout and schedule of dmuon_ns_ex, so both give the same bits
+  const ChunkLayout L = chunk_layout(m, n, dtype);
   const ChunkOffsets off = chunk_offsets(L, 1);
   const size_t need = kHeader + (size_t)off.total;
   if (need > (size_t)DMUON_NOALLOC_SCRATCH_BYTES)
@@ -89,7 +97,7 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
                         "dmuon_ns_noalloc: a " + std::to_string(rows) + "x" + std::to_string(cols) +
                             " matrix needs " + std::to_string(need) + " bytes of scratch; the fixed array holds " +
                             std::to_string((size_t)DMUON_NOALLOC_SCRATCH_BYTES));
-  float sched[3 * 1000];
+  float sched[3 * 1000];  // on the stack
   for (int32_t k = 0; k < steps; ++k) {
     sched[3 * k] = coeffs ? coeffs[3 * k] : DMUON_DEFAULT_A;
     sched[3 * k + 1] = coeffs ? coeffs[3 * k + 1] : DMUON_DEFAULT_B;
@@ -101,12 +109,12 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return record_error(DMUON_ERR_UNSUPPORTED, "device ordinal beyond 63");
-  DeviceSetup* d = nullptr;
+  DeviceSetup d;
   e = setup_device(dev, &d);
   if (e != cudaSuccess) return cuda_error(e, "scratch address lookup");
-  if (d->major != 10) return record_error(DMUON_ERR_UNSUPPORTED, "this library is built for sm_100a");
+  if (d.major != 10) return record_error(DMUON_ERR_UNSUPPORTED, "this library is built for sm_100a");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  char* base = static_cast<char*>(d->scratch);
+  char* base = static_cast<char*>(d.scratch);
   int* status_word = status ? status : reinterpret_cast<int*>(base);
   char* ws = base + kHeader;
   e = cudaMemsetAsync(status_word, 0, sizeof(int), st);
@@ -125,31 +133,14 @@ extern "C" dmuon_status_t dmuon_ns_noalloc(const void* X, void* out, int64_t row
                       ((row16 && aligned16(X)) ? 1 : 0) | ((row16 && aligned16(out)) ? 2 : 0)};
   float* partials = reinterpret_cast<float*>(ws + off.partials);
   float* scale = reinterpret_cast<float*>(ws + off.scale);
-  e = launch_momentum(tab, dtype, ElemMode::kLoad, ws + off.x0, partials, 0.f, 0, st);
+  e = launch_momentum(tab, dtype, ElemMode::kLoad, ws + off.x0, partials, 0.f, 0, st, nullptr, x_dtype(L, dtype));
   if (e == cudaSuccess) e = launch_norm_finalize(partials, 1, (int)L.tiles_per_mat, scale, nullptr, st);
-  void* cur = ws + off.x0;
-  void* nxt = ws + off.x1;
-  void* G = ws + off.g;
-  void* P = ws + off.p;
-  for (int32_t k = 0; k < steps && e == cudaSuccess; ++k) {
-    const float a = sched[3 * k], b = sched[3 * k + 1], c = sched[3 * k + 2];
-    const float* sc = k == 0 ? scale : nullptr;
-    if (L.path == Path::kTensorBf16) {
-      e = tc_gram(cur, G, 1, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, status_word, d->sm_count, st);
-      if (e == cudaSuccess) e = tc_poly(G, P, 1, (int)m, L.ldm, L.ldm, b, c, status_word, d->sm_count, st);
-      if (e == cudaSuccess)
-        e = tc_apply(P, cur, nxt, 1, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, status_word, d->sm_count,
-                     st);
-    } else {
-      const bool xbf16 = L.path == Path::kSmallBf16;
-      e = simt_gram(cur, G, 1, (int)m, (int)n, L.ldn, L.ldm, 1.f, sc, xbf16, st, status_word);
-      if (e == cudaSuccess) e = simt_poly(G, P, 1, (int)m, L.ldm, L.ldm, b, c, st, status_word);
-      if (e == cudaSuccess) e = simt_apply(P, cur, nxt, 1, (int)m, (int)n, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st, status_word);
-    }
-    std::swap(cur, nxt);
-  }
-  if (e == cudaSuccess)
-    e = launch_update(tab, dtype, ElemMode::kCopyOut, cur, steps == 0 ? scale : nullptr, 0.f, 0.f, n, st);
+  if (e != cudaSuccess) return cuda_error(e, "dmuon_ns_noalloc launch");
+  void* result = nullptr;
+  const dmuon_status_t rc = ns_chain(L, 1, m, n, ws, off, steps, sched, status_word, d.sm_count, st, &result);
+  if (rc != DMUON_OK) return rc;
+  e = launch_update(tab, dtype, ElemMode::kCopyOut, result, steps == 0 ? scale : nullptr, 0.f, 0.f, n, st,
+                    x_dtype(L, dtype));
   if (e != cudaSuccess) return cuda_error(e, "dmuon_ns_noalloc launch");
   return DMUON_OK;
 }

@@ -109,10 +109,11 @@ typedef struct {
  *   coeffs HOST array of 3*steps floats (a_k, b_k, c_k for iteration k), or
  *          NULL for the default triple at every iteration
  * Works over the smaller side (transposes internally when rows > cols).
- * Uses the library's cached workspace for this (device, stream).  When
- * max(rows, cols) >= 1.25 min(rows, cols) and the tensor path runs, the last
- * two iterations are carried out as one block in Gram space (the same result
- * in exact arithmetic, fewer flops); see dmuon_gram_poly.
+ * Uses the library's cached workspace for this (device, stream).  The shape
+ * decides the path as for dmuon_step (see there); on the tensor-core path the
+ * last two iterations of wide matrices are carried out as one block in Gram
+ * space (the same result in exact arithmetic, fewer flops); see
+ * dmuon_gram_poly.
  */
 DMUON_API dmuon_status_t dmuon_ns(const void* X, void* out, int64_t rows, int64_t cols, int32_t steps,
                         const float* coeffs, dmuon_stream_t stream);
@@ -147,9 +148,18 @@ DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int
  * runs inside the chain's last product (its epilogue writes the parameters;
  * DMUON_FUSED_UPDATE=0 runs it as a separate pass, with the same bits).  With
  * several chunks the momentum stage (and any separate update) runs on an
- * internal stream underneath the Newton-Schulz chain and is joined back into
- * `stream` before the call returns, on error paths too; the results do not
- * depend on that schedule.
+ * internal least-priority stream underneath the Newton-Schulz chains, which
+ * run on an internal greatest-priority stream; both fork from `stream` and are
+ * joined back into it before the call returns, on error paths too.  The
+ * results do not depend on that schedule.
+ *
+ * Routing by shape (m = min(R, C), n = max(R, C)), all in one call: fp32
+ * matrices run an FFMA chain with fp32 X, G and p(G); bf16 matrices with
+ * m <= 64 keep G and p(G) in fp32 (FFMA); bf16 matrices with m < 256 and
+ * n < 3 m keep X in fp32 as well (FFMA; bf16 storage of X cannot resolve the
+ * many small singular values of such near-square matrices within 2e-2); all
+ * other bf16 matrices run the tcgen05 chain, whose last two iterations run
+ * in Gram space when n >= 2 m, or n >= 1.25 m and m >= 512.
  */
 DMUON_API dmuon_status_t dmuon_step(void* const* params, const void* const* grads, void* const* mom_bufs,
                           const dmuon_shape_t* shapes, int32_t count, float lr, float momentum,
@@ -178,10 +188,12 @@ DMUON_API dmuon_status_t dmuon_step_clipped(void* const* params, const void* con
  * place (DMuon Training Guide, "Gradient Clipping": the Muon-only clip runs
  * after the gradient reduce and before momentum + Newton-Schulz; the default
  * strategy is global p-norm clipping).  Read with PyTorch's clip_grad_norm_
- * formula, which the same section pairs it with:
+ * formula: the section gives DMuon's clip that routine's name and max_norm
+ * argument and uses the two side by side:
  *   total = (sum over every element of every matrix of |g|^p)^(1/p)
  *           (p = inf: max |g|)
- *   coef  = min(1, max_norm / (total + 1e-6)),  g <- fl(g * fl32(coef))
+ *   coef  = min(1, max_norm / (total + 1e-6)) (NaN if total is NaN),
+ *   g <- fl(g * fl32(coef))
  * Every gradient is rewritten; with coef = 1 the values are unchanged.
  *   grads      HOST array of `count` DEVICE pointers (shapes[i], row-major)
  *   shapes     HOST array of `count` shapes; gradients must not overlap
@@ -189,8 +201,10 @@ DMUON_API dmuon_status_t dmuon_step_clipped(void* const* params, const void* con
  *   norm_type  1, 2 or INFINITY (others: DMUON_ERR_UNSUPPORTED)
  *   total_norm DEVICE double or NULL: receives `total`
  * Deterministic (fixed-order fp64 reduction of per-tile fp32 partials).
- * Non-finite gradients: a NaN anywhere makes `total` NaN and coef 1 (nothing
- * is scaled); an infinity (and no NaN) makes `total` inf and coef 0.
+ * Non-finite gradients follow PyTorch's formula: a NaN anywhere makes `total`
+ * NaN and coef NaN, so every gradient becomes NaN; an infinity (and no NaN)
+ * makes `total` inf and coef 0 (finite values become 0, infinities NaN).
+ * `total` is the value to check for non-finite gradients before a step.
  */
 DMUON_API dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* shapes, int32_t count,
                                               float max_norm, float norm_type, double* total_norm,
@@ -272,10 +286,10 @@ DMUON_API dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, 
 /* Allocation-free variant                                                   */
 /* ------------------------------------------------------------------------ */
 
-/* Size of the fixed scratch array behind dmuon_ns_noalloc (16 MiB).  Every
+/* Size of the fixed scratch array behind dmuon_ns_noalloc (32 MiB).  Every
  * GPU on which the library is loaded holds this array until the process
  * exits. */
-#define DMUON_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define DMUON_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /*
  * dmuon_ns_noalloc - dmuon_ns_ex for callers that must not allocate device
@@ -285,19 +299,22 @@ DMUON_API dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, 
  * (cudaMalloc can synchronise the device and its cost is unpredictable).
  * Instead of the cached workspace of dmuon_ns_ex it uses one fixed
  * DMUON_NOALLOC_SCRATCH_BYTES array in device memory that the library
- * reserves when it is loaded; it never calls cudaMalloc or cudaFree.
+ * reserves when it is loaded; it never calls cudaMalloc or cudaFree.  It runs
+ * the kernels of dmuon_ns_ex in the same order, so both give the same bits.
  *   X, out, rows, cols, steps, coeffs, dtype  as for dmuon_ns_ex
  *   status  device, 1 int32, or NULL: cleared at the start of the call, then
  *           set to DMUON_ERR_TIMEOUT if a bounded device wait ran out (with
  *           NULL the word lives in the scratch array and is not reported)
  * Limit: the problem must fit the array; a matrix whose workspace (two m x n
- * copies of X, two m x m Gram-sized matrices and the norm partials, m =
- * min(rows, cols)) exceeds it is rejected with DMUON_ERR_INVALID_ARG and a
- * message naming both sizes.  Examples that fit: bf16 2048 x 1024, fp32
- * 1024 x 512.
+ * copies of X, the Gram-sized m x m matrices of its schedule - two, or five
+ * for a wide bf16 matrix whose last iterations run in Gram space - and the
+ * norm partials, m = min(rows, cols)) exceeds it is rejected with
+ * DMUON_ERR_INVALID_ARG and a message naming both sizes.  Examples that fit:
+ * bf16 4096 x 1024 and 2048 x 1024, fp32 2048 x 1024; bf16 2048 x 2048 does
+ * not.
  * Set-up: the first call on each device, with that device current, looks up
  * the array's device address; make that first call before any stream
- * capture.
+ * capture.  A set-up that fails is not remembered: the next call retries it.
  * Sharing: every call on a device uses the same array and leaves its
  * contents behind; calls that can overlap on the GPU (different streams
  * without ordering between them, or several host threads) race on it and
@@ -365,6 +382,24 @@ typedef struct {
 
 DMUON_API dmuon_status_t dmuon_profile_start(void);
 DMUON_API int32_t dmuon_profile_stop(dmuon_kernel_stat_t* stats, int32_t max_stats);
+
+/*
+ * dmuon_profile_stop_launches - ends the same profiling window as
+ * dmuon_profile_stop (use one or the other), but reports every launch, in
+ * the order the calls enqueued them: its kernel kind, its duration, its
+ * start relative to the first launch's start (launches on two streams may
+ * overlap), and its algorithmic work.  Fills up to max_recs records and
+ * returns the number of launches (or -1 on a CUDA error).
+ */
+typedef struct {
+    char name[32];
+    double start_ms;
+    double ms;
+    double flops;
+    double bytes;
+} dmuon_launch_record_t;
+
+DMUON_API int32_t dmuon_profile_stop_launches(dmuon_launch_record_t* recs, int32_t max_recs);
 
 /* Static string: version, target architecture, tile configuration. */
 DMUON_API const char* dmuon_build_info(void);

@@ -38,7 +38,8 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_get_last_error", "dmuon_stream_status", "dmuon_release_workspace",
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
             "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout",
-            "dmuon_clip_grad_norm", "dmuon_step_clipped", "dmuon_selftest_bounds")
+            "dmuon_clip_grad_norm", "dmuon_step_clipped", "dmuon_selftest_bounds",
+            "dmuon_profile_stop_launches")
 
 
 class DmuonError(RuntimeError):
@@ -51,6 +52,11 @@ class KernelStat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
                 ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
                 ("bytes", ctypes.c_double)]
+
+
+class LaunchRecord(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("start_ms", ctypes.c_double), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 class Shape(ctypes.Structure):
@@ -87,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_build_info": ([], ctypes.c_char_p),
         "dmuon_profile_start": ([], i32),
         "dmuon_profile_stop": ([ctypes.POINTER(KernelStat), i32], i32),
+        "dmuon_profile_stop_launches": ([ctypes.POINTER(LaunchRecord), i32], i32),
         "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
         "dmuon_selftest_timeout": ([i32, vp], i32),
         "dmuon_clip_grad_norm": ([ctypes.POINTER(vp), ctypes.POINTER(Shape), i32, f32, f32, vp, vp], i32),
@@ -120,11 +127,14 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, dev: Optional[torch.device] = None) -> ctypes.c_void_p:
+    """The cudaStream_t of `stream` (default: the current stream of `dev`)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
     if isinstance(stream, int):
         return ctypes.c_void_p(stream)
+    if dev is not None and getattr(stream, "device", dev) != dev:
+        raise ValueError(f"the stream belongs to {stream.device}, the tensors to {dev}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -132,10 +142,33 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _need_cuda(*ts: torch.Tensor) -> None:
+def _device_of(*ts: Optional[torch.Tensor]) -> torch.device:
+    """The one CUDA device that every given tensor (None skipped) lives on.
+
+    The library launches on the calling thread's current device, so a call
+    whose tensors sit on another device (or on several) is refused here, and
+    the wrappers make the tensors' device current around the call."""
+    dev = None
     for t in ts:
+        if t is None:
+            continue
         if not t.is_cuda:
             raise ValueError("tensors must live on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"all tensors of one call must be on one device ({dev} and {t.device})")
+    if dev is None:
+        raise ValueError("no tensor given")
+    return dev
+
+
+def _out_word(t: Optional[torch.Tensor], dtype: torch.dtype, name: str) -> None:
+    """Checks an optional one-element device output (status word, norm)."""
+    if t is None:
+        return
+    if t.dtype != dtype or not t.is_cuda or t.numel() < 1 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor of at least one element")
 
 
 def _coeffs(steps: int, coeffs):
@@ -179,14 +212,16 @@ def _rows_ld(t: torch.Tensor):
 # ------------------------------------------------------------- whole path
 def dmuon_ns(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=None, stream=None) -> None:
     """out = Gram Newton-Schulz(X / (||X|| + eps)); bf16 or fp32 (``dmuon_ns_ex``)."""
-    _need_cuda(X, out)
+    dev = _device_of(X, out)
     if X.shape != out.shape or X.dim() != 2 or X.dtype != out.dtype:
         raise ValueError("X and out must be 2D tensors of equal shape and dtype")
     if not (X.is_contiguous() and out.is_contiguous()):
         raise ValueError("X and out must be contiguous")
     c = _coeffs(steps, coeffs)
-    _check(_lib.dmuon_ns_ex(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps, c,
-                            _dtype_code(X), _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_ns_ex(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps, c,
+                                _dtype_code(X), st))
 
 
 def dmuon_ns_noalloc(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=None,
@@ -200,16 +235,17 @@ def dmuon_ns_noalloc(X: torch.Tensor, out: torch.Tensor, steps: int = 5, coeffs=
     DMUON_ERR_TIMEOUT if a bounded device wait ran out.  Calls share the
     array: calls that could overlap on the GPU must be serialised.
     """
-    _need_cuda(X, out)
+    _out_word(status, torch.int32, "status")
+    dev = _device_of(X, out, status)
     if X.shape != out.shape or X.dim() != 2 or X.dtype != out.dtype:
         raise ValueError("X and out must be 2D tensors of equal shape and dtype")
     if not (X.is_contiguous() and out.is_contiguous()):
         raise ValueError("X and out must be contiguous")
-    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
-        raise ValueError("status must be a CUDA int32 tensor")
-    _check(_lib.dmuon_ns_noalloc(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps,
-                                 _coeffs(steps, coeffs), _dtype_code(X), _ptr(status),
-                                 _stream(stream)))
+    c = _coeffs(steps, coeffs)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_ns_noalloc(_ptr(X), _ptr(out), X.shape[0], X.shape[1], steps, c,
+                                     _dtype_code(X), _ptr(status), st))
 
 
 def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
@@ -225,9 +261,13 @@ def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
     n = len(params)
     if len(grads) != n or len(mom_bufs) != n:
         raise ValueError("params, grads and mom_bufs must have the same length")
+    if max_norm is not None:
+        _out_word(total_norm, torch.float64, "total_norm")
+    if n == 0:
+        return
+    dev = _device_of(*params, *grads, *mom_bufs, total_norm if max_norm is not None else None)
     shapes = []
     for p, g, b in zip(params, grads, mom_bufs):
-        _need_cuda(p, g, b)
         if p.dim() != 2 or p.shape != g.shape or p.shape != b.shape:
             raise ValueError("each param, grad and buffer must be 2D with one shape")
         if not (p.dtype == g.dtype == b.dtype):
@@ -240,15 +280,15 @@ def dmuon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
     ga = (vp * max(1, n))(*[t.data_ptr() for t in grads])
     ba = (vp * max(1, n))(*[t.data_ptr() for t in mom_bufs])
     c = _coeffs(ns_steps, coeffs)
-    if max_norm is None:
-        _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
-                               ns_steps, c, wd, _stream(stream)))
-        return
-    if total_norm is not None and (total_norm.dtype != torch.float64 or not total_norm.is_cuda):
-        raise ValueError("total_norm must be a CUDA float64 tensor")
-    _check(_lib.dmuon_step_clipped(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
-                                   ns_steps, c, wd, float(max_norm), float(norm_type), _ptr(total_norm),
-                                   _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        if max_norm is None:
+            _check(_lib.dmuon_step(pa, ga, ba, _shape_array(shapes), n, lr, momentum, int(bool(nesterov)),
+                                   ns_steps, c, wd, st))
+        else:
+            _check(_lib.dmuon_step_clipped(pa, ga, ba, _shape_array(shapes), n, lr, momentum,
+                                           int(bool(nesterov)), ns_steps, c, wd, float(max_norm),
+                                           float(norm_type), _ptr(total_norm), st))
 
 
 def dmuon_step_ptrs(params: Sequence[int], grads: Sequence[int], mom_bufs: Sequence[int],
@@ -274,18 +314,21 @@ def dmuon_step_ptrs(params: Sequence[int], grads: Sequence[int], mom_bufs: Seque
 def dmuon_clip_grad_norm(grads: Sequence[torch.Tensor], max_norm: float, norm_type: float = 2.0,
                          total_norm: Optional[torch.Tensor] = None, stream=None) -> None:
     """Global p-norm clipping of the gradients, in place (see dmuon.h)."""
+    _out_word(total_norm, torch.float64, "total_norm")
+    n = len(grads)
+    if n == 0:
+        return
+    dev = _device_of(*grads, total_norm)
     shapes = []
     for g in grads:
-        _need_cuda(g)
         if g.dim() != 2 or not g.is_contiguous():
             raise ValueError("gradients must be contiguous 2D tensors")
         shapes.append((g.shape[0], g.shape[1], _dtype_code(g)))
-    if total_norm is not None and (total_norm.dtype != torch.float64 or not total_norm.is_cuda):
-        raise ValueError("total_norm must be a CUDA float64 tensor")
-    n = len(grads)
     ga = (ctypes.c_void_p * max(1, n))(*[g.data_ptr() for g in grads])
-    _check(_lib.dmuon_clip_grad_norm(ga, _shape_array(shapes), n, float(max_norm), float(norm_type),
-                                     _ptr(total_norm), _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_clip_grad_norm(ga, _shape_array(shapes), n, float(max_norm), float(norm_type),
+                                         _ptr(total_norm), st))
 
 
 def dmuon_plan_groups(shapes: Sequence[Tuple[int, int, int]]):
@@ -309,60 +352,66 @@ def dmuon_step_launches(shapes, ns_steps: int = 5) -> int:
 # ------------------------------------------------------------- stage calls
 def dmuon_gram(X: torch.Tensor, G: torch.Tensor, alpha: float = 1.0, stream=None) -> None:
     """G = alpha X X^T over a batch ([B,] m x n -> [B,] m x m)."""
-    _need_cuda(X, G)
+    dev = _device_of(X, G)
     b, m, n, ldx = _rows_ld(X)
     b2, m2, m3, ldg = _rows_ld(G)
     if (b2, m2, m3) != (b, m, m) or X.dtype != G.dtype:
         raise ValueError("G must be [B,] m x m with X's dtype")
-    _check(_lib.dmuon_gram(_ptr(X), _ptr(G), b, m, n, ldx, ldg, alpha, _dtype_code(X),
-                           _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_gram(_ptr(X), _ptr(G), b, m, n, ldx, ldg, alpha, _dtype_code(X), st))
 
 
 def dmuon_gram_poly(G: torch.Tensor, P: torch.Tensor, b: float, c: float, stream=None) -> None:
     """P = b G + c G G for symmetric G ([B,] m x m)."""
-    _need_cuda(G, P)
+    dev = _device_of(G, P)
     bb, m, m2, ldg = _rows_ld(G)
     b2, p1, p2, ldp = _rows_ld(P)
     if m != m2 or (b2, p1, p2) != (bb, m, m) or G.dtype != P.dtype:
         raise ValueError("G and P must be [B,] m x m of one dtype")
-    _check(_lib.dmuon_gram_poly(_ptr(G), _ptr(P), bb, m, ldg, ldp, b, c, _dtype_code(G),
-                                _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_gram_poly(_ptr(G), _ptr(P), bb, m, ldg, ldp, b, c, _dtype_code(G), st))
 
 
 def dmuon_poly_apply(P: torch.Tensor, X: torch.Tensor, Y: torch.Tensor, a: float,
                      alpha: float = 1.0, stream=None) -> None:
     """Y = alpha (a X + P X) ([B,] m x m, [B,] m x n -> [B,] m x n)."""
-    _need_cuda(P, X, Y)
+    dev = _device_of(P, X, Y)
     bp, m, m2, ldp = _rows_ld(P)
     bx, mx, n, ldx = _rows_ld(X)
     by, my, ny, ldy = _rows_ld(Y)
     if not (bp == bx == by and m == m2 == mx == my and n == ny) or not (P.dtype == X.dtype == Y.dtype):
         raise ValueError("shape or dtype mismatch")
-    _check(_lib.dmuon_poly_apply(_ptr(P), _ptr(X), _ptr(Y), bx, m, n, ldp, ldx, ldy, a, alpha,
-                                 _dtype_code(X), _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_poly_apply(_ptr(P), _ptr(X), _ptr(Y), bx, m, n, ldp, ldx, ldy, a, alpha,
+                                     _dtype_code(X), st))
 
 
 def dmuon_momentum(buf: torch.Tensor, grad: torch.Tensor, x0: torch.Tensor, momentum: float = 0.95,
                    nesterov: bool = True, sumsq: Optional[torch.Tensor] = None, stream=None) -> None:
     """buf <- mu buf + g ; x0 = g + mu buf (or buf); optional fp64 sum of squares of x0."""
-    _need_cuda(buf, grad, x0)
+    _out_word(sumsq, torch.float64, "sumsq")
+    dev = _device_of(buf, grad, x0, sumsq)
     if not (buf.shape == grad.shape == x0.shape) or buf.dim() != 2:
         raise ValueError("buf, grad and x0 must be 2D of one shape")
-    if sumsq is not None and (sumsq.dtype != torch.float64 or not sumsq.is_cuda):
-        raise ValueError("sumsq must be a CUDA float64 tensor")
-    _check(_lib.dmuon_momentum(_ptr(buf), _ptr(grad), _ptr(x0), buf.shape[0], buf.shape[1],
-                               momentum, int(bool(nesterov)), _dtype_code(buf), _ptr(sumsq),
-                               _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_momentum(_ptr(buf), _ptr(grad), _ptr(x0), buf.shape[0], buf.shape[1],
+                                   momentum, int(bool(nesterov)), _dtype_code(buf), _ptr(sumsq), st))
 
 
 def dmuon_update(param: torch.Tensor, O: torch.Tensor, lr: float, wd: float = 0.0,
                  stream=None) -> None:
     """param <- param (1 - lr wd) - lr 0.2 sqrt(max(m,n)) O."""
-    _need_cuda(param, O)
+    dev = _device_of(param, O)
     if param.shape != O.shape or param.dim() != 2 or param.dtype != O.dtype:
         raise ValueError("param and O must be 2D of one shape and dtype")
-    _check(_lib.dmuon_update(_ptr(param), _ptr(O), param.shape[0], param.shape[1], lr, wd,
-                             _dtype_code(param), _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_update(_ptr(param), _ptr(O), param.shape[0], param.shape[1], lr, wd,
+                                 _dtype_code(param), st))
 
 
 # ---------------------------------------------------------- status / misc
@@ -402,6 +451,16 @@ def dmuon_profile_stop() -> dict:
     return {arr[i].name.decode(): {"launches": int(arr[i].launches), "total_ms": arr[i].total_ms,
                                    "flops": arr[i].flops, "bytes": arr[i].bytes}
             for i in range(min(n, 32))}
+
+
+def dmuon_profile_stop_launches(max_records: int = 100000) -> list:
+    """[{name, start_ms, ms, flops, bytes}] for every launch since start, in enqueue order."""
+    arr = (LaunchRecord * max_records)()
+    n = _lib.dmuon_profile_stop_launches(arr, max_records)
+    if n < 0:
+        raise DmuonError(DMUON_ERR_CUDA, dmuon_get_last_error())
+    return [{"name": arr[i].name.decode(), "start_ms": arr[i].start_ms, "ms": arr[i].ms,
+             "flops": arr[i].flops, "bytes": arr[i].bytes} for i in range(min(n, max_records))]
 
 
 def dmuon_build_info() -> str:

@@ -112,6 +112,9 @@ bool fault_injected(const char* what) {
   const char* e = std::getenv("DMUON_FAULT_INJECT");
   return e && std::strcmp(e, what) == 0;
 }
+// DMUON_FAULT_INJECT=chain_wait: the fused chain's last dependency is never
+// met, so its bounded waits run out (for the failure-detection test)
+bool env_is_inject_chain() { return fault_injected("chain_wait"); }
 
 // Stream-ordered, grow-only workspace per (device, stream).
 dmuon_status_t get_workspace(size_t bytes, cudaStream_t st, void** out) {
@@ -205,11 +208,11 @@ bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
 
 // ------------------------------------------------------------ kernel timing
 enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
-            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kApplyUpdTc, kNumKinds };
+            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kApplyUpdTc, kChainTc, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
                                            "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
                                            "copy_out", "symm_tc", "chain_small", "clip_norm", "clip_scale",
-                                           "apply_update_tc"};
+                                           "apply_update_tc", "chain_tc"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -286,6 +289,25 @@ bool thin_chain(const ChunkLayout& L, int64_t m, int64_t n, int32_t steps) {
          n <= small_ns_max_n((int)m, L.path == Path::kSmallBf16 ? 2 : 4) && !env_is("DMUON_SMALL_CHAIN", '0');
 }
 
+// The tensor-path chain of a chunk runs as one persistent launch when its
+// products are small (tc_chain_small) and the chain can (tc_chain_fusable);
+// DMUON_FUSED_CHAIN=1 fuses every chain that can be fused, =0 none.
+bool fuse_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, int32_t steps) {
+  if (L.path != Path::kTensorBf16 || env_is("DMUON_FUSED_CHAIN", '0')) return false;
+  const std::vector<int> blocks = chain_blocks(L, steps);
+  if (!tc_chain_fusable((int)m, blocks)) return false;
+  return env_is("DMUON_FUSED_CHAIN", '1') || tc_chain_small(b, (int)m, (int)n, blocks);
+}
+
+// Executed flops of a tensor-path chain: gram m^2 n, symmetric products m^3,
+// applies 2 m^2 n per matrix (one triangle of every symmetric product).
+double chain_flops(const std::vector<int>& blocks, double m, double n) {
+  double f = 0.0;
+  for (int len : blocks)
+    f += m * m * n + (len == 1 ? 1.0 : (len == 2 ? 5.0 : 9.0)) * m * m * m + 2.0 * m * m * n;
+  return f;
+}
+
 // The tensor path ends with a tensor-core apply, whose epilogue can update
 // the parameters directly (DMUON_FUSED_UPDATE=0 keeps the separate pass).
 bool fuses_update(const ChunkLayout& L, int32_t steps) {
@@ -349,6 +371,26 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
     return DMUON_OK;
   }
 
+  // the whole chain in one persistent launch (same tiles, same epilogues, same bits)
+  if (tc && fuse_chain(L, b, m, n, steps)) {
+    const std::vector<int> blocks = chain_blocks(L, steps);
+    ChainBuffers cb{};
+    cb.x[0] = cur;
+    cb.x[1] = nxt;
+    for (int i = 0; i < L.gslots && i < 5; ++i) cb.slot[i] = slot(i);
+    cb.counters = reinterpret_cast<unsigned*>(ws + off.counters);
+    int rx = 0;
+    Prof p(kChainTc, st, fb * chain_flops(blocks, fm, fn), upd ? 4.0 * fb * fm * fn : 0.0);
+    e = tc_chain(cb, b, mi, ni, L.ldn, L.ldm, blocks, sched, scale, upd, sw, sms, env_is_inject_chain(), st, &rx);
+    p.done(st);
+    if (e == cudaSuccess) {
+      *result = rx < 0 ? nullptr : (rx == 0 ? cur : nxt);
+      return DMUON_OK;
+    }
+    if (e != cudaErrorNotSupported) return cuda_fail(e, "fused chain launch");
+    e = cudaSuccess;  // not fusable: the chain runs product by product below
+  }
+
   // Blocks of iterations (chain_blocks).  A block of one is the iteration as
   // written: G = X X^T, P = b G + c G G, X <- a X + P X.  In a longer block
   // every matrix is a polynomial of the block's Gram matrix G:
@@ -402,9 +444,10 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
 }
 
 // Kernels one chunk launches: momentum, norm, the chain, update (unless fused).
-int64_t chunk_launches_for(const ChunkLayout& L, int64_t m, int64_t n, int32_t steps) {
+int64_t chunk_launches_for(const ChunkLayout& L, int b, int64_t m, int64_t n, int32_t steps) {
   int64_t k = fuses_update(L, steps) ? 2 : 3;
   if (thin_chain(L, m, n, steps)) return k + 1;
+  if (fuse_chain(L, b, m, n, steps)) return k + 1;
   for (int len : chain_blocks(L, steps)) k += len == 1 ? 3 : (len == 2 ? 7 : 11);  // gram + products + apply
   return k;
 }
@@ -771,7 +814,7 @@ int64_t dmuon_step_launches(const dmuon_shape_t* shapes, int32_t count, int32_t 
   const StepPlan P = make_step_plan(shapes, count);
   int64_t n = 0;
   for (const ChunkRef& ck : P.chunks)
-    n += chunk_launches_for(P.layouts[ck.cls], P.classes[ck.cls].m, P.classes[ck.cls].n, ns_steps);
+    n += chunk_launches_for(P.layouts[ck.cls], ck.b, P.classes[ck.cls].m, P.classes[ck.cls].n, ns_steps);
   return n;
 }
 

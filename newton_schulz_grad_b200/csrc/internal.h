@@ -148,6 +148,30 @@ struct UpdTable {
 cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int n, int64_t ldp, int64_t ldx,
                             float a, float alpha, const float* scale, const UpdTable& u, int* status,
                             int num_sms, cudaStream_t st);
+// The whole chain of a chunk in one persistent launch (tensor path): every
+// product of the iteration blocks `blocks` (chain_blocks) in order, per-matrix
+// dependency counters between them.  x[0] holds X at entry; slot[0..4] are
+// the m x m buffers (slots 2-4 only for Gram-space blocks); counters has
+// batch + 1 entries (zeroed here: one per matrix, then the tile counter).  upd: the last apply updates the parameters.
+// *result_x: the x buffer holding the result (-1 when fused with the update).
+// cudaErrorNotSupported: this chain cannot run fused (too many products, or
+// its products would pick different CTA groupings); run it product by
+// product instead.  inject_timeout: a test hook whose last dependency is never
+// met, so its bounded waits run out (DMUON_ERR_TIMEOUT).
+struct ChainBuffers {
+  void* x[2];
+  void* slot[5];
+  unsigned* counters;
+};
+bool tc_chain_fusable(int m, const std::vector<int>& blocks);
+// True when the chain's products average at most two waves of tiles on a
+// B200 (74 CTA pairs or 148 CTAs): launched one by one they would be
+// dominated by launch, ramp-up and tail, so the fused launch pays off.  Large
+// chunks run one launch per product (measured faster there).
+bool tc_chain_small(int batch, int m, int n, const std::vector<int>& blocks);
+cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t ldn, int64_t ldm,
+                     const std::vector<int>& blocks, const float* sched, const float* scale, const UpdTable* upd,
+                     int* status, int num_sms, bool inject_timeout, cudaStream_t st, int* result_x);
 // decay = 1 - lr wd and step_scale = fl32(lr 0.2 sqrt(scale_dim)), each rounded
 // as the update kernels use them.
 void update_coeffs(float lr, float wd, int64_t scale_dim, float* decay, float* step_scale);
@@ -212,7 +236,7 @@ int64_t workspace_cap_bytes();
 int64_t chunk_size(const ChunkLayout& L, int64_t members, int64_t cap);
 // Offsets of the pieces of a chunk of `b` matrices inside the workspace.
 struct ChunkOffsets {
-  int64_t x0, x1, g, p, partials, scale, total;
+  int64_t x0, x1, g, p, partials, scale, counters, total;  // counters: fused-chain dependencies
 };
 ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b);
 

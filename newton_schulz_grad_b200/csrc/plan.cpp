@@ -87,7 +87,7 @@ ChunkLayout chunk_layout(int64_t m, int64_t n, int32_t dtype, bool allow_blocked
   L.xbytes = m * L.ldn * xs;
   L.gbytes = m * L.ldm * gs;
   L.tiles_per_mat = ((m + kElemTile - 1) / kElemTile) * ((n + kElemTile - 1) / kElemTile);
-  L.per_matrix = 2 * L.xbytes + L.gslots * L.gbytes + L.tiles_per_mat * 4 + 4 + 6 * 256;
+  L.per_matrix = 2 * L.xbytes + L.gslots * L.gbytes + L.tiles_per_mat * 4 + 8 + 7 * 256;
   return L;
 }
 
@@ -171,6 +171,7 @@ ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b) {
   o.p = at; at += round_up(b * L.gbytes, 256) * (L.gslots - 1);
   o.partials = at; at += round_up(b * L.tiles_per_mat * 4, 256);
   o.scale = at; at += round_up(b * 4, 256);
+  o.counters = at; at += round_up((b + 1) * 4, 256);  // one per matrix, then the tile counter
   o.total = at;
   return o;
 }

@@ -44,8 +44,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
+#include <memory>
 #include <mutex>
 
 #include "bounds.cuh"
@@ -352,6 +354,20 @@ __device__ __forceinline__ float half_of(const uint32_t* w, int j) {
   return __uint_as_float((j & 1) ? (x & 0xffff0000u) : (x << 16));
 }
 
+// Loads of the epilogue's E operand (b G, a X).  COH: the operand was written
+// earlier in the same kernel (the fused chain), so it is read through L2
+// (ld.global.cg), never from a possibly stale L1 line or the non-coherent
+// read-only path; otherwise through the read-only path.
+template <bool COH>
+__device__ __forceinline__ uint4 ld_e16(const __nv_bfloat16* p) {
+  return COH ? __ldcg(reinterpret_cast<const uint4*>(p)) : __ldg(reinterpret_cast<const uint4*>(p));
+}
+template <bool COH>
+__device__ __forceinline__ __nv_bfloat16 ld_e1(const __nv_bfloat16* p) {
+  return COH ? __ushort_as_bfloat16(__ldcg(reinterpret_cast<const unsigned short*>(p))) : *p;
+}
+
+template <bool COH>
 __device__ __forceinline__ void load_upd_chunk(const UpdTable& u, const TcArgs& a, int b, int r, int c0,
                                                UpdChunk& k) {
   const int m = a.m, n = a.n;
@@ -395,12 +411,12 @@ __device__ __forceinline__ void load_upd_chunk(const UpdTable& u, const TcArgs& 
       for (int j = 0; j < 16; ++j) k.e[j] = 0u;
     } else if (full) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(k.e)[i] = __ldg(reinterpret_cast<const uint4*>(ep) + i);
+      for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(k.e)[i] = ld_e16<COH>(ep + 8 * i);
     } else {
       const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
 #pragma unroll
       for (int j = 0; j < 32; j += 2)
-        k.e[j >> 1] = pack2((c0 + j < n) ? ep[j] : z, (c0 + j + 1 < n) ? ep[j + 1] : z);
+        k.e[j >> 1] = pack2((c0 + j < n) ? ld_e1<COH>(ep + j) : z, (c0 + j + 1 < n) ? ld_e1<COH>(ep + j + 1) : z);
     }
   }
 }
@@ -448,18 +464,19 @@ __device__ __forceinline__ void store_upd_chunk(const UpdTable& u, const TcArgs&
 }
 
 // Epilogue of one apply tile with the fused update (see epilogue_row).
+template <bool COH>
 __device__ __forceinline__ void epilogue_row_update(const TcArgs& a, const UpdTable& u, uint32_t taddr, int b,
                                                     int r, int J) {
   const bool row_ok = r < a.m;
   const float alpha = a.p1 * (a.scale ? a.scale[b] : 1.f);
   const int cbase = J * BN;
   UpdChunk k0, k1;
-  if (row_ok) load_upd_chunk(u, a, b, r, cbase, k0);
+  if (row_ok) load_upd_chunk<COH>(u, a, b, r, cbase, k0);
   // one chunk: load the next chunk's operands, then drain this one
   auto chunk = [&](int ch, const UpdChunk& cur, UpdChunk& nxt) -> bool {
     const int c0 = cbase + ch * 32;
     if (c0 >= a.n) return false;  // warp-uniform
-    if (row_ok && ch + 1 < BN / 32 && c0 + 32 < a.n) load_upd_chunk(u, a, b, r, c0 + 32, nxt);
+    if (row_ok && ch + 1 < BN / 32 && c0 + 32 < a.n) load_upd_chunk<COH>(u, a, b, r, c0 + 32, nxt);
     uint32_t raw[32];
     tmem_ld32(taddr + (uint32_t)(ch * 32), raw);
     tmem_ld_wait();
@@ -505,11 +522,11 @@ __device__ __forceinline__ void prefetch_update_tile(const UpdTable& u, int b, i
 // accumulator columns [col0, col0 + 256), output row r, output columns from
 // J * 256.  Warp-collective (tcgen05.ld).  UPD (apply only): update the
 // parameters instead of storing the result.
-template <int MODE, bool UPD>
+template <int MODE, bool UPD, bool COH = false>
 __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename UpdSel<UPD>::type& u, uint32_t taddr,
                                              int b, int r, int J) {
   if constexpr (UPD) {
-    epilogue_row_update(a, u, taddr, b, r, J);
+    epilogue_row_update<COH>(a, u, taddr, b, r, J);
     return;
   }
   const bool row_ok = r < a.m;
@@ -544,10 +561,10 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename Upd
         for (int j = 0; j < 32; ++j) e[j] = 0.f;
       } else if (full_chunk) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(ep) + q), e + 8 * q);
+        for (int q = 0; q < 4; ++q) unpack_bf16x8(ld_e16<COH>(ep + 8 * q), e + 8 * q);
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ep[j]) : 0.f;
+        for (int j = 0; j < 32; ++j) e[j] = (c0 + j < a.n) ? __bfloat162float(ld_e1<COH>(ep + j)) : 0.f;
       }
       if (MODE == kApply) {
 #pragma unroll
@@ -960,6 +977,424 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
+// ====================================================== fused chain kernel
+// One persistent launch for a chunk's whole Newton-Schulz chain.  The phases
+// (every gram, polynomial / Gram-space product and apply of the chain, in
+// order) form one tile list, phase by phase and matrix by matrix within a
+// phase.  A tile of phase j of matrix b needs every tile of phases < j of that
+// matrix: each epilogue warp, after its stores, adds 1 (release) to the
+// matrix's counter, and the TMA producer waits (acquire, bounded by
+// %globaltimer) until the counter holds 4 x CTAs-per-tile x (tiles of the
+// earlier phases) before it loads the tile's operands.
+//
+// Tiles are claimed in increasing order from one global counter (the
+// producer of each CTA, or of the pair's leader, takes the next index and
+// passes it to its MMA and epilogue warps, and to the peer CTA, through a
+// ring of 4 shared-memory slots).  Every dependency points to a lower index
+// and only running CTAs claim tiles, so the smallest unfinished tile always
+// has its inputs done and a running CTA to finish it, however many CTAs are
+// resident (other kernels, or a second chain on another stream, included).
+// The tail of one phase overlaps the head of the next for the matrices
+// already done, and the chain pays one launch instead of one per product.
+constexpr int kMaxPhases = 32;
+constexpr int kRing = 4;
+enum { kMapX0 = 0, kMapX1 = 1, kMapS0 = 2, kMapX0mn = 7, kMapX1mn = 8, kChainMaps = 9 };
+
+struct PhaseDesc {
+  TcArgs a;
+  int mode;        // kGram, kPoly (symmetric products) or kApply
+  int upd;         // apply whose epilogue updates the parameters
+  int mapA, mapB;  // tensor maps of the operands
+  int tile_start;  // global index of the phase's first tile
+  uint32_t dep;    // counter value (per matrix) the phase's tiles wait for
+};
+
+struct ChainParams {
+  CUtensorMap maps[kChainMaps];  // K-major {64 x 128} for X0, X1, S0..S4; MN-major {64 x 64} for X0, X1
+  PhaseDesc ph[kMaxPhases];
+  UpdTable u;
+  unsigned* counters;  // one per matrix, then the tile counter; all zero at launch
+  int* status;
+  uint64_t dep_limit_ns;
+  int nphases, total_tiles, batch;
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add(unsigned* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// orders this thread's generic-proxy accesses with its later async-proxy
+// (TMA) accesses of global memory
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+// store to the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (the slot was written by the peer CTA).
+__device__ __noinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, int* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 128; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(status) != 0) return false;
+    if (global_timer() - t0 > kTimeoutNs) {
+      atomicCAS(status, 0, (int)DMUON_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Bounded wait until *c >= target; false when the limit ran out (recorded as
+// DMUON_ERR_TIMEOUT) or another thread already failed.
+__device__ __noinline__ bool wait_count(const unsigned* c, uint32_t target, int* status, uint64_t limit_ns) {
+  if (ld_acquire_u32(c) >= target) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      if (ld_acquire_u32(c) >= target) return true;
+      __nanosleep(64);
+    }
+    if (*reinterpret_cast<volatile int*>(status) != 0) return false;
+    if (global_timer() - t0 > limit_ns) {
+      atomicCAS(status, 0, (int)DMUON_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ int find_phase(const ChainParams& P, int t) {
+  int j = 0;
+  while (j + 1 < P.nphases && t >= P.ph[j + 1].tile_start) ++j;
+  return j;
+}
+__device__ __forceinline__ void decode_phase_tile(const PhaseDesc& ph, int t, int& b, int& I, int& J) {
+  if (ph.mode == kApply)
+    decode_tile<kApply>(ph.a, t - ph.tile_start, b, I, J);
+  else
+    decode_tile<kGram>(ph.a, t - ph.tile_start, b, I, J);
+}
+
+// G = 1: one CTA, 128 x 256 tiles (cta_group::1); G = 2: CTA pair, 256 x 256
+// tiles (cta_group::2).  Both load K-major operands as boxes of 128 rows (the
+// one-CTA kernel's 256 B rows as two), so one set of tensor maps serves both.
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ ChainParams P) {
+  constexpr int STAGES = G == 2 ? STAGES2 : STAGES1;
+  constexpr int STAGE_BYTES = G == 2 ? STAGE2_BYTES : STAGE1_BYTES;
+  constexpr int A_BYTES = G == 2 ? A2_BYTES : A1_BYTES;
+  constexpr int TM = G == 2 ? BM2 : BM1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* qbars = bars + kBarriers;                        // ring: full[kRing], empty[kRing]
+  int* ring = reinterpret_cast<int*>(qbars + 2 * kRing);    // tile index per slot
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + kRing);
+  const Bars B = bar_layout(bars);
+  const uint32_t qfull0 = smem_u32(qbars), qempty0 = smem_u32(qbars + kRing);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = G == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  int* status = P.status;
+  unsigned* next_tile = P.counters + P.batch;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(B.full0 + 8 * s, 1);
+      mbar_init(B.empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(B.tfull0 + 8 * s, 1);
+      mbar_init(B.tempty0 + 8 * s, 4 * G);  // one arrival per epilogue warp (of both CTAs)
+    }
+    mbar_init(B.done, 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(qfull0 + 8 * s, 1);              // the leader's producer
+      mbar_init(qempty0 + 8 * s, G == 2 ? 10 : 5);  // MMA + 4 epilogue warps (+ peer producer + 4 warps)
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int i = 0; i < kChainMaps; ++i)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[i])) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc<G>(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish<G>();
+  }
+  tc_fence_before();
+  if (G == 2)
+    cluster_sync();
+  else
+    __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // the leader's ring-empty barriers (every consumer of both CTAs arrives there)
+  const uint32_t qempty_leader0 = G == 2 ? mapa_shared(qempty0, 0) : qempty0;
+  // next tile of the ring for a consumer: wait for the slot, read it, free it
+  auto take = [&](int& qs, uint32_t& qph, bool remote_writer) -> int {
+    const bool ok = remote_writer ? wait_bar_cluster(qfull0 + 8 * qs, qph, status)
+                                  : wait_bar(qfull0 + 8 * qs, qph, status);
+    const int t = ok ? *reinterpret_cast<volatile int*>(ring + qs) : -1;
+    return t;
+  };
+  auto release = [&](int qs) {
+    if (G == 2)
+      mbar_arrive_cluster(qempty_leader0 + 8 * qs);
+    else
+      mbar_arrive(qempty0 + 8 * qs);
+  };
+  auto advance = [](int& qs, uint32_t& qph) {
+    if (++qs == kRing) {
+      qs = 0;
+      qph ^= 1u;
+    }
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      const uint32_t full_base = G == 2 ? mapa_shared(B.full0, 0) : B.full0;
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      int qs = 0;
+      uint32_t qph = 0;
+      bool ok = true;
+      while (ok) {
+        int t;
+        if (leader) {
+          // claim the next tile and publish it to this CTA (and the peer)
+          // (every consumer has read this slot; the peer's arrivals are remote)
+          const bool free = G == 2 ? wait_bar_cluster(qempty0 + 8 * qs, qph ^ 1u, status)
+                                   : wait_bar(qempty0 + 8 * qs, qph ^ 1u, status);
+          if (!free) break;
+          t = (int)atomicAdd(next_tile, 1u);
+          if (t >= P.total_tiles) t = -1;
+          ring[qs] = t;
+          if (G == 2) st_cluster_u32(mapa_shared(smem_u32(ring + qs), 1), (uint32_t)t);
+          mbar_arrive(qfull0 + 8 * qs);
+          if (G == 2) mbar_arrive_cluster(mapa_shared(qfull0 + 8 * qs, 1));
+        } else {
+          t = take(qs, qph, true);
+          release(qs);
+        }
+        advance(qs, qph);
+        if (t < 0) break;
+        const PhaseDesc& ph = P.ph[find_phase(P, t)];
+        int b, I, J;
+        decode_phase_tile(ph, t, b, I, J);
+        if (ph.dep != 0) {
+          if (!wait_count(P.counters + b, ph.dep, status, P.dep_limit_ns)) break;
+          fence_proxy_async_global();  // the operands were written by generic stores
+        }
+        const CUtensorMap* mA = &P.maps[ph.mapA];
+        const CUtensorMap* mB = &P.maps[ph.mapB];
+        const int num_kb = (ph.a.k + BK - 1) / BK;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(B.full0 + 8 * stage, G * STAGE_BYTES);
+          const uint32_t fb = full_base + 8 * stage;
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          if constexpr (G == 2) {
+            tma_load_3d_pair(sa, mA, fb, kb * BK, I * TM + (int)rank * 128, b);
+            if (ph.mode == kApply) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                tma_load_3d_pair(sb + q * 8192, mB, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d_pair(sb, mB, fb, kb * BK, J * BN + (int)rank * 128, b);
+            }
+          } else {
+            tma_load_3d(sa, mA, fb, kb * BK, I * TM, b);
+            if (ph.mode == kApply) {
+#pragma unroll
+              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mB, fb, J * BN + q * 64, kb * BK, b);
+            } else {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) tma_load_3d(sb + h * 16384, mB, fb, kb * BK, J * BN + h * 128, b);
+            }
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (leader) {
+        const int64_t first = issued > STAGES ? issued - STAGES : 0;
+        for (int64_t i = first; i < issued; ++i) {
+          if (!wait_bar(B.full0 + 8 * (int)(i % STAGES), (uint32_t)((i / STAGES) & 1), status)) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ----------------------------------------------------------------- MMA
+      constexpr uint32_t idesc_k = make_idesc(false, TM);
+      constexpr uint32_t idesc_mn = make_idesc(true, TM);
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t b_desc0_k = sdesc_sw128(smem_u32(smem) + A_BYTES, 16, 1024);
+      const uint64_t b_desc0_mn = sdesc_sw128(smem_u32(smem) + A_BYTES, 8192, 1024);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      int qs = 0;
+      uint32_t qph = 0;
+      bool ok = true;
+      while (ok) {
+        const int t = take(qs, qph, false);
+        release(qs);
+        advance(qs, qph);
+        if (t < 0) break;
+        const PhaseDesc& ph = P.ph[find_phase(P, t)];
+        const bool mn = ph.mode == kApply;
+        const uint32_t idesc = mn ? idesc_mn : idesc_k;
+        const uint64_t b_desc0 = mn ? b_desc0_mn : b_desc0_k;
+        const uint64_t b_step = mn ? (uint64_t)(UK * 128 / 16) : (uint64_t)(UK * 2 / 16);
+        const int num_kb = (ph.a.k + BK - 1) / BK;
+        if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bar(B.full0 + 8 * stage, phase, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t soff = (uint64_t)((stage * STAGE_BYTES) >> 4);
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k)
+            tc_mma<G>(d, a_desc0 + soff + (uint64_t)(k * (UK * 2 / 16)), b_desc0 + soff + (uint64_t)k * b_step, idesc,
+                      (kb | k) != 0 ? 1u : 0u);
+          if constexpr (G == 2)
+            tc_commit_pair(B.empty0 + 8 * stage, 0x3);
+          else
+            tc_commit<1>(B.empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if constexpr (G == 2)
+          tc_commit_pair(B.tfull0 + 8 * acc, 0x3);
+        else
+          tc_commit<1>(B.tfull0 + 8 * acc);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit<G>(B.done);
+      wait_bar(B.done, 0, status);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int wq = warp & 3;
+    const uint32_t tempty0 = G == 2 ? mapa_shared(B.tempty0, 0) : B.tempty0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int qs = 0;
+    uint32_t qph = 0;
+    int t = take(qs, qph, G == 2 && !leader);
+    __syncwarp();
+    if (lane == 0) release(qs);
+    advance(qs, qph);
+    bool prefetched = false;  // t's update parameters were already pulled into L2
+    while (t >= 0) {
+      const PhaseDesc& ph = P.ph[find_phase(P, t)];
+      int b, I, J;
+      decode_phase_tile(ph, t, b, I, J);
+      const int r0 = I * TM + (int)rank * 128 + wq * 32;
+      // the next tile (claimed ahead by the producer): its update parameters
+      // are pulled into L2 while this tile drains
+      const int tn = take(qs, qph, G == 2 && !leader);
+      __syncwarp();
+      if (lane == 0) release(qs);
+      advance(qs, qph);
+      bool next_prefetched = false;
+      if (ph.upd) {
+        if (!prefetched) prefetch_update_tile(P.u, b, r0, J * BN, ph.a.m, ph.a.n, lane);
+        if (tn >= 0) {
+          const PhaseDesc& pn = P.ph[find_phase(P, tn)];
+          if (pn.upd) {
+            int b2, I2, J2;
+            decode_phase_tile(pn, tn, b2, I2, J2);
+            prefetch_update_tile(P.u, b2, I2 * TM + (int)rank * 128 + wq * 32, J2 * BN, pn.a.m, pn.a.n, lane);
+            next_prefetched = true;
+          }
+        }
+      }
+      prefetched = next_prefetched;
+      if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN);
+      const NoUpd none{};
+      // a local copy: read from the indexed parameter table, the arguments would
+      // be reloaded after every store of the epilogue (which might alias them)
+      const TcArgs a = ph.a;
+      if (ph.upd)
+        epilogue_row<kApply, true, true>(a, P.u, taddr, b, r0 + lane, J);
+      else if (ph.mode == kApply)
+        epilogue_row<kApply, false, true>(a, none, taddr, b, r0 + lane, J);
+      else if (ph.mode == kPoly)
+        epilogue_row<kPoly, false, true>(a, none, taddr, b, r0 + lane, J);
+      else
+        epilogue_row<kGram, false, true>(a, none, taddr, b, r0 + lane, J);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        // this warp's part of the tile is stored: publish it, then free the accumulator
+        red_release_add(P.counters + b, 1u);  // release: after the warp's stores (ordered by the __syncwarp)
+        if constexpr (G == 2)
+          mbar_arrive_cluster(tempty0 + 8 * acc);
+        else
+          mbar_arrive(tempty0 + 8 * acc);
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      t = tn;
+    }
+  }
+  tc_fence_before();
+  if (G == 2)
+    cluster_sync();
+  else
+    __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<G>(tmem_base, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
@@ -1030,6 +1465,45 @@ bool use_pair(int m, bool triangle) {
   return one_area * kOneCtaCost >= pair_area;
 }
 
+// Largest number of CTA pairs (clusters of 2 at the pair kernels' shared
+// memory) that can be resident at once on the current device: SMs / 2 unless
+// the GPCs leave some SMs unpaired.  Persistent pair launches use no more,
+// so no pair starts only after others finish, and the fused chain (whose CTAs
+// wait on one another) relies on it.
+int max_pair_units(int num_sms) {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return num_sms / 2;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] > 0) return cached[dev];
+  int n = 0;
+  cudaError_t e = cudaFuncSetAttribute(k_chain<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(num_sms & ~1));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&n, (void*)k_chain<2>, &cfg);
+  }
+  if (e != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms / 2;
+  }
+  cached[dev] = n < num_sms / 2 ? n : num_sms / 2;
+  return cached[dev];
+}
+
 template <int MODE, bool UPD = false>
 cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms, bool pair,
                    cudaStream_t st, const typename UpdSel<UPD>::type& u = {}) {
@@ -1046,13 +1520,81 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int 
   if (total > 0x7fffffff) return cudaErrorInvalidValue;
   a.total_tiles = (int)total;
   if (pair) {
-    const int64_t pairs = total < num_sms / 2 ? total : num_sms / 2;
+    const int units = max_pair_units(num_sms);
+    const int64_t pairs = total < units ? total : units;
     k_tc2<MODE, UPD><<<(int)(2 * pairs), kThreads, SMEM2_BYTES, st>>>(ma, mb, a, u);
   } else {
     const int grid = (int)(total < num_sms ? total : num_sms);
     k_tc<MODE, UPD><<<grid, kThreads, SMEM1_BYTES, st>>>(ma, mb, a, u);
   }
   return cudaGetLastError();
+}
+
+// Arguments of each product; the per-product launches and the fused chain
+// build them the same way, so both compute the same tiles with the same
+// epilogues.
+TcArgs gram_args(void* G, int batch, int m, int n, int64_t ldg, float alpha, const float* scale, int* status,
+                 bool pair) {
+  TcArgs a{};
+  a.C = static_cast<__nv_bfloat16*>(G);
+  a.E = nullptr;
+  a.sC = (int64_t)m * ldg;
+  a.ldc = ldg;
+  a.m = m; a.n = m; a.k = n;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
+  a.tiles_n = (m + BN - 1) / BN;
+  a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
+  a.total_tiles = a.tiles_per_mat * batch;
+  a.p0 = alpha;
+  a.scale = scale;
+  a.status = status;
+  return a;
+}
+
+TcArgs symm_args(const void* E, void* C, int batch, int m, int64_t lde, int64_t ldc, float p0, float p1, float p2,
+                 int* status, bool pair) {
+  TcArgs a{};
+  a.C = static_cast<__nv_bfloat16*>(C);
+  a.E = static_cast<const __nv_bfloat16*>(E);
+  a.sC = (int64_t)m * ldc;
+  a.sE = (int64_t)m * lde;
+  a.ldc = ldc;
+  a.lde = lde;
+  a.m = m; a.n = m; a.k = m;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
+  a.tiles_n = (m + BN - 1) / BN;
+  a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
+  a.total_tiles = a.tiles_per_mat * batch;
+  a.p0 = p0;
+  a.p1 = p1;
+  a.p2 = p2;
+  a.status = status;
+  return a;
+}
+
+// Y may be NULL (the fused update stores nothing but the parameters).
+TcArgs apply_args(const void* X, void* Y, int batch, int m, int n, int64_t ldx, int64_t ldy, float a_coef,
+                  float alpha, const float* scale, int* status, bool pair) {
+  TcArgs a{};
+  a.C = static_cast<__nv_bfloat16*>(Y);
+  a.E = static_cast<const __nv_bfloat16*>(X);
+  a.sC = Y ? (int64_t)m * ldy : 0;
+  a.sE = (int64_t)m * ldx;
+  a.ldc = Y ? ldy : 0;
+  a.lde = ldx;
+  a.m = m; a.n = n; a.k = m;
+  a.tm = pair ? BM2 : BM1;
+  a.tiles_m = (m + a.tm - 1) / a.tm;
+  a.tiles_n = (n + BN - 1) / BN;
+  a.tiles_per_mat = a.tiles_m * a.tiles_n;
+  a.total_tiles = a.tiles_per_mat * batch;
+  a.p0 = a_coef;
+  a.p1 = alpha;
+  a.scale = scale;
+  a.status = status;
+  return a;
 }
 
 }  // namespace
@@ -1066,19 +1608,7 @@ cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx
   cudaError_t e = make_map(&ma, X, n, m, batch, ldx, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, BK, pair ? 128 : BN);
   if (e != cudaSuccess) return e;
-  TcArgs a{};
-  a.C = static_cast<__nv_bfloat16*>(G);
-  a.E = nullptr;
-  a.sC = (int64_t)m * ldg;
-  a.ldc = ldg;
-  a.m = m; a.n = m; a.k = n;
-  a.tm = pair ? BM2 : BM1;
-  a.tiles_m = (m + a.tm - 1) / a.tm;
-  a.tiles_n = (m + BN - 1) / BN;
-  a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
-  a.p0 = alpha;
-  a.scale = scale;
-  a.status = status;
+  TcArgs a = gram_args(G, batch, m, n, ldg, alpha, scale, status, pair);
   return launch<kGram>(ma, mb, a, batch, num_sms, pair, st);
 }
 
@@ -1091,22 +1621,7 @@ cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int ba
   cudaError_t e = make_map(&ma, A, m, m, batch, lda, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, B, m, m, batch, ldb, BK, pair ? 128 : BN);
   if (e != cudaSuccess) return e;
-  TcArgs a{};
-  a.C = static_cast<__nv_bfloat16*>(C);
-  a.E = static_cast<const __nv_bfloat16*>(E);
-  a.sC = (int64_t)m * ldc;
-  a.sE = (int64_t)m * lde;
-  a.ldc = ldc;
-  a.lde = lde;
-  a.m = m; a.n = m; a.k = m;
-  a.tm = pair ? BM2 : BM1;
-  a.tiles_m = (m + a.tm - 1) / a.tm;
-  a.tiles_n = (m + BN - 1) / BN;
-  a.tiles_per_mat = tri_tiles(a.tiles_m, a.tiles_n, a.tm);
-  a.p0 = p0;
-  a.p1 = p1;
-  a.p2 = p2;
-  a.status = status;
+  TcArgs a = symm_args(E, C, batch, m, lde, ldc, p0, p1, p2, status, pair);
   return launch<kPoly>(ma, mb, a, batch, num_sms, pair, st);
 }
 
@@ -1124,22 +1639,7 @@ cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, in
   cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
   if (e != cudaSuccess) return e;
-  TcArgs a{};
-  a.C = static_cast<__nv_bfloat16*>(Y);
-  a.E = static_cast<const __nv_bfloat16*>(X);
-  a.sC = (int64_t)m * ldy;
-  a.sE = (int64_t)m * ldx;
-  a.ldc = ldy;
-  a.lde = ldx;
-  a.m = m; a.n = n; a.k = m;
-  a.tm = pair ? BM2 : BM1;
-  a.tiles_m = (m + a.tm - 1) / a.tm;
-  a.tiles_n = (n + BN - 1) / BN;
-  a.tiles_per_mat = a.tiles_m * a.tiles_n;
-  a.p0 = a_coef;
-  a.p1 = alpha;
-  a.scale = scale;
-  a.status = status;
+  TcArgs a = apply_args(X, Y, batch, m, n, ldx, ldy, a_coef, alpha, scale, status, pair);
   return launch<kApply>(ma, mb, a, batch, num_sms, pair, st);
 }
 
@@ -1153,21 +1653,155 @@ cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int 
   cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
   if (e != cudaSuccess) return e;
-  TcArgs a{};
-  a.C = nullptr;  // nothing stored but the parameters
-  a.E = static_cast<const __nv_bfloat16*>(X);
-  a.sE = (int64_t)m * ldx;
-  a.lde = ldx;
-  a.m = m; a.n = n; a.k = m;
-  a.tm = pair ? BM2 : BM1;
-  a.tiles_m = (m + a.tm - 1) / a.tm;
-  a.tiles_n = (n + BN - 1) / BN;
-  a.tiles_per_mat = a.tiles_m * a.tiles_n;
-  a.p0 = a_coef;
-  a.p1 = alpha;
-  a.scale = scale;
-  a.status = status;
+  TcArgs a = apply_args(X, nullptr, batch, m, n, ldx, 0, a_coef, alpha, scale, status, pair);
   return launch<kApply, true>(ma, mb, a, batch, num_sms, pair, st, u);
+}
+
+bool tc_chain_fusable(int m, const std::vector<int>& blocks) {
+  int nph = 0;
+  for (int len : blocks) nph += len == 1 ? 3 : (len == 2 ? 7 : 11);
+  return nph > 0 && nph <= kMaxPhases && use_pair(m, true) == use_pair(m, false);
+}
+
+bool tc_chain_small(int batch, int m, int n, const std::vector<int>& blocks) {
+  // tiles of each product kind for this chunk (the grouping the chain uses)
+  const bool pair = use_pair(m, false);
+  const TcArgs g = gram_args(nullptr, batch, m, n, m, 1.f, nullptr, nullptr, pair);
+  const TcArgs sy = symm_args(nullptr, nullptr, batch, m, m, m, 0.f, 1.f, 0.f, nullptr, pair);
+  const TcArgs ap = apply_args(nullptr, nullptr, batch, m, n, n, n, 0.f, 1.f, nullptr, nullptr, pair);
+  int64_t tiles = 0, nph = 0;
+  for (int len : blocks) {
+    const int products = len == 1 ? 1 : (len == 2 ? 5 : 9);
+    tiles += g.total_tiles + (int64_t)products * sy.total_tiles + ap.total_tiles;
+    nph += 2 + products;
+  }
+  // B200: 74 CTA pairs or 148 CTAs
+  const int64_t units = pair ? 74 : 148;
+  return nph > 0 && tiles <= 2 * units * nph;
+}
+
+cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t ldn, int64_t ldm,
+                     const std::vector<int>& blocks, const float* sched, const float* scale, const UpdTable* upd,
+                     int* status, int num_sms, bool inject_timeout, cudaStream_t st, int* result_x) {
+  *result_x = 0;
+  if (batch == 0) return cudaSuccess;
+  // one CTA grouping for every product, the one the per-product launches
+  // would pick for each of them (so both schedules give the same bits)
+  const bool pair = use_pair(m, false);
+  if (!tc_chain_fusable(m, blocks) || batch > kMaxTable || !buf.counters) return cudaErrorNotSupported;
+  const bool blocked = false == std::all_of(blocks.begin(), blocks.end(), [](int l) { return l == 1; });
+  if (blocked && !(buf.slot[2] && buf.slot[3] && buf.slot[4])) return cudaErrorNotSupported;
+  const int G = pair ? 2 : 1;
+
+  std::unique_ptr<ChainParams> P(new ChainParams());
+  cudaError_t e = make_map(&P->maps[kMapX0], buf.x[0], n, m, batch, ldn, BK, 128);
+  if (e == cudaSuccess) e = make_map(&P->maps[kMapX1], buf.x[1], n, m, batch, ldn, BK, 128);
+  for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+    e = make_map(&P->maps[kMapS0 + i], buf.slot[i] ? buf.slot[i] : buf.slot[0], m, m, batch, ldm, BK, 128);
+  if (e == cudaSuccess) e = make_map(&P->maps[kMapX0mn], buf.x[0], n, m, batch, ldn, 64, BK);
+  if (e == cudaSuccess) e = make_map(&P->maps[kMapX1mn], buf.x[1], n, m, batch, ldn, 64, BK);
+  if (e != cudaSuccess) return e;
+
+  int j = 0;
+  int64_t tiles = 0, per_matrix = 0;
+  auto add = [&](const TcArgs& a, int mode, int mapA, int mapB, int u) {
+    PhaseDesc& ph = P->ph[j++];
+    ph.a = a;
+    ph.mode = mode;
+    ph.upd = u;
+    ph.mapA = mapA;
+    ph.mapB = mapB;
+    ph.tile_start = (int)tiles;
+    ph.dep = (uint32_t)(4 * G * per_matrix);  // every epilogue warp of every CTA of a tile adds 1
+    tiles += a.total_tiles;
+    per_matrix += a.tiles_per_mat;
+  };
+  int steps = 0;
+  for (int len : blocks) steps += len;
+  auto S = [&](int i) { return buf.slot[i]; };
+  int cur = 0, k = 0;
+  for (int len : blocks) {
+    const float* sc = k == 0 ? scale : nullptr;
+    const bool last = k + len == steps;
+    const bool fuse = last && upd != nullptr;
+    const float* c = sched + 3 * k;
+    if (len == 1) {
+      add(gram_args(S(0), batch, m, n, ldm, 1.f, sc, status, pair), kGram, kMapX0 + cur, kMapX0 + cur, 0);
+      add(symm_args(S(0), S(1), batch, m, ldm, ldm, c[1], c[2], 0.f, status, pair), kPoly, kMapS0, kMapS0, 0);
+      add(apply_args(buf.x[cur], fuse ? nullptr : buf.x[1 - cur], batch, m, n, ldn, ldn, c[0], 1.f, sc, status, pair),
+          kApply, kMapS0 + 1, kMapX0mn + cur, fuse ? 1 : 0);
+    } else {
+      const float* c1 = sched + 3 * (k + 1);
+      add(gram_args(S(0), batch, m, n, ldm, 1.f, sc, status, pair), kGram, kMapX0 + cur, kMapX0 + cur, 0);
+      add(symm_args(S(0), S(1), batch, m, ldm, ldm, c[1], c[2], c[0], status, pair), kPoly, kMapS0, kMapS0, 0);  // P0
+      add(symm_args(nullptr, S(2), batch, m, ldm, ldm, 0.f, 1.f, 0.f, status, pair), kPoly, kMapS0 + 1, kMapS0, 0);  // T = P0 G
+      add(symm_args(nullptr, S(0), batch, m, ldm, ldm, 0.f, 1.f, 0.f, status, pair), kPoly, kMapS0 + 2, kMapS0 + 1,
+          0);  // G1 = T P0
+      add(symm_args(S(0), S(3), batch, m, ldm, ldm, c1[1], c1[2], c1[0], status, pair), kPoly, kMapS0, kMapS0, 0);  // P1
+      add(symm_args(nullptr, S(4), batch, m, ldm, ldm, 0.f, 1.f, 0.f, status, pair), kPoly, kMapS0 + 3, kMapS0 + 1,
+          0);  // Q = P1 P0
+      int q = 4;
+      if (len == 3) {
+        const float* c2 = sched + 3 * (k + 2);
+        add(symm_args(nullptr, S(2), batch, m, ldm, ldm, 0.f, 1.f, 0.f, status, pair), kPoly, kMapS0 + 3, kMapS0,
+            0);  // T = P1 G1
+        add(symm_args(nullptr, S(0), batch, m, ldm, ldm, 0.f, 1.f, 0.f, status, pair), kPoly, kMapS0 + 2, kMapS0 + 3,
+            0);  // G2 = T P1
+        add(symm_args(S(0), S(1), batch, m, ldm, ldm, c2[1], c2[2], c2[0], status, pair), kPoly, kMapS0, kMapS0,
+            0);  // P2
+        add(symm_args(nullptr, S(2), batch, m, ldm, ldm, 0.f, 1.f, 0.f, status, pair), kPoly, kMapS0 + 1, kMapS0 + 4,
+            0);  // Q2 = P2 Q
+        q = 2;
+      }
+      add(apply_args(buf.x[cur], fuse ? nullptr : buf.x[1 - cur], batch, m, n, ldn, ldn, 0.f, 1.f, sc, status, pair),
+          kApply, kMapS0 + q, kMapX0mn + cur, fuse ? 1 : 0);  // X <- Q X
+    }
+    cur = 1 - cur;
+    k += len;
+  }
+  if (tiles <= 0) return cudaSuccess;
+  if (tiles > 0x7fffffff) return cudaErrorNotSupported;
+  P->nphases = j;
+  P->total_tiles = (int)tiles;
+  P->counters = buf.counters;
+  P->batch = batch;
+  P->status = status;
+  P->dep_limit_ns = kTimeoutNs;
+  if (inject_timeout) {
+    // a dependency nothing will meet: the last phase's waits run out
+    P->ph[j - 1].dep += 1;
+    P->dep_limit_ns = 20000000ull;
+  }
+  if (upd) P->u = *upd;
+  *result_x = (upd != nullptr) ? -1 : cur;
+
+  e = cudaMemsetAsync(buf.counters, 0, (size_t)(batch + 1) * sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_chain<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(k_chain<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int max_units = pair ? max_pair_units(num_sms) : num_sms;
+  const int units = (int)(tiles < max_units ? tiles : max_units);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(G * units));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = pair ? SMEM2_BYTES : SMEM1_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = pair ? 2 : 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pair ? 1 : 0;
+  e = pair ? cudaLaunchKernelEx(&cfg, k_chain<2>, *P) : cudaLaunchKernelEx(&cfg, k_chain<1>, *P);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 cudaError_t wait_selftest(int* status, int64_t limit_us, cudaStream_t st) {

@@ -66,7 +66,8 @@ def test_launch_count_and_workspace_llama7b():
     # overlapped execution with two buffers of half the 8 GiB cap: 5 chunks of
     # <= 26 and 8 chunks of 12.  Per chunk: momentum + norm (the update runs in
     # the last apply's epilogue), plus 3 per single iteration and gram + 5
-    # products + apply for the block of two.
+    # products + apply for the block of two (chunks this large run one launch
+    # per product)
     assert nsg.dmuon_step_launches(shapes, 5) == 5 * (2 + 15) + 8 * (2 + 9 + 7)
     os.environ["DMUON_GRAM_BLOCKS"] = "2"
     try:  # blocks of 2 and 3: gram + 5 products + apply, gram + 9 products + apply
@@ -80,6 +81,33 @@ def test_launch_count_and_workspace_llama7b():
         del os.environ["DMUON_FUSED_UPDATE"]
     ws = nsg.dmuon_workspace_bytes(shapes, 5)
     assert 5 << 30 < ws <= 8 << 30
+
+
+def test_launch_count_fused_chains(monkeypatch):
+    # small chunks fuse their whole chain into one launch; DMUON_FUSED_CHAIN=1
+    # fuses every chain that can be (blocks of 2 and 3, 18 products, included),
+    # =0 none
+    w = workloads.get("small_layer_bf16")
+    small = [(r, c, 1) for r, c in w.shapes]
+    assert nsg.dmuon_step_launches(small, 5) == 3 * (2 + 1)  # three classes, one chunk each
+    monkeypatch.setenv("DMUON_FUSED_CHAIN", "0")
+    assert nsg.dmuon_step_launches(small, 5) == (2 + 15) + 2 * (2 + 9 + 7)  # 1024^2; 256x1024 and 1024x2816 with the tail
+    w = workloads.get("llama_7b_bf16")
+    shapes = [(r, c, 1) for r, c in w.shapes]
+    monkeypatch.setenv("DMUON_FUSED_CHAIN", "1")
+    assert nsg.dmuon_step_launches(shapes, 5) == 13 * (2 + 1)
+    monkeypatch.setenv("DMUON_GRAM_BLOCKS", "2")
+    assert nsg.dmuon_step_launches(shapes, 5) == 13 * (2 + 1)
+
+
+def test_fused_chain_falls_back_where_products_disagree(monkeypatch):
+    # m = 2100: the triangle products would take the one-CTA kernel and the
+    # apply the CTA pair, so the chain runs product by product (same bits as
+    # before); the per-iteration limit of the fused launch is 32 products
+    assert nsg.dmuon_step_launches([(2100, 2100, 1)], 5) == 2 + 15
+    assert nsg.dmuon_step_launches([(2048, 2048, 1)], 5) == 2 + 1
+    assert nsg.dmuon_step_launches([(2048, 2048, 1)], 10) == 2 + 1
+    assert nsg.dmuon_step_launches([(2048, 2048, 1)], 11) == 2 + 33
 
 
 def test_overlap_can_be_disabled(monkeypatch):

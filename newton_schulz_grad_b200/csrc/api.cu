@@ -208,11 +208,12 @@ bool dtype_ok(int32_t d) { return d == DMUON_F32 || d == DMUON_BF16; }
 
 // ------------------------------------------------------------ kernel timing
 enum Kind { kMomentum, kNorm, kGramTc, kPolyTc, kApplyTc, kGramFfma, kPolyFfma, kApplyFfma, kUpdate,
-            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kApplyUpdTc, kChainTc, kNumKinds };
+            kLoad, kCopyOut, kSymmTc, kChainSmall, kClipNorm, kClipScale, kApplyUpdTc, kChainTc, kChainFfma,
+            kNumKinds };
 const char* const kKindNames[kNumKinds] = {"momentum", "norm", "gram_tc", "poly_tc", "apply_tc",
                                            "gram_ffma", "poly_ffma", "apply_ffma", "update", "load",
                                            "copy_out", "symm_tc", "chain_small", "clip_norm", "clip_scale",
-                                           "apply_update_tc", "chain_tc"};
+                                           "apply_update_tc", "chain_tc", "chain_ffma"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -220,6 +221,9 @@ struct ProfRec {
 };
 thread_local bool g_prof_on = false;
 thread_local std::vector<ProfRec> g_prof;
+// Event pairs reused from one profiling window to the next, so that a window
+// whose launches were seen before creates no events (only records them).
+thread_local std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
 
 // Brackets one kernel launch with events when profiling is on.
 struct Prof {
@@ -228,9 +232,21 @@ struct Prof {
   Prof(int kind, cudaStream_t st, double flops, double bytes) : on(g_prof_on) {
     if (!on) return;
     r = ProfRec{kind, nullptr, nullptr, flops, bytes};
-    if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
-      on = false;
-      return;
+    const size_t i = g_prof.size();
+    if (i < g_prof_pool.size()) {
+      r.a = g_prof_pool[i].first;
+      r.b = g_prof_pool[i].second;
+    } else {
+      if (cudaEventCreate(&r.a) != cudaSuccess) {
+        on = false;
+        return;
+      }
+      if (cudaEventCreate(&r.b) != cudaSuccess) {
+        cudaEventDestroy(r.a);
+        on = false;
+        return;
+      }
+      g_prof_pool.emplace_back(r.a, r.b);
     }
     cudaEventRecord(r.a, st);
   }
@@ -292,6 +308,12 @@ bool thin_chain(const ChunkLayout& L, int64_t m, int64_t n, int32_t steps) {
 // The tensor-path chain of a chunk runs as one persistent launch when its
 // products are small (tc_chain_small) and the chain can (tc_chain_fusable);
 // DMUON_FUSED_CHAIN=1 fuses every chain that can be fused, =0 none.
+// FFMA chains always fuse (their products are small: a few dozen tiles per
+// launch otherwise), up to 16 iterations, unless DMUON_FUSED_CHAIN=0.
+bool fuse_ffma_chain(const ChunkLayout& L, int32_t steps) {
+  return L.path != Path::kTensorBf16 && steps >= 1 && steps <= 16 && !env_is("DMUON_FUSED_CHAIN", '0');
+}
+
 bool fuse_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, int32_t steps) {
   if (L.path != Path::kTensorBf16 || env_is("DMUON_FUSED_CHAIN", '0')) return false;
   const std::vector<int> blocks = chain_blocks(L, steps);
@@ -371,6 +393,23 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
     return DMUON_OK;
   }
 
+  // FFMA chains (fp32, small near-square bf16, thin bf16 beyond the clustered
+  // kernel): every product in one launch (same tiles, same arithmetic, same bits)
+  if (!tc && fuse_ffma_chain(L, steps)) {
+    void* xs[2] = {cur, nxt};
+    int rx = 0;
+    Prof p(kChainFfma, st, fb * (3.0 * fm * fm * fn + fm * fm * fm) * steps, 0.0);
+    e = simt_chain(xs, G, P, b, mi, ni, L.ldn, L.ldm, steps, sched, scale, xbf16,
+                   reinterpret_cast<unsigned*>(ws + off.counters), sw, sms, env_is_inject_chain(), st, &rx);
+    p.done(st);
+    if (e == cudaSuccess) {
+      *result = rx == 0 ? cur : nxt;
+      return DMUON_OK;
+    }
+    if (e != cudaErrorNotSupported) return cuda_fail(e, "fused FFMA chain launch");
+    e = cudaSuccess;  // too many iterations: product by product below
+  }
+
   // the whole chain in one persistent launch (same tiles, same epilogues, same bits)
   if (tc && fuse_chain(L, b, m, n, steps)) {
     const std::vector<int> blocks = chain_blocks(L, steps);
@@ -447,7 +486,7 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
 int64_t chunk_launches_for(const ChunkLayout& L, int b, int64_t m, int64_t n, int32_t steps) {
   int64_t k = fuses_update(L, steps) ? 2 : 3;
   if (thin_chain(L, m, n, steps)) return k + 1;
-  if (fuse_chain(L, b, m, n, steps)) return k + 1;
+  if (fuse_ffma_chain(L, steps) || fuse_chain(L, b, m, n, steps)) return k + 1;
   for (int len : chain_blocks(L, steps)) k += len == 1 ? 3 : (len == 2 ? 7 : 11);  // gram + products + apply
   return k;
 }
@@ -1082,11 +1121,7 @@ dmuon_status_t dmuon_update(void* param, const void* O, int64_t rows, int64_t co
 }
 
 dmuon_status_t dmuon_profile_start(void) {
-  for (ProfRec& r : g_prof) {
-    cudaEventDestroy(r.a);
-    cudaEventDestroy(r.b);
-  }
-  g_prof.clear();
+  g_prof.clear();  // the events stay in the pool
   g_prof_on = true;
   return DMUON_OK;
 }
@@ -1113,10 +1148,6 @@ int32_t dmuon_profile_stop_launches(dmuon_launch_record_t* recs, int32_t max_rec
     }
     ++n;
   }
-  for (ProfRec& r : g_prof) {
-    cudaEventDestroy(r.a);
-    cudaEventDestroy(r.b);
-  }
   g_prof.clear();
   if (!ok) {
     fail(DMUON_ERR_CUDA, "profile events failed");
@@ -1141,8 +1172,6 @@ int32_t dmuon_profile_stop(dmuon_kernel_stat_t* stats, int32_t max_stats) {
     } else {
       ok = false;
     }
-    cudaEventDestroy(r.a);
-    cudaEventDestroy(r.b);
   }
   g_prof.clear();
   if (!ok) {

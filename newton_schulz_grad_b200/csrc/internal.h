@@ -96,6 +96,18 @@ cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, 
                        int64_t ldp, int64_t ldx, int64_t ldy, float a, float alpha,
                        const float* scale, bool xbf16, cudaStream_t st, int* status);
 
+// The whole FFMA chain (steps x (gram, poly, apply), per-iteration form) of a
+// chunk in one launch, tiles ordered phase by phase with per-matrix
+// dependency counters (the same tiles and arithmetic as the three kernels
+// above, so the same bits).  x[0] holds X at entry, x[1] is the ping-pong
+// buffer; counters has batch + 1 entries (zeroed here); *result_x: the x
+// buffer holding the result.  cudaErrorNotSupported: more than 16 iterations
+// (run product by product).  inject_timeout: a test hook whose last
+// dependency is never met, so its bounded waits run out (DMUON_ERR_TIMEOUT).
+cudaError_t simt_chain(void* const* x, void* G, void* P, int batch, int m, int n, int64_t ldx, int64_t ldg,
+                       int32_t steps, const float* sched, const float* scale, bool xbf16, unsigned* counters,
+                       int* status, int num_sms, bool inject_timeout, cudaStream_t st, int* result_x);
+
 // ---- clip.cu --------------------------------------------------------------------
 // Each matrix is read as a flat array of rows * cols elements; one partial per
 // chunk of kClipChunk elements (ceil(rows * cols / kClipChunk) per matrix).

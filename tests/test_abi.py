@@ -119,10 +119,16 @@ def test_overlap_can_be_disabled(monkeypatch):
     assert nsg.dmuon_workspace_bytes(shapes, 5) <= 8 << 30
 
 
-def test_launch_count_thin_and_fp32_chunks():
+def test_launch_count_thin_and_fp32_chunks(monkeypatch):
     # fp32 and thin bf16 classes keep the separate update; thin bf16 chains
-    # (m <= 64) are one clustered launch
+    # (m <= 64) are one clustered launch, the other FFMA chains one fused launch
+    # (up to 16 iterations, product by product beyond or with DMUON_FUSED_CHAIN=0)
+    assert nsg.dmuon_step_launches([(256, 512, 0)], 5) == 3 + 1
+    assert nsg.dmuon_step_launches([(100, 200, 1)], 5) == 3 + 1   # bf16, fp32 X
+    assert nsg.dmuon_step_launches([(256, 512, 0)], 17) == 3 + 17 * 3
+    monkeypatch.setenv("DMUON_FUSED_CHAIN", "0")
     assert nsg.dmuon_step_launches([(256, 512, 0)], 5) == 3 + 5 * 3
+    monkeypatch.delenv("DMUON_FUSED_CHAIN")
     assert nsg.dmuon_step_launches([(32, 4096, 1)] * 3, 5) == 3 + 1
     assert nsg.dmuon_step_launches([(4096, 32, 1)], 5) == 3 + 1
     assert nsg.dmuon_step_launches([(32, 4096, 1)], 0) == 3

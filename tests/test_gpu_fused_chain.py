@@ -117,3 +117,61 @@ def test_two_fused_chains_on_two_streams_at_once(monkeypatch):
             assert nsg.dmuon_stream_status(s) == nsg.DMUON_OK
         for g, w in zip(got, want):
             assert np.array_equal(bits(g), bits(w))
+
+
+# --------------------------------------------------------------- FFMA chains
+def seeded_any(shape, seed, dtype):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return torch.randn(*shape, generator=g).to(dtype).to("cuda")
+
+
+@pytest.mark.parametrize("shape,dtype", [((256, 512), torch.float32), ((40, 70), torch.float32),
+                                         ((300, 129), torch.float32), ((1, 300), torch.float32),
+                                         ((96, 200), torch.bfloat16), ((136, 130), torch.bfloat16),
+                                         ((48, 30000), torch.bfloat16), ((1024, 640), torch.float32)],
+                         ids=lambda v: str(v))
+def test_fused_ffma_chain_equals_product_launches_and_oracle(shape, dtype, monkeypatch):
+    # fp32 matrices, small near-square bf16 matrices (fp32 X) and thin bf16
+    # matrices too wide for the clustered kernel all run the FFMA chain
+    X = seeded_any(shape, 11 * shape[0] + shape[1], dtype)
+    fused, split = ns_both(X, monkeypatch)
+    assert np.array_equal(bits(fused), bits(split))
+    tol = 1e-4 if dtype == torch.float32 else 2e-2
+    assert rel_fro(to64(fused), om.newton_schulz(to64(X), 5)) < tol
+
+
+def test_fused_ffma_chain_steps_and_custom_coefficients(monkeypatch):
+    X = seeded_any((256, 512), 3, torch.float32)
+    coeffs = [(3.0, -3.2, 1.2), (2.0, -1.5, 0.5), (1.5, -0.5, 0.0)] * 6
+    for steps in (1, 2, 7, 16, 17):  # 17 iterations: product by product
+        fused, split = ns_both(X, monkeypatch, steps=steps, coeffs=coeffs[:steps])
+        assert np.array_equal(bits(fused), bits(split))
+    c32 = [tuple(float(np.float32(v)) for v in t) for t in coeffs[:7]]
+    fused, _ = ns_both(X, monkeypatch, steps=7, coeffs=coeffs[:7])
+    assert rel_fro(to64(fused), om.newton_schulz(to64(X), 7, c32)) < 1e-4
+
+
+def test_fused_ffma_chain_wait_runs_out_and_recovers(monkeypatch):
+    X = seeded_any((256, 512), 4, torch.float32)
+    out = torch.empty_like(X)
+    monkeypatch.setenv("DMUON_FAULT_INJECT", "chain_wait")
+    nsg.dmuon_ns(X, out)
+    assert nsg.dmuon_stream_status() == nsg.DMUON_ERR_TIMEOUT
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    monkeypatch.delenv("DMUON_FAULT_INJECT")
+    fused, split = ns_both(X, monkeypatch)
+    assert np.array_equal(bits(fused), bits(split))
+
+
+def test_fused_ffma_chain_in_a_step(monkeypatch):
+    # the single-matrix fp32 workload through dmuon_step: fused == per product
+    w = workloads.get("single_256x512_f32")
+    runs = []
+    for fused in ("1", "0"):
+        monkeypatch.setenv("DMUON_FUSED_CHAIN", fused)
+        ps, gs, bs = workloads.make_all(w, "cuda")
+        nsg.dmuon_step(ps, gs, bs, wd=0.1)
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        runs.append([bits(t) for t in ps + bs])
+    for a, b in zip(*runs):
+        assert np.array_equal(a, b)

@@ -26,11 +26,6 @@ struct Elt<__nv_bfloat16> {
   static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
-// The elementwise passes touch every element once, so their loads and stores
-// are cache-streaming (ld/st.global.cs: lines allocated evict-first in L1 and
-// L2): when they run underneath the Newton-Schulz chain they do not push the
-// chain's operands out of L2.
-//
 // Load 8 consecutive elements starting at p into fp32 (vectorised when `vec`;
 // otherwise element by element, only the first `valid` ones, the rest 0).
 template <typename T>
@@ -39,13 +34,13 @@ __device__ __forceinline__ void load8(const T* p, float (&v)[8], bool vec, int v
 template <>
 __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8], bool vec, int valid) {
   if (vec) {
-    float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-    float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (i < valid) ? __ldcs(p + i) : 0.f;
+    for (int i = 0; i < 8; ++i) v[i] = (i < valid) ? p[i] : 0.f;
   }
 }
 
@@ -53,7 +48,7 @@ template <>
 __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8], bool vec,
                                                      int valid) {
   if (vec) {
-    uint4 raw = __ldcs(reinterpret_cast<const uint4*>(p));
+    uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -63,7 +58,7 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (i < valid) ? __bfloat162float(__ldcs(p + i)) : 0.f;
+    for (int i = 0; i < 8; ++i) v[i] = (i < valid) ? __bfloat162float(p[i]) : 0.f;
   }
 }
 
@@ -75,12 +70,12 @@ __device__ __forceinline__ void store8(T* p, const float (&v)[8], bool vec, int 
 template <>
 __device__ __forceinline__ void store8<float>(float* p, const float (&v)[8], bool vec, int valid) {
   if (vec) {
-    __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
-    __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(v[4], v[5], v[6], v[7]));
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      if (i < valid) __stcs(p + i, v[i]);
+      if (i < valid) p[i] = v[i];
   }
 }
 
@@ -92,11 +87,11 @@ __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const fl
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
 #pragma unroll
     for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    __stcs(reinterpret_cast<uint4*>(p), raw);
+    *reinterpret_cast<uint4*>(p) = raw;
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      if (i < valid) __stcs(p + i, __float2bfloat16_rn(v[i]));
+      if (i < valid) p[i] = __float2bfloat16_rn(v[i]);
   }
 }
 

@@ -68,6 +68,9 @@ def parse_args(argv=None):
                     help="time dmuon_step_clipped: global 2-norm clipping of the gradients to this bound")
     ap.add_argument("--lib", choices=["torch", "quack"], default="torch",
                     help="--stage lib_chain / lib_apply: the library whose GEMMs run the comparison")
+    ap.add_argument("--owners", action="store_true",
+                    help="dedicated ownership over the ranks: every rank holds the whole set, steps the "
+                         "matrices it owns and broadcasts them (strong scaling); default: one replica per rank")
     ap.add_argument("--launch-detail", default=None, metavar="PATH",
                     help="after the timed region, write every launch of one more step (kind, start, "
                          "duration, work) to PATH as JSON")
@@ -311,7 +314,11 @@ def run_ours(args):
     # graph capture needs a non-default stream; the library keeps one
     # workspace per stream, so warm-up and capture use the same one
     run_stream = torch.cuda.Stream(dev) if args.graph else stream
-    launches_per_step = nsg.dmuon_step_launches(shapes, w.ns_steps)
+    if args.owners:  # this rank launches the step of the matrices it owns
+        own = nsg.dmuon_assign_owners(shapes, world)[0]
+        launches_per_step = nsg.dmuon_step_launches([s for s, o in zip(shapes, own) if o == rank], w.ns_steps)
+    else:
+        launches_per_step = nsg.dmuon_step_launches(shapes, w.ns_steps)
     if args.clip_norm is not None:
         # one norm launch per table of <= 256 matrices of one shape, plus the coefficient
         groups = {}
@@ -322,6 +329,15 @@ def run_ours(args):
     def step():
         nsg.dmuon_step_ptrs(pp, gp, bp, shapes, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov,
                             ns_steps=w.ns_steps, wd=w.wd, stream=run_stream, max_norm=args.clip_norm)
+
+    if args.owners:
+        if args.graph or args.clip_norm is not None:
+            raise SystemExit("--owners runs without --graph and --clip-norm")
+        from newton_schulz_grad_b200.distributed import owned_step
+
+        def step():  # noqa: F811
+            owned_step(ps, gs, bs, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov, ns_steps=w.ns_steps,
+                       wd=w.wd)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -378,7 +394,8 @@ def run_ours(args):
         raise RuntimeError(f"timed steps failed: {nsg.STATUS_NAMES[st]}")
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = reduce_max(ms_local, dev)
-    value = aggregate_value(w.count, world, ms)
+    # replicas: every rank steps the whole set; owners: the ranks share one set
+    value = aggregate_value(w.count, 1 if args.owners else world, ms)
 
     peaks, peak_src = load_peaks()
     sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
@@ -435,7 +452,7 @@ def run_ours(args):
                 elem_iso[k] = {"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / float(peaks["hbm_gbs"]), 3)}
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.owners:  # the e2e pipeline steps whole replicas
         e2e = run_e2e(args, w, ps, gs, bs, shapes, stream, dev, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -444,7 +461,8 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "matrices/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "higher_is_better": True, "scaling": "strong" if args.owners else "weak", "vs_baseline": None,
+        "dtype": w.dtype,
         "data": "synthetic (seeded low-rank + noise gradients, random-init parameters)",
         "config": workload_config(w, args, world),
         "ns_tflops": round(executed / (ms / 1e3) / 1e12, 1),
@@ -489,7 +507,8 @@ def workload_config(w, args, world: int) -> dict:
             "ns_steps": w.ns_steps, "nesterov": w.nesterov, "lr": w.lr, "wd": w.wd,
             **({"clip": {"max_norm": args.clip_norm, "norm_type": 2.0, "fused": "dmuon_step_clipped"}}
                if getattr(args, "clip_norm", None) is not None else {}),
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "parallelism": (f"dedicated owners x{world}" if getattr(args, "owners", False) else f"replicas x{world}")
+            if world > 1 else "single GPU",
             "l2": f"no flush: each step touches {w.elements() * 2 * 7 / 1e9:.1f} GB "
                   f"(inputs alone {w.elements() * 2 * 3 / 1e9:.1f} GB) >> 126 MB L2"}
 

@@ -223,6 +223,26 @@ DMUON_API dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_sh
 DMUON_API dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int32_t* group_of,
                                  int32_t* order, int32_t* num_groups);
 
+/*
+ * dmuon_assign_owners - dedicated ownership of the matrices over `world`
+ * ranks (host only, no GPU).  DMuon FAQ, "Why isn't DMuon just ZeRO-1?": one
+ * rank owns a whole matrix and runs its Muon step, the other ranks receive the
+ * updated parameter; Training Guide, "Verify Parameter Assignment": the
+ * assignment is load-balanced and reported with per-rank loads and an
+ * imbalance.  The pages give no rule; this one: the load of a matrix is the
+ * flops of one Newton-Schulz iteration, 3 m^2 n + m^3 (m = min side); matrices
+ * go from the most expensive down (equal costs: lower index first), each to the
+ * rank with the least load so far (equal loads: lower rank).  The same input
+ * gives the same assignment on every rank.
+ *   shapes     HOST array of `count` shapes
+ *   world      number of ranks, >= 1
+ *   owner_of   HOST out, `count` ints: the rank that owns matrix i
+ *   loads      HOST out, `world` doubles: the flops each rank owns
+ *   imbalance  HOST out, 1 double: max(loads) / mean(loads) - 1 (0 when empty)
+ */
+DMUON_API dmuon_status_t dmuon_assign_owners(const dmuon_shape_t* shapes, int32_t count, int32_t world,
+                                             int32_t* owner_of, double* loads, double* imbalance);
+
 /* ------------------------------------------------------------------------ */
 /* Stage calls: the individual kernels of the path, over `batch` matrices    */
 /* stored one after another (matrix b starts at b * rows * ld elements).     */

@@ -39,7 +39,7 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
             "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout",
             "dmuon_clip_grad_norm", "dmuon_step_clipped", "dmuon_selftest_bounds",
-            "dmuon_profile_stop_launches")
+            "dmuon_profile_stop_launches", "dmuon_assign_owners")
 
 
 class DmuonError(RuntimeError):
@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
         "dmuon_profile_start": ([], i32),
         "dmuon_profile_stop": ([ctypes.POINTER(KernelStat), i32], i32),
         "dmuon_profile_stop_launches": ([ctypes.POINTER(LaunchRecord), i32], i32),
+        "dmuon_assign_owners": ([ctypes.POINTER(Shape), i32, i32, ctypes.POINTER(i32),
+                                 ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], i32),
         "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
         "dmuon_selftest_timeout": ([i32, vp], i32),
         "dmuon_clip_grad_norm": ([ctypes.POINTER(vp), ctypes.POINTER(Shape), i32, f32, f32, vp, vp], i32),
@@ -339,6 +341,16 @@ def dmuon_plan_groups(shapes: Sequence[Tuple[int, int, int]]):
     k = ctypes.c_int32(0)
     _check(_lib.dmuon_plan_groups(_shape_array(shapes), n, g, o, ctypes.byref(k)))
     return list(g)[:n], list(o)[:n], k.value
+
+
+def dmuon_assign_owners(shapes: Sequence[Tuple[int, int, int]], world: int):
+    """(owner_of, loads, imbalance): dedicated ownership over `world` ranks (host only)."""
+    n = len(shapes)
+    own = (ctypes.c_int32 * max(1, n))()
+    loads = (ctypes.c_double * max(1, world))()
+    imb = ctypes.c_double(0.0)
+    _check(_lib.dmuon_assign_owners(_shape_array(shapes), n, int(world), own, loads, ctypes.byref(imb)))
+    return list(own)[:n], list(loads)[:world], imb.value
 
 
 def dmuon_workspace_bytes(shapes, ns_steps: int = 5) -> int:

@@ -841,6 +841,26 @@ dmuon_status_t dmuon_plan_groups(const dmuon_shape_t* shapes, int32_t count, int
   return DMUON_OK;
 }
 
+dmuon_status_t dmuon_assign_owners(const dmuon_shape_t* shapes, int32_t count, int32_t world, int32_t* owner_of,
+                                   double* loads, double* imbalance) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
+  if (world < 1) return fail(DMUON_ERR_INVALID_ARG, "world must be >= 1");
+  if (!loads || !imbalance || (count > 0 && (!shapes || !owner_of)))
+    return fail(DMUON_ERR_INVALID_ARG, "null pointer argument");
+  for (int32_t i = 0; i < count; ++i) {
+    dmuon_status_t rc = check_shape(shapes[i].rows, shapes[i].cols, "dmuon_assign_owners");
+    if (rc != DMUON_OK) return rc;
+  }
+  assign_owners(shapes, count, world, owner_of, loads);
+  double total = 0.0, most = 0.0;
+  for (int32_t r = 0; r < world; ++r) {
+    total += loads[r];
+    most = std::max(most, loads[r]);
+  }
+  *imbalance = total > 0.0 ? most / (total / world) - 1.0 : 0.0;
+  return DMUON_OK;
+}
+
 int64_t dmuon_workspace_bytes(const dmuon_shape_t* shapes, int32_t count, int32_t ns_steps) {
   (void)ns_steps;
   if (count <= 0 || !shapes) return 0;

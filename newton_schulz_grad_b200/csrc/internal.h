@@ -269,5 +269,8 @@ struct StepPlan {
   int64_t buffer_bytes = 0;  // one buffer (two are used when overlapping)
 };
 StepPlan make_step_plan(const dmuon_shape_t* shapes, int32_t count);
+// Dedicated ownership of `count` matrices over `world` ranks (see
+// dmuon_assign_owners); loads has `world` entries.
+void assign_owners(const dmuon_shape_t* shapes, int32_t count, int32_t world, int32_t* owner_of, double* loads);
 
 }  // namespace dmuon

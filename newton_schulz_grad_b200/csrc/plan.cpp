@@ -176,4 +176,28 @@ ChunkOffsets chunk_offsets(const ChunkLayout& L, int64_t b) {
   return o;
 }
 
+// Dedicated ownership (every matrix to one rank): longest processing time
+// first over the Newton-Schulz flops of one iteration, 3 m^2 n + m^3; equal
+// costs in index order, equal loads to the lower rank.
+void assign_owners(const dmuon_shape_t* shapes, int32_t count, int32_t world, int32_t* owner_of,
+                   double* loads) {
+  std::vector<double> cost((size_t)count);
+  std::vector<int32_t> order((size_t)count);
+  for (int32_t i = 0; i < count; ++i) {
+    const double m = (double)std::min(shapes[i].rows, shapes[i].cols);
+    const double n = (double)std::max(shapes[i].rows, shapes[i].cols);
+    cost[(size_t)i] = 3.0 * m * m * n + m * m * m;
+    order[(size_t)i] = i;
+  }
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return cost[a] > cost[b]; });
+  for (int32_t r = 0; r < world; ++r) loads[r] = 0.0;
+  for (int32_t i : order) {
+    int32_t best = 0;
+    for (int32_t r = 1; r < world; ++r)
+      if (loads[r] < loads[best]) best = r;
+    owner_of[i] = best;
+    loads[best] += cost[(size_t)i];
+  }
+}
+
 }  // namespace dmuon

@@ -5,6 +5,7 @@ Importable by the tests, ``__graft_entry__.smoke()`` and the CPU legs of
 computes and the readings it takes where the documentation is silent.
 """
 from . import muon, emulate  # noqa: F401
-from .muon import (DEFAULT_COEFFS, NORM_EPS, apply_update, clip_grad_norm, coeff_schedule,  # noqa: F401
+from .muon import (DEFAULT_COEFFS, NORM_EPS, apply_update, assign_owners, clip_grad_norm,  # noqa: F401
+                   coeff_schedule, ns_iteration_flops,
                    frobenius_normalize, gram_ns_iterations, lr_scale, momentum_update,
                    muon_step, newton_schulz, orient, shape_groups)

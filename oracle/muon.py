@@ -208,3 +208,38 @@ def shape_groups(shapes: Sequence[Tuple[int, int, int]]):
         members[gid].append(i)
     order = [i for grp in members for i in grp]
     return group_of, order, len(members)
+
+
+def ns_iteration_flops(rows: int, cols: int) -> float:
+    """Flops of one Gram Newton-Schulz iteration on one matrix: 3 m^2 n + m^3
+    (m = min side, n = max side; one triangle of each symmetric product)."""
+    m, n = float(min(rows, cols)), float(max(rows, cols))
+    return 3.0 * m * m * n + m * m * m
+
+
+def assign_owners(shapes: Sequence[Tuple[int, int]], world: int):
+    """Dedicated ownership: every matrix to one rank, loads balanced.
+
+    DMuon FAQ, "Why isn't DMuon just ZeRO-1?": one rank owns the whole matrix and
+    runs Newton-Schulz on it, the others receive the updated parameter;
+    Training Guide, "Verify Parameter Assignment": the assignment is reported
+    with per-rank loads and an imbalance figure.  Reading (the pages give no
+    rule): the load of a matrix is its Newton-Schulz flops per iteration; the
+    matrices are taken from the most expensive down (equal costs: lower index
+    first) and each goes to the rank with the least load so far (equal loads:
+    lower rank); imbalance = max load / mean load - 1.  Returns (owner_of,
+    loads, imbalance).
+    """
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    cost = [ns_iteration_flops(r, c) for r, c in shapes]
+    order = sorted(range(len(shapes)), key=lambda i: (-cost[i], i))
+    loads = [0.0] * world
+    owner_of = [0] * len(shapes)
+    for i in order:
+        r = min(range(world), key=lambda k: (loads[k], k))
+        owner_of[i] = r
+        loads[r] += cost[i]
+    mean = sum(loads) / world
+    imbalance = (max(loads) / mean - 1.0) if mean > 0 else 0.0
+    return owner_of, loads, imbalance

@@ -28,8 +28,9 @@
 //
 // Both are persistent (one CTA, or CTA pair, per SM / SM pair), warp
 // specialised (warp 0 TMA producer, warp 1 TMEM allocator + single MMA
-// thread, warps 2-5 epilogue), with two TMEM accumulators (2 x 256 fp32
-// columns) so the epilogue of one tile overlaps the MMAs of the next.  The
+// thread, warps 2-5 epilogue, 2-9 for reductions up to 2048), with two TMEM
+// accumulators (2 x 256 fp32 columns) so the epilogue of one tile overlaps
+// the MMAs of the next.  The
 // polynomial terms (alpha, b G, a X) are fused into the epilogue.  For gram
 // and poly only tiles that touch the lower triangle are computed; every
 // element r >= c is stored, and r > c also at its mirror (c, r), so each
@@ -60,7 +61,23 @@ constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int UK = 16;  // K of one tcgen05.mma kind::f16
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int kThreads = 192;
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2.. epilogue.
+// A warp reaches only the TMEM lane quarter (warp index mod 4).  EPI = 4: one
+// epilogue warp per quarter drains all 256 accumulator columns.  EPI = 8: two
+// warps per quarter, 128 columns each, twice the drain rate, which short
+// reductions need to keep the MMAs busy (a 128 x 256 x 1408 tile's MMAs take
+// about half as long as four warps take to drain it).  Long reductions keep
+// four: the extra warps share issue slots with the MMA-issuing warp and
+// leave fewer registers to a co-resident elementwise kernel.
+template <int EPI>
+struct Epi {
+  static_assert(EPI == 4 || EPI == 8, "four or eight epilogue warps");
+  static constexpr int kCols = BN / (EPI / 4);  // accumulator columns per epilogue warp
+  static constexpr int kChunks = kCols / 32;    // 32-column chunks per epilogue warp
+  static constexpr int kThreads = 64 + 32 * EPI;
+};
+// Reductions up to this length use eight epilogue warps.
+constexpr int kShortK = 2048;
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s per wait
 
 // one-CTA kernel
@@ -464,19 +481,18 @@ __device__ __forceinline__ void store_upd_chunk(const UpdTable& u, const TcArgs&
 }
 
 // Epilogue of one apply tile with the fused update (see epilogue_row).
-template <bool COH>
+template <bool COH, int NCH>
 __device__ __forceinline__ void epilogue_row_update(const TcArgs& a, const UpdTable& u, uint32_t taddr, int b,
-                                                    int r, int J) {
+                                                    int r, int cbase) {
   const bool row_ok = r < a.m;
   const float alpha = a.p1 * (a.scale ? a.scale[b] : 1.f);
-  const int cbase = J * BN;
   UpdChunk k0, k1;
   if (row_ok) load_upd_chunk<COH>(u, a, b, r, cbase, k0);
   // one chunk: load the next chunk's operands, then drain this one
   auto chunk = [&](int ch, const UpdChunk& cur, UpdChunk& nxt) -> bool {
     const int c0 = cbase + ch * 32;
     if (c0 >= a.n) return false;  // warp-uniform
-    if (row_ok && ch + 1 < BN / 32 && c0 + 32 < a.n) load_upd_chunk<COH>(u, a, b, r, c0 + 32, nxt);
+    if (row_ok && ch + 1 < NCH && c0 + 32 < a.n) load_upd_chunk<COH>(u, a, b, r, c0 + 32, nxt);
     uint32_t raw[32];
     tmem_ld32(taddr + (uint32_t)(ch * 32), raw);
     tmem_ld_wait();
@@ -484,33 +500,34 @@ __device__ __forceinline__ void epilogue_row_update(const TcArgs& a, const UpdTa
     return true;
   };
 #pragma unroll 1
-  for (int ch = 0; ch < BN / 32; ch += 2) {
+  for (int ch = 0; ch < NCH; ch += 2) {
     if (!chunk(ch, k0, k1)) break;
     if (!chunk(ch + 1, k1, k0)) break;
   }
 }
 
 // Before an update tile's accumulator is ready: pull the parameters it
-// rewrites into L2 (oriented rows [r0, r0 + 32) of this warp, columns
-// [col0, col0 + 256)), so the epilogue's loads do not wait on DRAM.
+// rewrites into L2 (oriented rows [r0, r0 + 32) of this warp, its NCOL
+// columns from col0), so the epilogue's loads do not wait on DRAM.
+template <int NCOL>
 __device__ __forceinline__ void prefetch_update_tile(const UpdTable& u, int b, int r0, int col0, int m, int n,
                                                      int lane) {
   const char* p = static_cast<const char*>(u.p[b]);
   const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
   if (r0 >= m) return;
   if (tr) {
-    // source rows col0 .. col0 + 255, 64 bytes (32 columns from r0) each: 8 per lane
+    // source rows col0 .. col0 + NCOL - 1, 64 bytes (32 columns from r0) each
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = col0 + lane * 8 + i;
+    for (int i = 0; i < NCOL / 32; ++i) {
+      const int c = col0 + lane * (NCOL / 32) + i;
       if (c < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + ((int64_t)c * m + r0) * 2));
     }
   } else {
-    // row r0 + lane, 512 bytes from col0: four 128-byte lines
+    // row r0 + lane, 2 NCOL bytes from col0: 128-byte lines
     const int r = r0 + lane;
     if (r < m) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < NCOL / 64; ++i) {
         const int c = col0 + i * 64;
         if (c < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + ((int64_t)r * n + c) * 2));
       }
@@ -518,15 +535,15 @@ __device__ __forceinline__ void prefetch_update_tile(const UpdTable& u, int b, i
   }
 }
 
-// Epilogue of one tile for one accumulator row: TMEM lane quarter `wq` of
-// accumulator columns [col0, col0 + 256), output row r, output columns from
-// J * 256.  Warp-collective (tcgen05.ld).  UPD (apply only): update the
-// parameters instead of storing the result.
-template <int MODE, bool UPD, bool COH = false>
+// Epilogue of one tile for one accumulator row: NCH chunks of 32 accumulator
+// columns from taddr (TMEM lane quarter of the warp), output row r, output
+// columns from cbase.  Warp-collective (tcgen05.ld).  UPD (apply only):
+// update the parameters instead of storing the result.
+template <int MODE, bool UPD, bool COH, int NCH>
 __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename UpdSel<UPD>::type& u, uint32_t taddr,
-                                             int b, int r, int J) {
+                                             int b, int r, int cbase) {
   if constexpr (UPD) {
-    epilogue_row_update<COH>(a, u, taddr, b, r, J);
+    epilogue_row_update<COH, NCH>(a, u, taddr, b, r, cbase);
     return;
   }
   const bool row_ok = r < a.m;
@@ -540,8 +557,8 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename Upd
   __nv_bfloat16* Cm = a.C + (int64_t)b * a.sC;
   const __nv_bfloat16* Em = a.E ? a.E + (int64_t)b * a.sE : nullptr;
 #pragma unroll 1
-  for (int ch = 0; ch < BN / 32; ++ch) {
-    const int c0 = J * BN + ch * 32;
+  for (int ch = 0; ch < NCH; ++ch) {
+    const int c0 = cbase + ch * 32;
     if (c0 >= a.n) break;  // warp-uniform
     uint32_t raw[32];
     tmem_ld32(taddr + (uint32_t)(ch * 32), raw);
@@ -641,8 +658,8 @@ __device__ __forceinline__ Bars bar_layout(uint64_t* bars) {
 }
 
 // ================================================================ one CTA
-template <int MODE, bool UPD>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MODE, bool UPD, int EPI>
+__global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
     k_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
          const TcArgs a, const __grid_constant__ typename UpdSel<UPD>::type u) {
   extern __shared__ uint8_t smem_raw[];
@@ -661,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(B.tfull0 + 8 * s, 1);
-      mbar_init(B.tempty0 + 8 * s, 4);  // one arrival per epilogue warp
+      mbar_init(B.tempty0 + 8 * s, EPI);  // one arrival per epilogue warp
     }
     mbar_init(B.done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -769,7 +786,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue
-    const int wq = warp & 3;  // TMEM lanes 32*wq .. 32*wq+31
+    using E = Epi<EPI>;
+    const int wq = warp & 3;                     // TMEM lanes 32*wq .. 32*wq+31
+    const int half = ((warp - 2) >> 2) * E::kCols;  // this warp's accumulator columns from half
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
@@ -777,17 +796,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_tile<MODE>(a, t, b, I, J);
       if constexpr (UPD) {
         // this CTA's first tile now, then always the next one during this epilogue
-        if (t == (int)blockIdx.x) prefetch_update_tile(u, b, I * BM1 + wq * 32, J * BN, a.m, a.n, lane);
+        if (t == (int)blockIdx.x)
+          prefetch_update_tile<E::kCols>(u, b, I * BM1 + wq * 32, J * BN + half, a.m, a.n, lane);
         if (t + (int)gridDim.x < a.total_tiles) {
           int b2, I2, J2;
           decode_tile<MODE>(a, t + (int)gridDim.x, b2, I2, J2);
-          prefetch_update_tile(u, b2, I2 * BM1 + wq * 32, J2 * BN, a.m, a.n, lane);
+          prefetch_update_tile<E::kCols>(u, b2, I2 * BM1 + wq * 32, J2 * BN + half, a.m, a.n, lane);
         }
       }
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
-      epilogue_row<MODE, UPD>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
-                         I * BM1 + wq * 32 + lane, J);
+      epilogue_row<MODE, UPD, false, E::kChunks>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) +
+                                                         (uint32_t)(acc * BN + half),
+                                                 b, I * BM1 + wq * 32 + lane, J * BN + half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(B.tempty0 + 8 * acc);
@@ -805,8 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // =============================================================== CTA pair
-template <int MODE, bool UPD>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int MODE, bool UPD, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 1)
     k_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const TcArgs a, const __grid_constant__ typename UpdSel<UPD>::type u) {
   extern __shared__ uint8_t smem_raw[];
@@ -829,7 +850,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(B.tfull0 + 8 * s, 1);   // the leader's commit, multicast to both
-      mbar_init(B.tempty0 + 8 * s, 8);  // in the leader: one per epilogue warp of both CTAs
+      mbar_init(B.tempty0 + 8 * s, 2 * EPI);  // in the leader: one per epilogue warp of both CTAs
     }
     mbar_init(B.done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -941,7 +962,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------- epilogue (both CTAs)
+    using E = Epi<EPI>;
     const int wq = warp & 3;
+    const int half = ((warp - 2) >> 2) * E::kCols;
     const uint32_t tempty_leader0 = mapa_shared(B.tempty0, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -949,17 +972,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int b, I, J;
       decode_tile<MODE>(a, t, b, I, J);
       if constexpr (UPD) {
-        if (t == pair) prefetch_update_tile(u, b, I * BM2 + (int)rank * 128 + wq * 32, J * BN, a.m, a.n, lane);
+        if (t == pair)
+          prefetch_update_tile<E::kCols>(u, b, I * BM2 + (int)rank * 128 + wq * 32, J * BN + half, a.m, a.n,
+                                         lane);
         if (t + npairs < a.total_tiles) {
           int b2, I2, J2;
           decode_tile<MODE>(a, t + npairs, b2, I2, J2);
-          prefetch_update_tile(u, b2, I2 * BM2 + (int)rank * 128 + wq * 32, J2 * BN, a.m, a.n, lane);
+          prefetch_update_tile<E::kCols>(u, b2, I2 * BM2 + (int)rank * 128 + wq * 32, J2 * BN + half, a.m,
+                                         a.n, lane);
         }
       }
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
-      epilogue_row<MODE, UPD>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN), b,
-                         I * BM2 + (int)rank * 128 + wq * 32 + lane, J);
+      epilogue_row<MODE, UPD, false, E::kChunks>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) +
+                                                         (uint32_t)(acc * BN + half),
+                                                 b, I * BM2 + (int)rank * 128 + wq * 32 + lane, J * BN + half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
@@ -1095,8 +1122,8 @@ __device__ __forceinline__ void decode_phase_tile(const PhaseDesc& ph, int t, in
 // G = 1: one CTA, 128 x 256 tiles (cta_group::1); G = 2: CTA pair, 256 x 256
 // tiles (cta_group::2).  Both load K-major operands as boxes of 128 rows (the
 // one-CTA kernel's 256 B rows as two), so one set of tensor maps serves both.
-template <int G>
-__global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ ChainParams P) {
+template <int G, int EPI>
+__global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_constant__ ChainParams P) {
   constexpr int STAGES = G == 2 ? STAGES2 : STAGES1;
   constexpr int STAGE_BYTES = G == 2 ? STAGE2_BYTES : STAGE1_BYTES;
   constexpr int A_BYTES = G == 2 ? A2_BYTES : A1_BYTES;
@@ -1124,12 +1151,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(B.tfull0 + 8 * s, 1);
-      mbar_init(B.tempty0 + 8 * s, 4 * G);  // one arrival per epilogue warp (of both CTAs)
+      mbar_init(B.tempty0 + 8 * s, EPI * G);  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(B.done, 1);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(qfull0 + 8 * s, 1);              // the leader's producer
-      mbar_init(qempty0 + 8 * s, G == 2 ? 10 : 5);  // MMA + 4 epilogue warps (+ peer producer + 4 warps)
+      // MMA + the epilogue warps (+ the peer's producer and epilogue warps)
+      mbar_init(qempty0 + 8 * s, G * (1 + EPI));
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int i = 0; i < kChainMaps; ++i)
@@ -1316,7 +1344,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
     __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue
+    using E = Epi<EPI>;
     const int wq = warp & 3;
+    const int half = ((warp - 2) >> 2) * E::kCols;
     const uint32_t tempty0 = G == 2 ? mapa_shared(B.tempty0, 0) : B.tempty0;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -1340,13 +1370,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
       advance(qs, qph);
       bool next_prefetched = false;
       if (ph.upd) {
-        if (!prefetched) prefetch_update_tile(P.u, b, r0, J * BN, ph.a.m, ph.a.n, lane);
+        if (!prefetched) prefetch_update_tile<E::kCols>(P.u, b, r0, J * BN + half, ph.a.m, ph.a.n, lane);
         if (tn >= 0) {
           const PhaseDesc& pn = P.ph[find_phase(P, tn)];
           if (pn.upd) {
             int b2, I2, J2;
             decode_phase_tile(pn, tn, b2, I2, J2);
-            prefetch_update_tile(P.u, b2, I2 * TM + (int)rank * 128 + wq * 32, J2 * BN, pn.a.m, pn.a.n, lane);
+            prefetch_update_tile<E::kCols>(P.u, b2, I2 * TM + (int)rank * 128 + wq * 32, J2 * BN + half, pn.a.m,
+                                           pn.a.n, lane);
             next_prefetched = true;
           }
         }
@@ -1354,19 +1385,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
       prefetched = next_prefetched;
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, status)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN + half);
+      const int c0 = J * BN + half;
       const NoUpd none{};
       // a local copy: read from the indexed parameter table, the arguments would
       // be reloaded after every store of the epilogue (which might alias them)
       const TcArgs a = ph.a;
       if (ph.upd)
-        epilogue_row<kApply, true, true>(a, P.u, taddr, b, r0 + lane, J);
+        epilogue_row<kApply, true, true, E::kChunks>(a, P.u, taddr, b, r0 + lane, c0);
       else if (ph.mode == kApply)
-        epilogue_row<kApply, false, true>(a, none, taddr, b, r0 + lane, J);
+        epilogue_row<kApply, false, true, E::kChunks>(a, none, taddr, b, r0 + lane, c0);
       else if (ph.mode == kPoly)
-        epilogue_row<kPoly, false, true>(a, none, taddr, b, r0 + lane, J);
+        epilogue_row<kPoly, false, true, E::kChunks>(a, none, taddr, b, r0 + lane, c0);
       else
-        epilogue_row<kGram, false, true>(a, none, taddr, b, r0 + lane, J);
+        epilogue_row<kGram, false, true, E::kChunks>(a, none, taddr, b, r0 + lane, c0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1481,11 +1513,12 @@ int max_pair_units(int num_sms) {
   std::lock_guard<std::mutex> lock(mu);
   if (cached[dev] > 0) return cached[dev];
   int n = 0;
-  cudaError_t e = cudaFuncSetAttribute(k_chain<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(k_chain<2, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
   if (e == cudaSuccess) {
+    // shared memory allows one CTA per SM whatever the epilogue width
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(num_sms & ~1));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(Epi<8>::kThreads);
     cfg.dynamicSmemBytes = SMEM2_BYTES;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1494,7 +1527,7 @@ int max_pair_units(int num_sms) {
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    e = cudaOccupancyMaxActiveClusters(&n, (void*)k_chain<2>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, (void*)k_chain<2, 8>, &cfg);
   }
   if (e != cudaSuccess || n <= 0) {
     cudaGetLastError();
@@ -1504,30 +1537,47 @@ int max_pair_units(int num_sms) {
   return cached[dev];
 }
 
-template <int MODE, bool UPD = false>
-cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms, bool pair,
-                   cudaStream_t st, const typename UpdSel<UPD>::type& u = {}) {
+// Epilogue warps for a reduction of length k; DMUON_EPI_WARPS=4 or 8 forces
+// one width (for measurements).
+int epi_warps(int64_t k) {
+  const char* v = std::getenv("DMUON_EPI_WARPS");
+  const int forced = v ? std::atoi(v) : 0;
+  if (forced == 4 || forced == 8) return forced;
+  return k <= kShortK ? 8 : 4;
+}
+
+template <int MODE, bool UPD, int EPI>
+cudaError_t launch_epi(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a, int64_t total, int num_sms,
+                       bool pair, cudaStream_t st, const typename UpdSel<UPD>::type& u) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_tc<MODE, UPD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
+    attr_err = cudaFuncSetAttribute(k_tc<MODE, UPD, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(k_tc2<MODE, UPD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+      attr_err =
+          cudaFuncSetAttribute(k_tc2<MODE, UPD, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  if (pair) {
+    const int units = max_pair_units(num_sms);
+    const int64_t pairs = total < units ? total : units;
+    k_tc2<MODE, UPD, EPI><<<(int)(2 * pairs), Epi<EPI>::kThreads, SMEM2_BYTES, st>>>(ma, mb, a, u);
+  } else {
+    const int grid = (int)(total < num_sms ? total : num_sms);
+    k_tc<MODE, UPD, EPI><<<grid, Epi<EPI>::kThreads, SMEM1_BYTES, st>>>(ma, mb, a, u);
+  }
+  return cudaGetLastError();
+}
+
+template <int MODE, bool UPD = false>
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms, bool pair,
+                   cudaStream_t st, const typename UpdSel<UPD>::type& u = {}) {
   const int64_t total = (int64_t)a.tiles_per_mat * batch;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffff) return cudaErrorInvalidValue;
   a.total_tiles = (int)total;
-  if (pair) {
-    const int units = max_pair_units(num_sms);
-    const int64_t pairs = total < units ? total : units;
-    k_tc2<MODE, UPD><<<(int)(2 * pairs), kThreads, SMEM2_BYTES, st>>>(ma, mb, a, u);
-  } else {
-    const int grid = (int)(total < num_sms ? total : num_sms);
-    k_tc<MODE, UPD><<<grid, kThreads, SMEM1_BYTES, st>>>(ma, mb, a, u);
-  }
-  return cudaGetLastError();
+  if (epi_warps(a.k) == 8) return launch_epi<MODE, UPD, 8>(ma, mb, a, total, num_sms, pair, st, u);
+  return launch_epi<MODE, UPD, 4>(ma, mb, a, total, num_sms, pair, st, u);
 }
 
 // Arguments of each product; the per-product launches and the fused chain
@@ -1692,6 +1742,8 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
   const bool blocked = false == std::all_of(blocks.begin(), blocks.end(), [](int l) { return l == 1; });
   if (blocked && !(buf.slot[2] && buf.slot[3] && buf.slot[4])) return cudaErrorNotSupported;
   const int G = pair ? 2 : 1;
+  // every product but the Gram matrix reduces over m
+  const int EPI = epi_warps(m);
 
   std::unique_ptr<ChainParams> P(new ChainParams());
   cudaError_t e = make_map(&P->maps[kMapX0], buf.x[0], n, m, batch, ldn, BK, 128);
@@ -1712,7 +1764,7 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
     ph.mapA = mapA;
     ph.mapB = mapB;
     ph.tile_start = (int)tiles;
-    ph.dep = (uint32_t)(4 * G * per_matrix);  // every epilogue warp of every CTA of a tile adds 1
+    ph.dep = (uint32_t)(EPI * G * per_matrix);  // every epilogue warp of every CTA of a tile adds 1
     tiles += a.total_tiles;
     per_matrix += a.tiles_per_mat;
   };
@@ -1780,16 +1832,21 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_chain<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM1_BYTES);
+    const int one = SMEM1_BYTES, two = SMEM2_BYTES;
+    attr_err = cudaFuncSetAttribute(k_chain<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, one);
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(k_chain<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+      attr_err = cudaFuncSetAttribute(k_chain<1, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, one);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(k_chain<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, two);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(k_chain<2, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, two);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int max_units = pair ? max_pair_units(num_sms) : num_sms;
   const int units = (int)(tiles < max_units ? tiles : max_units);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(G * units));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(EPI == 8 ? Epi<8>::kThreads : Epi<4>::kThreads);
   cfg.dynamicSmemBytes = pair ? SMEM2_BYTES : SMEM1_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
@@ -1799,7 +1856,10 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = pair ? 1 : 0;
-  e = pair ? cudaLaunchKernelEx(&cfg, k_chain<2>, *P) : cudaLaunchKernelEx(&cfg, k_chain<1>, *P);
+  if (EPI == 8)
+    e = pair ? cudaLaunchKernelEx(&cfg, k_chain<2, 8>, *P) : cudaLaunchKernelEx(&cfg, k_chain<1, 8>, *P);
+  else
+    e = pair ? cudaLaunchKernelEx(&cfg, k_chain<2, 4>, *P) : cudaLaunchKernelEx(&cfg, k_chain<1, 4>, *P);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1813,7 +1873,8 @@ const char* tc_config_string() {
   return "tcgen05 bf16->fp32: CTA-pair kernel (cta_group::2, M256xN256xK16, 6 x 32 KB stages per CTA) for "
          "m >= 256 unless 128-row tiles compute over 6 % less area, one-CTA kernel (cta_group::1, "
          "M128xN256xK16, 4 x 48 KB stages) otherwise; BK=64 SW128, 2 TMEM accumulators, persistent "
-         "192-thread CTAs (TMA warp, MMA warp, 4 epilogue warps); last apply of a chain fused with the update";
+         "CTAs (TMA warp, MMA warp, 4 epilogue warps, 8 for reductions up to 2048); last apply of a chain "
+         "fused with the update";
 }
 
 }  // namespace dmuon

@@ -175,3 +175,25 @@ def test_fused_ffma_chain_in_a_step(monkeypatch):
         runs.append([bits(t) for t in ps + bs])
     for a, b in zip(*runs):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("shape", [(1408, 2048), (2048, 1408), (300, 700), (4096, 4096), (1024, 2816)],
+                         ids=lambda s: f"{s[0]}x{s[1]}")
+@pytest.mark.parametrize("fused", ["0", "1"])
+def test_epilogue_width_gives_the_same_bits(shape, fused, monkeypatch):
+    # four or eight epilogue warps drain the same accumulator columns with the
+    # same arithmetic: the width may change the speed, never a bit
+    monkeypatch.setenv("DMUON_FUSED_CHAIN", fused)
+    X = seeded(shape, 7 * shape[0] + shape[1])
+    p0 = seeded(shape, 11 + shape[0], 0.02)
+    g = seeded(shape, 13 + shape[1])
+    outs = []
+    for width in ("4", "8"):
+        monkeypatch.setenv("DMUON_EPI_WARPS", width)
+        o = torch.empty_like(X)
+        nsg.dmuon_ns(X, o)
+        p, b = p0.clone(), torch.zeros_like(p0)
+        nsg.dmuon_step([p], [g], [b], wd=0.1)     # the last apply fused with the update
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        outs.append((bits(o), bits(p)))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])

@@ -43,6 +43,9 @@ def test_llama7b_full_step_sampled_parity():
     w = workloads.get("llama_7b_bf16")
     sample = [1, 4, 6]  # k_proj (4096x4096), gate_proj (11008x4096), down_proj (4096x11008)
     sample += [w.count - 3]  # a last-layer gate_proj (last chunk of its class)
+    # layer 16's v_proj and gate_proj: members 66 of 128 and 48 of 96 of their
+    # classes, in the middle chunk of each (chunks of 26 and of 12)
+    sample += [114, 116]
     full_step_sampled_parity(w, sample)
 
 

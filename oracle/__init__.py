@@ -6,6 +6,7 @@ computes and the readings it takes where the documentation is silent.
 """
 from . import muon, emulate  # noqa: F401
 from .muon import (DEFAULT_COEFFS, NORM_EPS, apply_update, assign_owners, clip_grad_norm,  # noqa: F401
+                   clip_grad_norm_buckets,
                    coeff_schedule, ns_iteration_flops,
                    frobenius_normalize, gram_ns_iterations, lr_scale, momentum_update,
                    muon_step, newton_schulz, orient, shape_groups)

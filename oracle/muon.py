@@ -188,6 +188,22 @@ def clip_grad_norm(grads: Sequence[np.ndarray], max_norm: float, norm_type: floa
         return [g * coef for g in gs], total, coef
 
 
+def clip_grad_norm_buckets(buckets: Sequence[Sequence[np.ndarray]], max_norms: Sequence[float],
+                           norm_types: Sequence[float]):
+    """Several independent clips at once.
+
+    Training Guide, "Fused CUDA clip for regular / Muon / AdamW": when several
+    gradient groups (buckets) are clipped together, each bucket keeps the
+    semantics of its own clip: bucket k is clipped by the global
+    norm_types[k]-norm of its gradients alone, with max_norms[k], exactly as
+    clip_grad_norm clips that list.  An empty bucket has total 0.  Returns one
+    (clipped gradients, total, coef) per bucket.
+    """
+    if not (len(buckets) == len(max_norms) == len(norm_types)):
+        raise ValueError("one max_norm and one norm_type per bucket")
+    return [clip_grad_norm(b, float(mx), float(nt)) for b, mx, nt in zip(buckets, max_norms, norm_types)]
+
+
 def shape_groups(shapes: Sequence[Tuple[int, int, int]]):
     """Partition matrices by (rows, cols, dtype).
 

@@ -404,3 +404,40 @@ def test_clip_infinity_gives_zero_coefficient():
         out, total, coef = om.clip_grad_norm(gs, 1.0, norm_type)
         assert total == np.inf and coef == 0.0
         assert np.isnan(out[0][0, 1]) and out[0][0, 0] == 0.0 and out[1][0, 0] == 0.0
+
+
+def test_clip_buckets_match_pytorch_per_bucket():
+    # Training Guide, "Fused CUDA clip for regular / Muon / AdamW": every bucket
+    # keeps the semantics of its own clip.  PyTorch's clip_grad_norm_, called
+    # once per bucket (CPU, fp64), pins totals, coefficients and values; the
+    # buckets differ in norm type, max_norm, size, and one holds a NaN (which
+    # must not reach the others) and one is below its bound
+    buckets = [[gauss((5, 7), 50), gauss((2, 9), 51) * 4.0],
+               [gauss((3, 3), 52)],
+               [gauss((1, 13), 53) * 0.01, gauss((6, 2), 54)],
+               [gauss((4, 4), 55)]]
+    buckets[3][0][1, 2] = np.nan
+    max_norms = [1.5, 0.25, 1e6, 1.0]
+    norm_types = [2.0, float("inf"), 1.0, 2.0]
+    got = om.clip_grad_norm_buckets(buckets, max_norms, norm_types)
+    assert len(got) == 4
+    for bucket, mx, nt, (out, total, coef) in zip(buckets, max_norms, norm_types, got):
+        ts = [torch.nn.Parameter(torch.zeros(g.shape, dtype=torch.float64)) for g in bucket]
+        for t, g in zip(ts, bucket):
+            t.grad = torch.from_numpy(g.copy())
+        want = float(torch.nn.utils.clip_grad_norm_(ts, mx, norm_type=nt))
+        assert (np.isnan(total) and np.isnan(want)) or total == pytest.approx(want, rel=1e-12, abs=0)
+        for o, t in zip(out, ts):
+            w = t.grad.numpy()
+            assert np.array_equal(np.isnan(o), np.isnan(w))
+            assert np.allclose(o[~np.isnan(w)], w[~np.isnan(w)], rtol=1e-12, atol=0)
+    # the NaN stayed in its bucket; the bucket below its bound is unchanged
+    assert not any(np.isnan(o).any() for _, (out, _, _) in zip(range(3), got) for o in out)
+    assert got[2][2] == 1.0 and all(np.array_equal(o, g) for o, g in zip(got[2][0], buckets[2]))
+
+
+def test_clip_buckets_empty_bucket_and_argument_errors():
+    out, total, coef = om.clip_grad_norm_buckets([[], [gauss((2, 2), 56)]], [1.0, 1.0], [2.0, 2.0])[0]
+    assert out == [] and total == 0.0 and coef == 1.0
+    with pytest.raises(ValueError):
+        om.clip_grad_norm_buckets([[gauss((2, 2), 57)]], [1.0, 2.0], [2.0])

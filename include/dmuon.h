@@ -211,6 +211,37 @@ DMUON_API dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_sh
                                               dmuon_stream_t stream);
 
 /*
+ * dmuon_clip_grad_norm_buckets - several independent global-norm clips in one
+ * set of launches (DMuon Training Guide, "Fused CUDA clip for regular / Muon /
+ * AdamW": when several gradient groups are clipped together, the norms, the
+ * clip coefficients and the in-place scaling of every bucket are computed
+ * together, each bucket with the semantics of its own clip).  Bucket k is
+ * clipped exactly as dmuon_clip_grad_norm would clip its gradients alone, with
+ * max_norms[k] and norm_types[k]: the same formula, reduction order and bits.
+ * A gradient of any rank is passed as rows x cols with rows * cols = its
+ * element count (the clip reads every gradient as one flat array).
+ *   grads, shapes, count  every bucket's gradients, as for dmuon_clip_grad_norm
+ *                 (none may overlap another, in any bucket)
+ *   bucket_of    HOST array of `count` ints in [0, num_buckets)
+ *   num_buckets  1 .. 128
+ *   max_norms    HOST array of num_buckets floats, each finite and >= 0
+ *   norm_types   HOST array of num_buckets floats, each 1, 2 or INFINITY
+ *   total_norms  DEVICE array of num_buckets doubles, or NULL: bucket k's
+ *                total in total_norms[k] (0 for an empty bucket)
+ * Launches on `stream`: the norm partials of every bucket's same-shape tables,
+ * one launch computing every bucket's total and coefficient (one block per
+ * bucket), the in-place scaling of every table.  A NaN in one bucket makes
+ * that bucket's gradients NaN and leaves the others alone.  Errors: as
+ * dmuon_clip_grad_norm, plus DMUON_ERR_INVALID_ARG for a bucket index out of
+ * range or a bad count of buckets.
+ */
+DMUON_API dmuon_status_t dmuon_clip_grad_norm_buckets(void* const* grads, const dmuon_shape_t* shapes,
+                                                      int32_t count, const int32_t* bucket_of,
+                                                      int32_t num_buckets, const float* max_norms,
+                                                      const float* norm_types, double* total_norms,
+                                                      dmuon_stream_t stream);
+
+/*
  * dmuon_plan_groups - the shape grouping dmuon_step uses (host only, no GPU).
  * Matrices with equal (rows, cols, dtype) form a group; group ids follow
  * first appearance; `order` lists the groups one after another, members in

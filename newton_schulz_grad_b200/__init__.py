@@ -39,7 +39,7 @@ EXPORTED = ("dmuon_ns", "dmuon_ns_ex", "dmuon_step", "dmuon_plan_groups", "dmuon
             "dmuon_workspace_bytes", "dmuon_step_launches", "dmuon_build_info",
             "dmuon_profile_start", "dmuon_profile_stop", "dmuon_ns_noalloc", "dmuon_selftest_timeout",
             "dmuon_clip_grad_norm", "dmuon_step_clipped", "dmuon_selftest_bounds",
-            "dmuon_profile_stop_launches", "dmuon_assign_owners")
+            "dmuon_profile_stop_launches", "dmuon_assign_owners", "dmuon_clip_grad_norm_buckets")
 
 
 class DmuonError(RuntimeError):
@@ -99,6 +99,8 @@ def _load() -> ctypes.CDLL:
         "dmuon_ns_noalloc": ([vp, vp, i64, i64, i32, fp, i32, vp, vp], i32),
         "dmuon_selftest_timeout": ([i32, vp], i32),
         "dmuon_clip_grad_norm": ([ctypes.POINTER(vp), ctypes.POINTER(Shape), i32, f32, f32, vp, vp], i32),
+        "dmuon_clip_grad_norm_buckets": ([ctypes.POINTER(vp), ctypes.POINTER(Shape), i32, ctypes.POINTER(i32), i32,
+                                          ctypes.POINTER(f32), ctypes.POINTER(f32), vp, vp], i32),
         "dmuon_selftest_bounds": ([vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -331,6 +333,60 @@ def dmuon_clip_grad_norm(grads: Sequence[torch.Tensor], max_norm: float, norm_ty
     with torch.cuda.device(dev):
         _check(_lib.dmuon_clip_grad_norm(ga, _shape_array(shapes), n, float(max_norm), float(norm_type),
                                          _ptr(total_norm), st))
+
+
+_MAX_SIDE = 1 << 20
+
+
+def _flat_shape(t: torch.Tensor) -> Tuple[int, int]:
+    # the clip reads a gradient as one flat array: any rank, as rows x cols
+    n = t.numel()
+    if n == 0:
+        raise ValueError("empty gradient")
+    cols = t.shape[-1] if t.dim() >= 2 else n
+    if cols > _MAX_SIDE or n // cols > _MAX_SIDE:
+        cols = next((c for c in range(min(n, _MAX_SIDE), 0, -1) if n % c == 0 and n // c <= _MAX_SIDE), 0)
+        if cols == 0:
+            raise ValueError(f"a gradient of {n} elements cannot be described as rows x cols <= 2^20")
+    return n // cols, cols
+
+
+def dmuon_clip_grad_norm_buckets(buckets: Sequence[Sequence[torch.Tensor]], max_norms: Sequence[float],
+                                 norm_types=2.0, total_norms: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Independent global-norm clips of several gradient buckets, in place (see dmuon.h).
+
+    ``buckets[k]`` is a list of contiguous CUDA gradients of any rank, clipped
+    by its own ``max_norms[k]`` and ``norm_types[k]`` (one value for all
+    buckets, or one per bucket); ``total_norms`` (float64, one per bucket)
+    receives the totals.
+    """
+    nb = len(buckets)
+    if isinstance(norm_types, (int, float)):
+        norm_types = [float(norm_types)] * nb
+    if len(max_norms) != nb or len(norm_types) != nb:
+        raise ValueError("one max_norm and one norm_type per bucket")
+    if total_norms is not None and (total_norms.dtype != torch.float64 or not total_norms.is_cuda
+                                    or not total_norms.is_contiguous() or total_norms.numel() < nb):
+        raise ValueError("total_norms must be a contiguous CUDA float64 tensor with one entry per bucket")
+    grads, bucket_of = [], []
+    for k, b in enumerate(buckets):
+        for g in b:
+            if not g.is_contiguous():
+                raise ValueError("gradients must be contiguous")
+            grads.append(g)
+            bucket_of.append(k)
+    n = len(grads)
+    dev = _device_of(*grads, total_norms) if (n or total_norms is not None) else torch.device(
+        "cuda", torch.cuda.current_device())
+    shapes = [_flat_shape(g) + (_dtype_code(g),) for g in grads]
+    ga = (ctypes.c_void_p * max(1, n))(*[g.data_ptr() for g in grads])
+    bo = (ctypes.c_int32 * max(1, n))(*bucket_of)
+    mx = (ctypes.c_float * max(1, nb))(*[float(v) for v in max_norms])
+    nt = (ctypes.c_float * max(1, nb))(*[float(v) for v in norm_types])
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.dmuon_clip_grad_norm_buckets(ga, _shape_array(shapes), n, bo, nb, mx, nt, _ptr(total_norms),
+                                                 st))
 
 
 def dmuon_plan_groups(shapes: Sequence[Tuple[int, int, int]]):

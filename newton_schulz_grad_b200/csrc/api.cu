@@ -810,6 +810,23 @@ dmuon_status_t ns_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char*
 
 using namespace dmuon;
 
+// Shapes, dtypes and pointers of the gradients of a clip; none may overlap.
+static dmuon_status_t check_clip_grads(void* const* grads, const dmuon_shape_t* shapes, int32_t count, const char* what) {
+  if (!grads || !shapes) return fail(DMUON_ERR_INVALID_ARG, "null array argument");
+  std::vector<Interval> iv;
+  for (int32_t i = 0; i < count; ++i) {
+    dmuon_status_t rc = check_shape(shapes[i].rows, shapes[i].cols, what);
+    if (rc != DMUON_OK) return rc;
+    if (!dtype_ok(shapes[i].dtype) || shapes[i].reserved != 0)
+      return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": bad dtype or reserved field");
+    if (!grads[i]) return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": null pointer");
+    const uintptr_t bytes = (uintptr_t)(shapes[i].rows * shapes[i].cols) * esize(shapes[i].dtype);
+    iv.push_back({(uintptr_t)grads[i], (uintptr_t)grads[i] + bytes, i});
+  }
+  if (any_overlap(iv)) return fail(DMUON_ERR_INVALID_ARG, "gradients must not overlap");
+  return DMUON_OK;
+}
+
 extern "C" {
 
 const char* dmuon_get_last_error(void) { return g_last_error.c_str(); }
@@ -899,6 +916,83 @@ dmuon_status_t dmuon_step_clipped(void* const* params, const void* const* grads,
                    &req, stream);
 }
 
+dmuon_status_t dmuon_clip_grad_norm_buckets(void* const* grads, const dmuon_shape_t* shapes, int32_t count,
+                                            const int32_t* bucket_of, int32_t num_buckets, const float* max_norms,
+                                            const float* norm_types, double* total_norms, dmuon_stream_t stream) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count < 0");
+  if (num_buckets < 1 || num_buckets > kMaxClipBuckets)
+    return fail(DMUON_ERR_INVALID_ARG, "num_buckets must be in 1.." + std::to_string(kMaxClipBuckets));
+  if (!max_norms || !norm_types) return fail(DMUON_ERR_INVALID_ARG, "null max_norms or norm_types");
+  std::unique_ptr<ClipBuckets> B(new ClipBuckets());
+  for (int32_t k = 0; k < num_buckets; ++k) {
+    int p = 0;
+    dmuon_status_t rc = parse_clip(max_norms[k], norm_types[k], &p);
+    if (rc != DMUON_OK) return fail(rc, "bucket " + std::to_string(k) + ": " + dmuon_get_last_error());
+    B->max_norm[k] = max_norms[k];
+    B->p[k] = p;
+  }
+  if (count > 0 && !bucket_of) return fail(DMUON_ERR_INVALID_ARG, "null bucket_of");
+  for (int32_t i = 0; i < count; ++i)
+    if (bucket_of[i] < 0 || bucket_of[i] >= num_buckets)
+      return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": bucket out of range");
+  dmuon_status_t rc = count > 0 ? check_clip_grads(grads, shapes, count, "dmuon_clip_grad_norm_buckets") : DMUON_OK;
+  if (rc != DMUON_OK) return rc;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceState ds;
+  rc = device_state(&ds);
+  if (rc != DMUON_OK) return rc;
+  // each bucket's launch classes, grouped exactly as a separate clip of that
+  // bucket would group them (member indices mapped back to the whole list)
+  std::vector<std::vector<Group>> groups(num_buckets);
+  int64_t tiles = 0;
+  for (int32_t k = 0; k < num_buckets; ++k) {
+    std::vector<int32_t> idx;
+    std::vector<dmuon_shape_t> sub;
+    for (int32_t i = 0; i < count; ++i)
+      if (bucket_of[i] == k) {
+        idx.push_back(i);
+        sub.push_back(shapes[i]);
+      }
+    groups[k] = plan_groups(sub.data(), (int32_t)sub.size());
+    for (Group& g : groups[k])
+      for (int32_t& m : g.members) m = idx[m];
+    B->off[k] = tiles;
+    tiles += clip_tiles(groups[k]);
+  }
+  B->off[num_buckets] = tiles;
+  B->total = total_norms;
+  // partials, then one coefficient per bucket
+  const size_t coef_off = (((size_t)tiles * 4 + 255) / 256) * 256;
+  void* ws = nullptr;
+  rc = get_workspace(coef_off + (size_t)num_buckets * sizeof(float), st, &ws);
+  if (rc != DMUON_OK) return rc;
+  float* partials = static_cast<float*>(ws);
+  float* coefs = reinterpret_cast<float*>(static_cast<char*>(ws) + coef_off);
+  std::unique_ptr<ElemTable> tab(new ElemTable());
+  tab->status = ds.status_word;
+  const void* const* cg = const_cast<const void* const*>(grads);
+  NvtxRange range("clip buckets");
+  cudaError_t e = cudaSuccess;
+  for (int32_t k = 0; k < num_buckets && e == cudaSuccess; ++k)
+    e = for_each_clip_table(groups[k], cg, tab.get(), [&](const ElemTable& t, int32_t dtype, int64_t off, double bytes) {
+      Prof pr(kClipNorm, st, 0.0, bytes);
+      cudaError_t r = launch_clip_partials(t, dtype, B->p[k], partials + B->off[k] + off, st);
+      pr.done(st);
+      return r;
+    });
+  // an empty bucket reduces nothing: total 0, coefficient 1
+  if (e == cudaSuccess) e = launch_clip_coef_buckets(partials, *B, num_buckets, coefs, st);
+  for (int32_t k = 0; k < num_buckets && e == cudaSuccess; ++k)
+    e = for_each_clip_table(groups[k], cg, tab.get(), [&](const ElemTable& t, int32_t dtype, int64_t, double bytes) {
+      Prof pr(kClipScale, st, 0.0, 2.0 * bytes);
+      cudaError_t r = launch_clip_scale(t, dtype, coefs + k, st);
+      pr.done(st);
+      return r;
+    });
+  return e == cudaSuccess ? DMUON_OK : cuda_fail(e, "dmuon_clip_grad_norm_buckets");
+}
+
 dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* shapes, int32_t count,
                                     float max_norm, float norm_type, double* total_norm,
                                     dmuon_stream_t stream) {
@@ -907,18 +1001,8 @@ dmuon_status_t dmuon_clip_grad_norm(void* const* grads, const dmuon_shape_t* sha
   dmuon_status_t rc = parse_clip(max_norm, norm_type, &req.p);
   if (rc != DMUON_OK) return rc;
   if (count == 0) return DMUON_OK;
-  if (!grads || !shapes) return fail(DMUON_ERR_INVALID_ARG, "null array argument");
-  std::vector<Interval> iv;
-  for (int32_t i = 0; i < count; ++i) {
-    rc = check_shape(shapes[i].rows, shapes[i].cols, "dmuon_clip_grad_norm");
-    if (rc != DMUON_OK) return rc;
-    if (!dtype_ok(shapes[i].dtype) || shapes[i].reserved != 0)
-      return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": bad dtype or reserved field");
-    if (!grads[i]) return fail(DMUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": null pointer");
-    const uintptr_t bytes = (uintptr_t)(shapes[i].rows * shapes[i].cols) * esize(shapes[i].dtype);
-    iv.push_back({(uintptr_t)grads[i], (uintptr_t)grads[i] + bytes, i});
-  }
-  if (any_overlap(iv)) return fail(DMUON_ERR_INVALID_ARG, "gradients must not overlap");
+  rc = check_clip_grads(grads, shapes, count, "dmuon_clip_grad_norm");
+  if (rc != DMUON_OK) return rc;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   DeviceState ds;

@@ -6,6 +6,10 @@
 //   coef  = min(1, max_norm / (total + 1e-6)), NaN if total is NaN;
 //   g <- fl(g * fl32(coef))
 //
+// Bucketed clipping (several independent clips at once) uses the same three
+// kinds of launch: partials of every bucket's tables, one coefficient launch
+// with one block per bucket, the scaling passes.
+//
 // Three launches, all on the caller's stream: per-chunk partials of sum |g|^p
 // (or max |g|) for every launch class of matrices; one block that reduces all
 // partials in a fixed order in fp64 and computes the coefficient; an in-place
@@ -88,10 +92,11 @@ __global__ void __launch_bounds__(kThreads, 8)
   }
 }
 
-// One block: fixed-order fp64 reduction of all partials, then the coefficient.
-__global__ void __launch_bounds__(kThreads)
-    k_clip_coef(const float* __restrict__ partials, int64_t count, int p, float max_norm, float* coef,
-                double* total_out) {
+// One block: fixed-order fp64 reduction of `count` partials, then the
+// coefficient.  The single clip and every bucket of the bucketed one run this
+// same code, so a bucket gets the bits of a separate clip of its gradients.
+__device__ __forceinline__ void clip_coef_block(const float* __restrict__ partials, int64_t count, int p,
+                                                float max_norm, float* coef, double* total_out) {
   __shared__ double red[kThreads];
   double acc = 0.0;
   for (int64_t i = threadIdx.x; i < count; i += kThreads) {
@@ -113,6 +118,20 @@ __global__ void __launch_bounds__(kThreads)
     *coef = (float)((c < 1.0 || c != c) ? c : 1.0);
     if (total_out) *total_out = total;
   }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    k_clip_coef(const float* __restrict__ partials, int64_t count, int p, float max_norm, float* coef,
+                double* total_out) {
+  clip_coef_block(partials, count, p, max_norm, coef, total_out);
+}
+
+// Block k: bucket k's partials [off[k], off[k + 1]).
+__global__ void __launch_bounds__(kThreads)
+    k_clip_coef_buckets(const float* __restrict__ partials, const __grid_constant__ ClipBuckets B, float* coefs) {
+  const int k = blockIdx.x;
+  clip_coef_block(partials + B.off[k], B.off[k + 1] - B.off[k], B.p[k], B.max_norm[k], coefs + k,
+                  B.total ? B.total + k : nullptr);
 }
 
 template <typename T>
@@ -163,6 +182,13 @@ cudaError_t launch_clip_partials(const ElemTable& t, int dtype, int p, float* pa
 cudaError_t launch_clip_coef(const float* partials, int64_t count, int p, float max_norm, float* coef,
                              double* total, cudaStream_t st) {
   k_clip_coef<<<1, kThreads, 0, st>>>(partials, count, p, max_norm, coef, total);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_clip_coef_buckets(const float* partials, const ClipBuckets& b, int num_buckets, float* coefs,
+                                     cudaStream_t st) {
+  if (num_buckets <= 0 || num_buckets > kMaxClipBuckets) return cudaErrorInvalidValue;
+  k_clip_coef_buckets<<<num_buckets, kThreads, 0, st>>>(partials, b, coefs);
   return cudaGetLastError();
 }
 

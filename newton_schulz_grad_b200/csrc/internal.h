@@ -120,6 +120,17 @@ cudaError_t launch_clip_partials(const ElemTable& t, int dtype, int p, float* pa
 cudaError_t launch_clip_coef(const float* partials, int64_t count, int p, float max_norm, float* coef,
                              double* total, cudaStream_t st);
 cudaError_t launch_clip_scale(const ElemTable& t, int dtype, const float* coef, cudaStream_t st);
+// Bucketed clipping: bucket k owns partials [off[k], off[k + 1]) and gets its
+// own coefficient (coefs[k]) and total (total[k] when total is not null).
+constexpr int kMaxClipBuckets = 128;
+struct ClipBuckets {
+  int64_t off[kMaxClipBuckets + 1];
+  float max_norm[kMaxClipBuckets];
+  int32_t p[kMaxClipBuckets];  // 2, 1, or 0 for the infinity norm
+  double* total;
+};
+cudaError_t launch_clip_coef_buckets(const float* partials, const ClipBuckets& b, int num_buckets, float* coefs,
+                                     cudaStream_t st);
 
 // ---- small_ns.cu -------------------------------------------------------------
 // The whole chain for min side m <= 64 in one launch: one cluster of 8 CTAs per

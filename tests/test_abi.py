@@ -259,3 +259,39 @@ def test_overlap_only_when_both_buffers_fit_the_cap(monkeypatch):
     ws_over, launches_over = plan(64, "1")
     ws_serial, launches_serial = plan(64, "0")
     assert ws_over <= 64 << 20 and launches_over > launches_serial
+
+
+def _raw_buckets(count, ptrs, shapes, bucket_of, nb, max_norms, norm_types):
+    lib = nsg._lib
+    arr = (ctypes.c_void_p * max(1, count))(*ptrs)
+    bo = (ctypes.c_int32 * max(1, count))(*bucket_of)
+    mx = (ctypes.c_float * max(1, nb))(*max_norms)
+    nt = (ctypes.c_float * max(1, nb))(*norm_types)
+    return lib.dmuon_clip_grad_norm_buckets(arr, nsg._shape_array(shapes), count, bo, nb, mx, nt, None, None)
+
+
+def test_clip_buckets_validation_errors():
+    # every argument check comes before any device work, so this runs on the CPU
+    A, B = 1 << 20, 1 << 21
+    ok = [(4, 8, 1), (2, 2, 0)]
+    E = nsg.DMUON_ERR_INVALID_ARG
+    assert _raw_buckets(2, [A, B], ok, [0, 1], 0, [], []) == E                        # no bucket
+    assert _raw_buckets(2, [A, B], ok, [0, 1], 129, [1.0] * 129, [2.0] * 129) == E    # too many
+    assert _raw_buckets(2, [A, B], ok, [0, 2], 2, [1.0, 1.0], [2.0, 2.0]) == E        # index out of range
+    assert _raw_buckets(2, [A, B], ok, [0, -1], 2, [1.0, 1.0], [2.0, 2.0]) == E
+    assert _raw_buckets(2, [A, B], ok, [0, 1], 2, [1.0, float("nan")], [2.0, 2.0]) == E
+    assert _raw_buckets(2, [A, B], ok, [0, 1], 2, [1.0, -1.0], [2.0, 2.0]) == E
+    assert _raw_buckets(2, [A, B], ok, [0, 1], 2, [1.0, 1.0], [2.0, 3.0]) == nsg.DMUON_ERR_UNSUPPORTED
+    assert _raw_buckets(2, [A, A + 16], ok, [0, 1], 2, [1.0, 1.0], [2.0, 2.0]) == E   # overlap across buckets
+    assert _raw_buckets(2, [A, 0], ok, [0, 1], 2, [1.0, 1.0], [2.0, 2.0]) == E
+    assert _raw_buckets(-1, [A], ok[:1], [0], 1, [1.0], [2.0]) == E
+
+
+def test_clip_buckets_binding_flat_shapes():
+    import torch
+    f = nsg._flat_shape
+    assert f(torch.empty(5, 6, 7)) == (30, 7)
+    assert f(torch.empty(4096)) == (1, 4096)
+    assert f(torch.empty(3 << 20)) == (3, 1 << 20)         # a long vector, split exactly
+    r, c = f(torch.empty(2 ** 21 + 2))
+    assert r * c == 2 ** 21 + 2 and max(r, c) <= 1 << 20

@@ -200,3 +200,82 @@ def test_clip_non_finite_gradients():
         b[0][5, 6] = float("inf")
         total, k = check_clip(b, 1.0, norm_type)
         assert math.isinf(total) and k == 0.0
+
+
+# ------------------------------------------------------------- bucketed clip
+def _bucket_set(seed):
+    # Training Guide, "Fused CUDA clip for regular / Muon / AdamW": e.g. Muon
+    # matrices, AdamW matrices and vectors, regular parameters, each a bucket
+    gen = torch.Generator().manual_seed(seed)
+
+    def t(shape, dtype, scale=1.0):
+        return (torch.randn(*shape, generator=gen) * scale).to(dtype).cuda()
+    return [
+        [t((300, 700), torch.bfloat16), t((64, 64), torch.bfloat16), t((1, 1), torch.bfloat16)],
+        [t((4096,), torch.float32), t((3, 5, 7), torch.float32, 10.0), t((129, 33), torch.bfloat16)],
+        [],
+        [t((2048, 1408), torch.bfloat16, 1e-4), t((17,), torch.float32, 1e-4)],
+        [t((1000, 3), torch.float32, 3.0)],
+    ]
+
+
+def _as2d(g):
+    return g.view(-1, g.shape[-1]) if g.dim() >= 2 else g.view(1, -1)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_clip_buckets_equal_separate_clips_bit_for_bit(seed):
+    max_norms = [1.0, 5.0, 1.0, 1e4, 0.5]
+    norm_types = [2.0, float("inf"), 2.0, 1.0, 2.0]
+    buckets = _bucket_set(30 + seed)
+    sep = [[g.clone() for g in b] for b in buckets]
+    before = [[to64(_as2d(g)) for g in b] for b in buckets]
+    totals = torch.full((5,), -1.0, dtype=torch.float64, device="cuda")
+    nsg.dmuon_clip_grad_norm_buckets(buckets, max_norms, norm_types, totals)
+    want_totals = []
+    for b, mx, nt in zip(sep, max_norms, norm_types):
+        one = torch.zeros(1, dtype=torch.float64, device="cuda")
+        nsg.dmuon_clip_grad_norm([_as2d(g) for g in b], mx, nt, one)
+        want_totals.append(float(one.item()) if b else 0.0)
+    torch.cuda.synchronize()
+    assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+    assert totals.cpu().tolist() == want_totals          # same reduction order: same bits
+    for b, s in zip(buckets, sep):
+        for g, h in zip(b, s):
+            assert np.array_equal(bits(g), bits(h))
+    # and each bucket against the oracle's separate clip
+    got = om.clip_grad_norm_buckets(before, max_norms, norm_types)
+    for k, (out, total, coef) in enumerate(got):
+        assert math.isclose(float(totals[k].item()), total, rel_tol=1e-5, abs_tol=0.0)
+        for g, w in zip(buckets[k], out):
+            err = np.abs(to64(_as2d(g)) - w).max()
+            assert err <= 2 ** -7 * np.abs(w).max() + 1e-30, (k, err)
+    assert got[3][2] == 1.0 and got[0][2] < 1.0      # one bucket under its bound, one clipped
+
+
+def test_clip_buckets_nan_stays_in_its_bucket():
+    buckets = _bucket_set(40)
+    buckets[1][2][5, 6] = float("nan")
+    keep = [bits(g) for g in buckets[3]]
+    totals = torch.zeros(5, dtype=torch.float64, device="cuda")
+    nsg.dmuon_clip_grad_norm_buckets(buckets, [1.0] * 5, 2.0, totals)
+    torch.cuda.synchronize()
+    t = totals.cpu().tolist()
+    assert math.isnan(t[1]) and all(math.isfinite(v) for k, v in enumerate(t) if k != 1)
+    assert all(torch.isnan(g).all() for g in buckets[1])
+    assert all(torch.isfinite(g).all() for k in (0, 3, 4) for g in buckets[k])
+    assert all(np.array_equal(a, bits(g)) for a, g in zip(keep, buckets[3]))  # under its bound: unchanged
+
+
+def test_clip_buckets_many_buckets_and_tables():
+    # the largest bucket count, and a bucket spanning two launch tables
+    gen = torch.Generator().manual_seed(41)
+    buckets = [[(torch.randn(4, 8 + k % 5, generator=gen) * (1 + k)).cuda()] for k in range(127)]
+    buckets.append([torch.randn(16, 24, generator=gen).cuda() for _ in range(300)])
+    sep = [[g.clone() for g in b] for b in buckets]
+    nsg.dmuon_clip_grad_norm_buckets(buckets, [1.0 + 0.01 * k for k in range(128)], 2.0)
+    for k, b in enumerate(sep):
+        nsg.dmuon_clip_grad_norm(b, 1.0 + 0.01 * k, 2.0)
+    torch.cuda.synchronize()
+    for b, s in zip(buckets, sep):
+        assert all(np.array_equal(bits(g), bits(h)) for g, h in zip(b, s))

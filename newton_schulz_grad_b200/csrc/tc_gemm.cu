@@ -506,35 +506,6 @@ __device__ __forceinline__ void epilogue_row_update(const TcArgs& a, const UpdTa
   }
 }
 
-// Before an update tile's accumulator is ready: pull the parameters it
-// rewrites into L2 (oriented rows [r0, r0 + 32) of this warp, its NCOL
-// columns from col0), so the epilogue's loads do not wait on DRAM.
-template <int NCOL>
-__device__ __forceinline__ void prefetch_update_tile(const UpdTable& u, int b, int r0, int col0, int m, int n,
-                                                     int lane) {
-  const char* p = static_cast<const char*>(u.p[b]);
-  const bool tr = (u.tmask[b >> 5] >> (b & 31)) & 1u;
-  if (r0 >= m) return;
-  if (tr) {
-    // source rows col0 .. col0 + NCOL - 1, 64 bytes (32 columns from r0) each
-#pragma unroll
-    for (int i = 0; i < NCOL / 32; ++i) {
-      const int c = col0 + lane * (NCOL / 32) + i;
-      if (c < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + ((int64_t)c * m + r0) * 2));
-    }
-  } else {
-    // row r0 + lane, 2 NCOL bytes from col0: 128-byte lines
-    const int r = r0 + lane;
-    if (r < m) {
-#pragma unroll
-      for (int i = 0; i < NCOL / 64; ++i) {
-        const int c = col0 + i * 64;
-        if (c < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + ((int64_t)r * n + c) * 2));
-      }
-    }
-  }
-}
-
 // Epilogue of one tile for one accumulator row: NCH chunks of 32 accumulator
 // columns from taddr (TMEM lane quarter of the warp), output row r, output
 // columns from cbase.  Warp-collective (tcgen05.ld).  UPD (apply only):
@@ -794,16 +765,6 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
     for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
       int b, I, J;
       decode_tile<MODE>(a, t, b, I, J);
-      if constexpr (UPD) {
-        // this CTA's first tile now, then always the next one during this epilogue
-        if (t == (int)blockIdx.x)
-          prefetch_update_tile<E::kCols>(u, b, I * BM1 + wq * 32, J * BN + half, a.m, a.n, lane);
-        if (t + (int)gridDim.x < a.total_tiles) {
-          int b2, I2, J2;
-          decode_tile<MODE>(a, t + (int)gridDim.x, b2, I2, J2);
-          prefetch_update_tile<E::kCols>(u, b2, I2 * BM1 + wq * 32, J2 * BN + half, a.m, a.n, lane);
-        }
-      }
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
       epilogue_row<MODE, UPD, false, E::kChunks>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) +
@@ -971,17 +932,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
     for (int t = pair; t < a.total_tiles; t += npairs) {
       int b, I, J;
       decode_tile<MODE>(a, t, b, I, J);
-      if constexpr (UPD) {
-        if (t == pair)
-          prefetch_update_tile<E::kCols>(u, b, I * BM2 + (int)rank * 128 + wq * 32, J * BN + half, a.m, a.n,
-                                         lane);
-        if (t + npairs < a.total_tiles) {
-          int b2, I2, J2;
-          decode_tile<MODE>(a, t + npairs, b2, I2, J2);
-          prefetch_update_tile<E::kCols>(u, b2, I2 * BM2 + (int)rank * 128 + wq * 32, J2 * BN + half, a.m,
-                                         a.n, lane);
-        }
-      }
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, a.status)) break;
       tc_fence_after();
       epilogue_row<MODE, UPD, false, E::kChunks>(a, u, tmem_base + ((uint32_t)(wq * 32) << 16) +
@@ -1011,8 +961,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
 // phase.  A tile of phase j of matrix b needs every tile of phases < j of that
 // matrix: each epilogue warp, after its stores, adds 1 (release) to the
 // matrix's counter, and the TMA producer waits (acquire, bounded by
-// %globaltimer) until the counter holds 4 x CTAs-per-tile x (tiles of the
-// earlier phases) before it loads the tile's operands.
+// %globaltimer) until the counter holds epilogue warps x CTAs-per-tile x
+// (tiles of the earlier phases) before it loads the tile's operands.
 //
 // Tiles are claimed in increasing order from one global counter (the
 // producer of each CTA, or of the pair's leader, takes the next index and
@@ -1356,33 +1306,17 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
     __syncwarp();
     if (lane == 0) release(qs);
     advance(qs, qph);
-    bool prefetched = false;  // t's update parameters were already pulled into L2
     while (t >= 0) {
       const PhaseDesc& ph = P.ph[find_phase(P, t)];
       int b, I, J;
       decode_phase_tile(ph, t, b, I, J);
       const int r0 = I * TM + (int)rank * 128 + wq * 32;
-      // the next tile (claimed ahead by the producer): its update parameters
-      // are pulled into L2 while this tile drains
+      // the next tile's index (claimed ahead by the producer), read now so the
+      // ring slot frees early
       const int tn = take(qs, qph, G == 2 && !leader);
       __syncwarp();
       if (lane == 0) release(qs);
       advance(qs, qph);
-      bool next_prefetched = false;
-      if (ph.upd) {
-        if (!prefetched) prefetch_update_tile<E::kCols>(P.u, b, r0, J * BN + half, ph.a.m, ph.a.n, lane);
-        if (tn >= 0) {
-          const PhaseDesc& pn = P.ph[find_phase(P, tn)];
-          if (pn.upd) {
-            int b2, I2, J2;
-            decode_phase_tile(pn, tn, b2, I2, J2);
-            prefetch_update_tile<E::kCols>(P.u, b2, I2 * TM + (int)rank * 128 + wq * 32, J2 * BN + half, pn.a.m,
-                                           pn.a.n, lane);
-            next_prefetched = true;
-          }
-        }
-      }
-      prefetched = next_prefetched;
       if (!wait_bar(B.tfull0 + 8 * acc, acc_phase, status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * BN + half);

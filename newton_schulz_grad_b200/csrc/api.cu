@@ -164,7 +164,7 @@ dmuon_status_t get_workspace(size_t bytes, cudaStream_t st, void** out) {
 // letting the waiting momentum blocks take the SMs as they free up (which
 // delayed the chain kernel by about the momentum kernel's whole duration).
 struct SideStreams {
-  cudaStream_t aux = nullptr, chain = nullptr;
+  cudaStream_t aux = nullptr, chain = nullptr, chain2 = nullptr;
 };
 std::map<std::pair<int, uintptr_t>, SideStreams> g_side;
 
@@ -181,8 +181,10 @@ dmuon_status_t get_side_streams(cudaStream_t st, SideStreams* out) {
     SideStreams ss;
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.aux, cudaStreamNonBlocking, least);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.chain, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.chain2, cudaStreamNonBlocking, greatest);
     if (e != cudaSuccess) {
       if (ss.aux) cudaStreamDestroy(ss.aux);
+      if (ss.chain) cudaStreamDestroy(ss.chain);
       return cuda_fail(e, "cudaStreamCreateWithPriority");
     }
     it = g_side.emplace(key, ss).first;
@@ -319,6 +321,16 @@ bool fuse_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, int32_t steps
   const std::vector<int> blocks = chain_blocks(L, steps);
   if (!tc_chain_fusable((int)m, blocks)) return false;
   return env_is("DMUON_FUSED_CHAIN", '1') || tc_chain_small(b, (int)m, (int)n, blocks);
+}
+
+// The chunk's whole chain is one launch (thin, FFMA or small tensor chain).
+// Such chains are latency-bound (a few waves of tiles per product at most),
+// so two consecutive ones run on two chain streams and share the GPU;
+// DMUON_CHAIN_STREAMS=1 keeps one stream.  Large chains keep one stream: two
+// of them at once only draw more power under the cap.
+bool one_launch_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, int32_t steps) {
+  if (env_is("DMUON_CHAIN_STREAMS", '1')) return false;
+  return thin_chain(L, m, n, steps) || fuse_ffma_chain(L, steps) || fuse_chain(L, b, m, n, steps);
 }
 
 // Executed flops of a tensor-path chain: gram m^2 n, symmetric products m^3,
@@ -625,18 +637,22 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     clip_coef = clip_coef_ptr(cws, clip_tile_count);
   }
   // when overlapping, the elementwise stages run on `aux` and the chains on
-  // `cs`; otherwise everything runs on the caller's stream
-  cudaStream_t aux = st, cs = st;
+  // `cs` (or `cs2`, see one_launch_chain); otherwise everything runs on the
+  // caller's stream
+  cudaStream_t aux = st, cs = st, cs2 = st;
   if (P.overlap) {
     SideStreams ss;
     rc = get_side_streams(st, &ss);
     if (rc != DMUON_OK) return rc;
     aux = ss.aux;
     cs = ss.chain;
+    cs2 = ss.chain2;
     cudaError_t e = stream_after(aux, st);
     if (e == cudaSuccess) e = stream_after(cs, st);
+    if (e == cudaSuccess) e = stream_after(cs2, st);
     if (e != cudaSuccess) {
       stream_after(st, aux);
+      stream_after(st, cs);
       return cuda_fail(e, "stream fork");
     }
   }
@@ -644,15 +660,16 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
   // internal streams, so a call that fails part-way leaves none of its work
   // unordered.
   struct JoinSide {
-    cudaStream_t st, aux, cs;
+    cudaStream_t st, aux, cs, cs2;
     bool on;
     ~JoinSide() {
       if (on) {
         stream_after(st, aux);
         stream_after(st, cs);
+        stream_after(st, cs2);
       }
     }
-  } join{st, aux, cs, P.overlap};
+  } join{st, aux, cs, cs2, P.overlap};
   std::vector<void*> results(P.chunks.size(), nullptr);
   std::unique_ptr<UpdTable> upd_tab(new UpdTable());
 
@@ -696,9 +713,12 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
   // aux: M0 N0 | M1 N1 U0 | M2 N2 U1 | ...   cs: chain0 | chain1 | ...
   // U(i-1) waits only for chain(i-1) (event recorded when it was enqueued);
   // M(i+1) comes after that wait, so it overwrites buffer (i+1) % 2 only once
-  // chain(i-1), which used it, is done.  Without overlap, cs and aux are the
-  // caller's stream.
+  // chain(i-1), which used it, is done.  A one-launch chain whose predecessor
+  // ran on cs runs on cs2: it waits for its own momentum (so for chain(i-2))
+  // but not for chain(i-1), which uses the other buffer.  Without overlap,
+  // cs, cs2 and aux are the caller's stream.
   cudaEvent_t chain_done = nullptr;
+  cudaStream_t prev_cs = cs2;  // stream of the previous chunk's chain
   auto drop = [&]() {
     if (chain_done) cudaEventDestroy(chain_done);  // released once complete
     chain_done = nullptr;
@@ -724,7 +744,10 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     Prof pn(kNorm, aux, 0.0, 4.0 * (double)ck.b * (double)L.tiles_per_mat);
     e = launch_norm_finalize(partials, ck.b, (int)L.tiles_per_mat, scale, nullptr, aux);
     pn.done(aux);
-    if (e == cudaSuccess && P.overlap) e = stream_after(cs, aux);
+    const cudaStream_t csi =
+        (P.overlap && prev_cs == cs && one_launch_chain(L, ck.b, c.m, c.n, ns_steps)) ? cs2 : cs;
+    prev_cs = csi;
+    if (e == cudaSuccess && P.overlap) e = stream_after(csi, aux);
     if (e != cudaSuccess) {
       drop();
       return cuda_fail(e, "norm launch / stream join");
@@ -750,8 +773,8 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     }
     {
       NvtxRange r("chain " + std::to_string(c.m) + "x" + std::to_string(c.n) + " x" + std::to_string(ck.b));
-      rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched.data(), ds.status_word, ds.sm_count, cs, &results[i],
-                     upd);
+      rc = run_chain(L, ck.b, c.m, c.n, ws, off, ns_steps, sched.data(), ds.status_word, ds.sm_count, csi,
+                     &results[i], upd);
     }
     if (rc != DMUON_OK) {
       drop();
@@ -776,7 +799,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     }
     drop();
     e = cudaEventCreateWithFlags(&chain_done, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventRecord(chain_done, cs);
+    if (e == cudaSuccess) e = cudaEventRecord(chain_done, csi);
     if (e != cudaSuccess) {
       drop();
       return cuda_fail(e, "chain event");
@@ -791,6 +814,7 @@ dmuon_status_t step_impl(void* const* params, const void* const* grads, void* co
     join.on = false;
     e = stream_after(st, aux);
     if (e == cudaSuccess) e = stream_after(st, cs);
+    if (e == cudaSuccess) e = stream_after(st, cs2);
     if (e != cudaSuccess) return cuda_fail(e, "stream join");
   }
   return DMUON_OK;

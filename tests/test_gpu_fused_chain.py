@@ -197,3 +197,29 @@ def test_epilogue_width_gives_the_same_bits(shape, fused, monkeypatch):
         assert nsg.dmuon_stream_status() == nsg.DMUON_OK
         outs.append((bits(o), bits(p)))
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("name,idx,cap", [("small_layer_bf16", None, None),
+                                          ("small_layer_bf16", None, "64"),
+                                          ("moe_skewed_bf16", [0, 1, 2, 3, 4, 5, 192, 193, 240, 241], "256"),
+                                          ("single_256x512_f32", None, None)])
+def test_two_chain_streams_give_the_same_bits(name, idx, cap, monkeypatch):
+    # consecutive one-launch chains of a step run on two chain streams at
+    # once; they read and write disjoint buffers, so one stream or two must
+    # give the same bits (several chunks per class with the small cap)
+    w = workloads.get(name)
+    sk = workloads.skewed_indices(w)
+    idx = list(range(w.count)) if idx is None else idx
+    if cap:
+        monkeypatch.setenv("DMUON_WS_CAP_MB", cap)
+    runs = []
+    for streams in ("2", "1"):
+        monkeypatch.setenv("DMUON_CHAIN_STREAMS", streams)
+        mats = [workloads.make_matrix(w, i, "cuda", sk) for i in idx]
+        ps, gs, bs = [m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats]
+        for _ in range(2):                      # two steps: the second reuses the buffers
+            nsg.dmuon_step(ps, gs, bs, wd=w.wd)
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        runs.append([bits(t) for t in ps + bs])
+    for a, b in zip(*runs):
+        assert np.array_equal(a, b)

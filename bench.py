@@ -745,7 +745,8 @@ def run_stage(args):
         X = torch.randn(b, m, n, generator=gen, device=dev).to(bf)
         out = torch.empty_like(X)
         if args.stage == "apply":
-            run = lambda: nsg.dmuon_poly_apply(P, X, out, 3.4445)  # noqa: E731
+            # as in the step: the tensor path's p(G) carries a I, so its applies add no a X
+            run = lambda: nsg.dmuon_poly_apply(P, X, out, 0.0)  # noqa: E731
         elif args.lib == "quack":  # comparison only: the same product through quack
             from quack.gemm_interface import gemm_add
             run = lambda: gemm_add(P, X, C=X, out=out, alpha=1.0, beta=3.4445, tuned=False)  # noqa: E731

@@ -443,7 +443,10 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   }
 
   // Blocks of iterations (chain_blocks).  A block of one is the iteration as
-  // written: G = X X^T, P = b G + c G G, X <- a X + P X.  In a longer block
+  // written: G = X X^T, then X <- p(G) X.  The tensor path stores p(G) =
+  // a I + b G + c G G (the identity term in the polynomial's epilogue) and
+  // applies it as one product; the FFMA path keeps P = b G + c G G and adds
+  // a X in the apply's epilogue (X <- a X + P X).  In a longer block
   // every matrix is a polynomial of the block's Gram matrix G:
   //   P_j = p_j(G_j) (with a I),  G_{j+1} = P_j G_j P_j,  Q = P_j ... P_0,
   // and the block ends with X <- Q X (a fresh G starts the next block).
@@ -454,14 +457,15 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
     if (len == 1) {
       gram(cur, G, sc);
       if (e != cudaSuccess) break;
-      {
-        Prof p(tc ? kPolyTc : kPolyFfma, st, fb * fm * fm * fm, 0.0);
-        e = tc ? tc_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), sw, sms, st)
-               : simt_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), st, sw);
+      if (tc) {
+        symm(G, G, G, P, coef(k, 1), coef(k, 2), coef(k, 0), kPolyTc);  // P = a I + b G + c G G
+      } else {
+        Prof p(kPolyFfma, st, fb * fm * fm * fm, 0.0);
+        e = simt_poly(G, P, b, mi, L.ldm, L.ldm, coef(k, 1), coef(k, 2), st, sw);
         p.done(st);
       }
       if (e != cudaSuccess) break;
-      apply(P, cur, nxt, coef(k, 0), sc, k + 1 == steps);
+      apply(P, cur, nxt, tc ? 0.f : coef(k, 0), sc, k + 1 == steps);
       std::swap(cur, nxt);
       k += 1;
       continue;

@@ -1712,9 +1712,10 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
     const bool fuse = last && upd != nullptr;
     const float* c = sched + 3 * k;
     if (len == 1) {
+      // G, P = a I + b G + c G G, X <- P X (the per-product launches' schedule)
       add(gram_args(S(0), batch, m, n, ldm, 1.f, sc, status, pair), kGram, kMapX0 + cur, kMapX0 + cur, 0);
-      add(symm_args(S(0), S(1), batch, m, ldm, ldm, c[1], c[2], 0.f, status, pair), kPoly, kMapS0, kMapS0, 0);
-      add(apply_args(buf.x[cur], fuse ? nullptr : buf.x[1 - cur], batch, m, n, ldn, ldn, c[0], 1.f, sc, status, pair),
+      add(symm_args(S(0), S(1), batch, m, ldm, ldm, c[1], c[2], c[0], status, pair), kPoly, kMapS0, kMapS0, 0);
+      add(apply_args(buf.x[cur], fuse ? nullptr : buf.x[1 - cur], batch, m, n, ldn, ldn, 0.f, 1.f, sc, status, pair),
           kApply, kMapS0 + 1, kMapX0mn + cur, fuse ? 1 : 0);
     } else {
       const float* c1 = sched + 3 * (k + 1);

@@ -364,11 +364,14 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
   const double fm = (double)m, fn = (double)n, fb = (double)b;
   const int mi = (int)m, ni = (int)n;
   cudaError_t e = cudaSuccess;
+  // the chain's symmetric matrices are stored as their lower 256-column blocks
+  // and read back so (DMUON_LOWER_STORE=0: stored in full)
+  const bool low = !env_is("DMUON_LOWER_STORE", '0');
   // m x m slot s of the chunk (slot 0 is G, the rest follow P)
   auto slot = [&](int s) -> char* { return s == 0 ? (char*)G : (char*)P + (int64_t)(s - 1) * ((off.p - off.g)); };
   auto gram = [&](const void* X, void* out, const float* sc) {
     Prof p(tc ? kGramTc : kGramFfma, st, fb * fm * fm * fn, 0.0);
-    e = tc ? tc_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, sw, sms, st)
+    e = tc ? tc_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, sw, sms, st, low)
            : simt_gram(X, out, b, mi, ni, L.ldn, L.ldm, 1.f, sc, xbf16, st, sw);
     p.done(st);
   };
@@ -377,20 +380,20 @@ dmuon_status_t run_chain(const ChunkLayout& L, int b, int64_t m, int64_t n, char
     if (tc && last && upd) {
       // update bytes: read and write p
       Prof p(kApplyUpdTc, st, 2.0 * fb * fm * fm * fn, 4.0 * fb * fm * fn);
-      e = tc_apply_update(Pm, X, b, mi, ni, L.ldm, L.ldn, a, 1.f, sc, *upd, sw, sms, st);
+      e = tc_apply_update(Pm, X, b, mi, ni, L.ldm, L.ldn, a, 1.f, sc, *upd, sw, sms, st, low);
       p.done(st);
       fused = true;
       return;
     }
     Prof p(tc ? kApplyTc : kApplyFfma, st, 2.0 * fb * fm * fm * fn, 0.0);
-    e = tc ? tc_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, sw, sms, st)
+    e = tc ? tc_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, sw, sms, st, low)
            : simt_apply(Pm, X, Y, b, mi, ni, L.ldm, L.ldn, L.ldn, a, 1.f, sc, xbf16, st, sw);
     p.done(st);
   };
   // C = p1 (A B) + p0 E + p2 I on the tensor path (A, B symmetric and commuting)
   auto symm = [&](const void* A, const void* B, const void* E, void* C, float p0, float p1, float p2, int kind) {
     Prof p(kind, st, fb * fm * fm * fm, 0.0);
-    e = tc_symm(A, B, E, C, b, mi, L.ldm, L.ldm, L.ldm, L.ldm, p0, p1, p2, sw, sms, st);
+    e = tc_symm(A, B, E, C, b, mi, L.ldm, L.ldm, L.ldm, L.ldm, p0, p1, p2, sw, sms, st, low);
     p.done(st);
   };
   const auto coef = [&](int k, int i) { return sched[3 * k + i]; };

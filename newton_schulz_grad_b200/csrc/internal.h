@@ -144,18 +144,24 @@ cudaError_t small_ns(void* X, int batch, int m, int n, int64_t ld, int steps, co
 
 // ---- tc_gemm.cu -------------------------------------------------------------
 // tcgen05 chain kernels (bf16 in/out, fp32 accumulation in TMEM).
+// Inside a chain the symmetric matrices (G, p(G) and the Gram-space products)
+// may be stored as their lower 256-column blocks only (lower = true: the
+// producer skips the mirror stores outside the diagonal blocks) and read so
+// by their consumers (lower / lower_p = true: the operand's upper k-blocks
+// are loaded as the transposed lower block).  The stage calls store and read
+// full matrices.
 cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,
-                    float alpha, const float* scale, int* status, int num_sms, cudaStream_t st);
+                    float alpha, const float* scale, int* status, int num_sms, cudaStream_t st, bool lower = false);
 cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b,
                     float c, int* status, int num_sms, cudaStream_t st);
 // C = p1 (A B) + p0 E + p2 I for symmetric, commuting A, B (E may be NULL);
 // one triangle computed, mirrored.
 cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int batch, int m, int64_t lda,
                     int64_t ldb, int64_t lde, int64_t ldc, float p0, float p1, float p2, int* status,
-                    int num_sms, cudaStream_t st);
+                    int num_sms, cudaStream_t st, bool lower = false);
 cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
                      int64_t ldx, int64_t ldy, float a, float alpha, const float* scale,
-                     int* status, int num_sms, cudaStream_t st);
+                     int* status, int num_sms, cudaStream_t st, bool lower_p = false);
 
 // The parameter update fused into the last apply of the chain: for matrix b
 // of the launch, O = bf16(alpha (a X + P X)) (the value tc_apply would store)
@@ -170,7 +176,7 @@ struct UpdTable {
 };
 cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int n, int64_t ldp, int64_t ldx,
                             float a, float alpha, const float* scale, const UpdTable& u, int* status,
-                            int num_sms, cudaStream_t st);
+                            int num_sms, cudaStream_t st, bool lower_p = false);
 // The whole chain of a chunk in one persistent launch (tensor path): every
 // product of the iteration blocks `blocks` (chain_blocks) in order, per-matrix
 // dependency counters between them.  x[0] holds X at entry; slot[0..4] are

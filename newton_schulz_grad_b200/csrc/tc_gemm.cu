@@ -116,7 +116,20 @@ struct TcArgs {
   float p0, p1, p2;  // gram: alpha; poly: p1 (A B) + p0 E + p2 I; apply: alpha (p0 X + P X)
   const float* scale;
   int* status;
+  // Symmetric matrices inside a chain are stored as their lower 256-column
+  // blocks only: an element (r, c) is written where c / 256 <= r / 256 (the
+  // diagonal 256 x 256 blocks in full).  lower: this launch's symmetric output
+  // is stored that way (no mirror stores outside the diagonal blocks).  sym
+  // bit 0 / bit 1: operand A / B is such a matrix; its k-blocks right of the
+  // operand's own 256-block are read as the transposed lower block.
+  int lower, sym;
 };
+
+// First k-block (of BK = 64) of a tile's operand that lies right of the
+// operand's 256-row block, i.e. in the unstored upper part: from there on the
+// operand is read transposed (MN-major).  Beyond every k-block when the
+// operand is stored in full.
+__device__ __forceinline__ int upper_kb(bool sym, int row0) { return sym ? 4 * ((row0 >> 8) + 1) : 0x7fffffff; }
 
 // Matrices in the launch (extent checks of debug builds).
 [[maybe_unused]] __device__ __forceinline__ int64_t batch_of(const TcArgs& a) { return a.total_tiles / a.tiles_per_mat; }
@@ -311,6 +324,8 @@ __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int M) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Operand-major bits of the instruction descriptor (bit 15: A, bit 16: B).
+constexpr uint32_t kIdescAMn = 1u << 15, kIdescBMn = 1u << 16;
 
 // Tile t -> (matrix b, row block I, column block J).
 template <int MODE>
@@ -594,6 +609,7 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& a, const typename Upd
       if (full_chunk && r > c0 + 31) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(rowp)[q] = pack_bf16x8(v + 8 * q);
+        if (a.lower && (c0 >> 8) != (r >> 8)) continue;  // the mirror lies outside the stored blocks
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (DMUON_IN(a.status, (int64_t)b * a.sC + (int64_t)(c0 + j) * a.ldc + r, 1, batch_of(a) * a.sC) &&
@@ -632,7 +648,8 @@ __device__ __forceinline__ Bars bar_layout(uint64_t* bars) {
 template <int MODE, bool UPD, int EPI>
 __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
     k_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-         const TcArgs a, const __grid_constant__ typename UpdSel<UPD>::type u) {
+         const __grid_constant__ CUtensorMap tmAt, const __grid_constant__ CUtensorMap tmBt, const TcArgs a,
+         const __grid_constant__ typename UpdSel<UPD>::type u) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -685,10 +702,18 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
           mbar_arrive_expect_tx(fb, STAGE1_BYTES);
           const uint32_t sa = smem_u32(smem + stage * STAGE1_BYTES);
           const uint32_t sb = sa + A1_BYTES;
-          tma_load_3d(sa, &tmA, fb, kb * BK, I * BM1, b);
+          if (kb >= upper_kb(MODE != kGram && (a.sym & 1), I * BM1)) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) tma_load_3d(sa + q * 8192, &tmAt, fb, I * BM1 + q * 64, kb * BK, b);
+          } else {
+            tma_load_3d(sa, &tmA, fb, kb * BK, I * BM1, b);
+          }
           if (MODE == kApply) {
 #pragma unroll
             for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmB, fb, J * BN + q * 64, kb * BK, b);
+          } else if (kb >= upper_kb(MODE == kPoly && (a.sym & 2), J * BN)) {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmBt, fb, J * BN + q * 64, kb * BK, b);
           } else {
             tma_load_3d(sb, &tmB, fb, kb * BK, J * BN, b);
           }
@@ -711,15 +736,26 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
       // ----------------------------------------------------------------- MMA
       constexpr uint32_t idesc = make_idesc(MODE == kApply, BM1);
       // stage 0, k-step 0; every other descriptor adds an offset to these
+      // (K-major: 16-row k-steps are 32 bytes apart; MN-major: 2048 bytes)
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t a_desc0_t = sdesc_sw128(smem_u32(smem), 8192, 1024);
       const uint64_t b_desc0 = (MODE == kApply) ? sdesc_sw128(smem_u32(smem) + A1_BYTES, 8192, 1024)
                                                 : sdesc_sw128(smem_u32(smem) + A1_BYTES, 16, 1024);
+      const uint64_t b_desc0_t = sdesc_sw128(smem_u32(smem) + A1_BYTES, 8192, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
+        // the k-blocks from which a lower-stored symmetric operand is read transposed
+        int ka = 0x7fffffff, kbt = 0x7fffffff;
+        if (MODE != kGram && a.sym) {
+          int b, I, J;
+          decode_tile<MODE>(a, t, b, I, J);
+          ka = upper_kb(a.sym & 1, I * BM1);
+          kbt = upper_kb(MODE == kPoly && (a.sym & 2), J * BN);
+        }
         if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
@@ -731,12 +767,15 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
           tc_fence_after();
           // descriptors of this stage: the bases plus the stage offset (16-byte units)
           const uint64_t soff = (uint64_t)((stage * STAGE1_BYTES) >> 4);
+          const bool at = kb >= ka, bt = kb >= kbt;
+          const uint64_t a0 = (at ? a_desc0_t : a_desc0) + soff;
+          const uint64_t b0 = (bt ? b_desc0_t : b_desc0) + soff;
+          const uint32_t astep = at ? UK * 128 / 16 : UK * 2 / 16;
+          const uint32_t bstep = (MODE == kApply || bt) ? UK * 128 / 16 : UK * 2 / 16;
+          const uint32_t id = idesc | (at ? kIdescAMn : 0u) | (bt ? kIdescBMn : 0u);
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k) {
-            const uint64_t ad = a_desc0 + soff + (uint64_t)(k * (UK * 2 / 16));
-            const uint64_t bd = b_desc0 + soff + (uint64_t)(k * ((MODE == kApply ? UK * 128 : UK * 2) / 16));
-            tc_mma<1>(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / UK; ++k)
+            tc_mma<1>(d, a0 + (uint64_t)(k * astep), b0 + (uint64_t)(k * bstep), id, (kb | k) != 0 ? 1u : 0u);
           tc_commit<1>(B.empty0 + 8 * stage);
           if (++stage == STAGES1) {
             stage = 0;
@@ -790,7 +829,8 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
 template <int MODE, bool UPD, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 1)
     k_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const TcArgs a, const __grid_constant__ typename UpdSel<UPD>::type u) {
+          const __grid_constant__ CUtensorMap tmAt, const __grid_constant__ CUtensorMap tmBt, const TcArgs a,
+          const __grid_constant__ typename UpdSel<UPD>::type u) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -848,11 +888,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
           const uint32_t fb = full_leader0 + 8 * stage;
           const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
           const uint32_t sb = sa + A2_BYTES;
-          tma_load_3d_pair(sa, &tmA, fb, kb * BK, I * BM2 + (int)rank * 128, b);
+          if (kb >= upper_kb(MODE != kGram && (a.sym & 1), I * BM2)) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+              tma_load_3d_pair(sa + q * 8192, &tmAt, fb, I * BM2 + (int)rank * 128 + q * 64, kb * BK, b);
+          } else {
+            tma_load_3d_pair(sa, &tmA, fb, kb * BK, I * BM2 + (int)rank * 128, b);
+          }
           if (MODE == kApply) {
 #pragma unroll
             for (int q = 0; q < 2; ++q)
               tma_load_3d_pair(sb + q * 8192, &tmB, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
+          } else if (kb >= upper_kb(MODE == kPoly && (a.sym & 2), J * BN)) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+              tma_load_3d_pair(sb + q * 8192, &tmBt, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
           } else {
             tma_load_3d_pair(sb, &tmB, fb, kb * BK, J * BN + (int)rank * 128, b);
           }
@@ -877,15 +927,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
       // ------------------------------------------------------ MMA (leader)
       constexpr uint32_t idesc = make_idesc(MODE == kApply, BM2);
       // stage 0, k-step 0; every other descriptor adds an offset to these
+      // (K-major: 16-row k-steps are 32 bytes apart; MN-major: 2048 bytes)
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t a_desc0_t = sdesc_sw128(smem_u32(smem), 8192, 1024);
       const uint64_t b_desc0 = (MODE == kApply) ? sdesc_sw128(smem_u32(smem) + A2_BYTES, 8192, 1024)
                                                 : sdesc_sw128(smem_u32(smem) + A2_BYTES, 16, 1024);
+      const uint64_t b_desc0_t = sdesc_sw128(smem_u32(smem) + A2_BYTES, 8192, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = pair; ok && t < a.total_tiles; t += npairs) {
+        // the k-blocks from which a lower-stored symmetric operand is read
+        // transposed (the same for both CTAs: their rows share a 256-block)
+        int ka = 0x7fffffff, kbt = 0x7fffffff;
+        if (MODE != kGram && a.sym) {
+          int b, I, J;
+          decode_tile<MODE>(a, t, b, I, J);
+          ka = upper_kb(a.sym & 1, I * BM2);
+          kbt = upper_kb(MODE == kPoly && (a.sym & 2), J * BN);
+        }
         if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
@@ -897,12 +959,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
           tc_fence_after();
           // descriptors of this stage: the bases plus the stage offset (16-byte units)
           const uint64_t soff = (uint64_t)((stage * STAGE2_BYTES) >> 4);
+          const bool at = kb >= ka, bt = kb >= kbt;
+          const uint64_t a0 = (at ? a_desc0_t : a_desc0) + soff;
+          const uint64_t b0 = (bt ? b_desc0_t : b_desc0) + soff;
+          const uint32_t astep = at ? UK * 128 / 16 : UK * 2 / 16;
+          const uint32_t bstep = (MODE == kApply || bt) ? UK * 128 / 16 : UK * 2 / 16;
+          const uint32_t id = idesc | (at ? kIdescAMn : 0u) | (bt ? kIdescBMn : 0u);
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k) {
-            const uint64_t ad = a_desc0 + soff + (uint64_t)(k * (UK * 2 / 16));
-            const uint64_t bd = b_desc0 + soff + (uint64_t)(k * ((MODE == kApply ? UK * 128 : UK * 2) / 16));
-            tc_mma<2>(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / UK; ++k)
+            tc_mma<2>(d, a0 + (uint64_t)(k * astep), b0 + (uint64_t)(k * bstep), id, (kb | k) != 0 ? 1u : 0u);
           tc_commit_pair(B.empty0 + 8 * stage, 0x3);
           if (++stage == STAGES2) {
             stage = 0;
@@ -1481,8 +1546,9 @@ int epi_warps(int64_t k) {
 }
 
 template <int MODE, bool UPD, int EPI>
-cudaError_t launch_epi(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a, int64_t total, int num_sms,
-                       bool pair, cudaStream_t st, const typename UpdSel<UPD>::type& u) {
+cudaError_t launch_epi(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mat, const CUtensorMap& mbt,
+                       const TcArgs& a, int64_t total, int num_sms, bool pair, cudaStream_t st,
+                       const typename UpdSel<UPD>::type& u) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -1495,23 +1561,26 @@ cudaError_t launch_epi(const CUtensorMap& ma, const CUtensorMap& mb, const TcArg
   if (pair) {
     const int units = max_pair_units(num_sms);
     const int64_t pairs = total < units ? total : units;
-    k_tc2<MODE, UPD, EPI><<<(int)(2 * pairs), Epi<EPI>::kThreads, SMEM2_BYTES, st>>>(ma, mb, a, u);
+    k_tc2<MODE, UPD, EPI><<<(int)(2 * pairs), Epi<EPI>::kThreads, SMEM2_BYTES, st>>>(ma, mb, mat, mbt, a, u);
   } else {
     const int grid = (int)(total < num_sms ? total : num_sms);
-    k_tc<MODE, UPD, EPI><<<grid, Epi<EPI>::kThreads, SMEM1_BYTES, st>>>(ma, mb, a, u);
+    k_tc<MODE, UPD, EPI><<<grid, Epi<EPI>::kThreads, SMEM1_BYTES, st>>>(ma, mb, mat, mbt, a, u);
   }
   return cudaGetLastError();
 }
 
+// mat / mbt: MN-major {64 x 64} maps of operands A / B, read where a.sym
+// says they are lower-stored symmetric matrices (otherwise unused).
 template <int MODE, bool UPD = false>
-cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs& a, int batch, int num_sms, bool pair,
-                   cudaStream_t st, const typename UpdSel<UPD>::type& u = {}) {
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mat, const CUtensorMap& mbt,
+                   TcArgs& a, int batch, int num_sms, bool pair, cudaStream_t st,
+                   const typename UpdSel<UPD>::type& u = {}) {
   const int64_t total = (int64_t)a.tiles_per_mat * batch;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffff) return cudaErrorInvalidValue;
   a.total_tiles = (int)total;
-  if (epi_warps(a.k) == 8) return launch_epi<MODE, UPD, 8>(ma, mb, a, total, num_sms, pair, st, u);
-  return launch_epi<MODE, UPD, 4>(ma, mb, a, total, num_sms, pair, st, u);
+  if (epi_warps(a.k) == 8) return launch_epi<MODE, UPD, 8>(ma, mb, mat, mbt, a, total, num_sms, pair, st, u);
+  return launch_epi<MODE, UPD, 4>(ma, mb, mat, mbt, a, total, num_sms, pair, st, u);
 }
 
 // Arguments of each product; the per-product launches and the fused chain
@@ -1584,7 +1653,7 @@ TcArgs apply_args(const void* X, void* Y, int batch, int m, int n, int64_t ldx, 
 }  // namespace
 
 cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg, float alpha,
-                    const float* scale, int* status, int num_sms, cudaStream_t st) {
+                    const float* scale, int* status, int num_sms, cudaStream_t st, bool lower) {
   if (batch == 0) return cudaSuccess;
   const bool pair = use_pair(m, true);
   CUtensorMap ma, mb;
@@ -1593,52 +1662,63 @@ cudaError_t tc_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, BK, pair ? 128 : BN);
   if (e != cudaSuccess) return e;
   TcArgs a = gram_args(G, batch, m, n, ldg, alpha, scale, status, pair);
-  return launch<kGram>(ma, mb, a, batch, num_sms, pair, st);
+  a.lower = lower ? 1 : 0;
+  return launch<kGram>(ma, mb, ma, mb, a, batch, num_sms, pair, st);
 }
 
 cudaError_t tc_symm(const void* A, const void* B, const void* E, void* C, int batch, int m, int64_t lda,
                     int64_t ldb, int64_t lde, int64_t ldc, float p0, float p1, float p2, int* status, int num_sms,
-                    cudaStream_t st) {
+                    cudaStream_t st, bool lower) {
   if (batch == 0) return cudaSuccess;
   const bool pair = use_pair(m, true);
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mat, mbt;
   cudaError_t e = make_map(&ma, A, m, m, batch, lda, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, B, m, m, batch, ldb, BK, pair ? 128 : BN);
+  // lower-stored operands: their upper k-blocks are read as transposed {64 x 64} boxes
+  if (e == cudaSuccess && lower) e = make_map(&mat, A, m, m, batch, lda, 64, BK);
+  if (e == cudaSuccess && lower) e = make_map(&mbt, B, m, m, batch, ldb, 64, BK);
   if (e != cudaSuccess) return e;
   TcArgs a = symm_args(E, C, batch, m, lde, ldc, p0, p1, p2, status, pair);
-  return launch<kPoly>(ma, mb, a, batch, num_sms, pair, st);
+  a.lower = lower ? 1 : 0;
+  a.sym = lower ? 3 : 0;
+  return lower ? launch<kPoly>(ma, mb, mat, mbt, a, batch, num_sms, pair, st)
+               : launch<kPoly>(ma, mb, ma, mb, a, batch, num_sms, pair, st);
 }
 
 cudaError_t tc_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b, float c,
                     int* status, int num_sms, cudaStream_t st) {
-  return tc_symm(G, G, G, P, batch, m, ldg, ldg, ldg, ldp, b, c, 0.f, status, num_sms, st);
+  return tc_symm(G, G, G, P, batch, m, ldg, ldg, ldg, ldp, b, c, 0.f, status, num_sms, st, false);
 }
 
 cudaError_t tc_apply(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp,
                      int64_t ldx, int64_t ldy, float a_coef, float alpha, const float* scale, int* status,
-                     int num_sms, cudaStream_t st) {
+                     int num_sms, cudaStream_t st, bool lower_p) {
   if (batch == 0) return cudaSuccess;
   const bool pair = use_pair(m, false);
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mat;
   cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
+  if (e == cudaSuccess && lower_p) e = make_map(&mat, P, m, m, batch, ldp, 64, BK);
   if (e != cudaSuccess) return e;
   TcArgs a = apply_args(X, Y, batch, m, n, ldx, ldy, a_coef, alpha, scale, status, pair);
-  return launch<kApply>(ma, mb, a, batch, num_sms, pair, st);
+  a.sym = lower_p ? 1 : 0;
+  return launch<kApply>(ma, mb, lower_p ? mat : ma, mb, a, batch, num_sms, pair, st);
 }
 
 cudaError_t tc_apply_update(const void* P, const void* X, int batch, int m, int n, int64_t ldp, int64_t ldx,
                             float a_coef, float alpha, const float* scale, const UpdTable& u, int* status,
-                            int num_sms, cudaStream_t st) {
+                            int num_sms, cudaStream_t st, bool lower_p) {
   if (batch == 0) return cudaSuccess;
   if (batch > kMaxTable) return cudaErrorInvalidValue;
   const bool pair = use_pair(m, false);
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mat;
   cudaError_t e = make_map(&ma, P, m, m, batch, ldp, BK, 128);
   if (e == cudaSuccess) e = make_map(&mb, X, n, m, batch, ldx, 64, BK);
+  if (e == cudaSuccess && lower_p) e = make_map(&mat, P, m, m, batch, ldp, 64, BK);
   if (e != cudaSuccess) return e;
   TcArgs a = apply_args(X, nullptr, batch, m, n, ldx, 0, a_coef, alpha, scale, status, pair);
-  return launch<kApply, true>(ma, mb, a, batch, num_sms, pair, st, u);
+  a.sym = lower_p ? 1 : 0;
+  return launch<kApply, true>(ma, mb, lower_p ? mat : ma, mb, a, batch, num_sms, pair, st, u);
 }
 
 bool tc_chain_fusable(int m, const std::vector<int>& blocks) {

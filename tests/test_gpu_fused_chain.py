@@ -223,3 +223,28 @@ def test_two_chain_streams_give_the_same_bits(name, idx, cap, monkeypatch):
         runs.append([bits(t) for t in ps + bs])
     for a, b in zip(*runs):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("shape", [(4096, 4096), (1408, 2048), (2048, 1408), (1024, 2816), (300, 700), (520, 1300),
+                                   (768, 768)], ids=lambda s: f"{s[0]}x{s[1]}")
+def test_lower_stored_symmetric_matrices_give_the_same_bits(shape, monkeypatch):
+    # the per-product chain stores G, p(G) and the Gram-space products as
+    # their lower 256-column blocks and reads the upper part of each operand
+    # as the transposed lower block; storing them in full must give the same
+    # bits (same operand values, same products), in Newton-Schulz and in a
+    # step with the fused update
+    monkeypatch.setenv("DMUON_FUSED_CHAIN", "0")
+    X = seeded(shape, 5 * shape[0] + shape[1])
+    p0 = seeded(shape, 17 + shape[0], 0.02)
+    g = seeded(shape, 19 + shape[1])
+    outs = []
+    for low in ("1", "0"):
+        monkeypatch.setenv("DMUON_LOWER_STORE", low)
+        o = torch.empty_like(X)
+        nsg.dmuon_ns(X, o)
+        p, b = p0.clone(), torch.zeros_like(p0)
+        nsg.dmuon_step([p], [g], [b], wd=0.1)
+        assert nsg.dmuon_stream_status() == nsg.DMUON_OK
+        outs.append((bits(o), bits(p)))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    assert rel_fro(to64(o), om.newton_schulz(to64(X), 5)) < 2e-2

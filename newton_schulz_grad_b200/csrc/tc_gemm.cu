@@ -1040,19 +1040,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
 // already done, and the chain pays one launch instead of one per product.
 constexpr int kMaxPhases = 32;
 constexpr int kRing = 4;
-enum { kMapX0 = 0, kMapX1 = 1, kMapS0 = 2, kMapX0mn = 7, kMapX1mn = 8, kChainMaps = 9 };
+enum { kMapX0 = 0, kMapX1 = 1, kMapS0 = 2, kMapX0mn = 7, kMapX1mn = 8, kMapS0t = 9, kChainMaps = 14 };
 
 struct PhaseDesc {
   TcArgs a;
   int mode;        // kGram, kPoly (symmetric products) or kApply
   int upd;         // apply whose epilogue updates the parameters
   int mapA, mapB;  // tensor maps of the operands
+  int mapAt, mapBt;  // their MN-major maps, for the transposed reads of lower-stored operands
   int tile_start;  // global index of the phase's first tile
   uint32_t dep;    // counter value (per matrix) the phase's tiles wait for
 };
 
 struct ChainParams {
-  CUtensorMap maps[kChainMaps];  // K-major {64 x 128} for X0, X1, S0..S4; MN-major {64 x 64} for X0, X1
+  CUtensorMap maps[kChainMaps];  // K-major {64 x 128} for X0, X1, S0..S4; MN-major {64 x 64} for X0, X1, S0..S4
   PhaseDesc ph[kMaxPhases];
   UpdTable u;
   unsigned* counters;  // one per matrix, then the tile counter; all zero at launch
@@ -1250,6 +1251,10 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
         }
         const CUtensorMap* mA = &P.maps[ph.mapA];
         const CUtensorMap* mB = &P.maps[ph.mapB];
+        const CUtensorMap* mAt = &P.maps[ph.mapAt];
+        const CUtensorMap* mBt = &P.maps[ph.mapBt];
+        const int ka = upper_kb(ph.a.sym & 1, I * TM);
+        const int kbt = upper_kb(ph.mode == kPoly && (ph.a.sym & 2), J * BN);
         const int num_kb = (ph.a.k + BK - 1) / BK;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, status)) {
@@ -1261,19 +1266,37 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
           if constexpr (G == 2) {
-            tma_load_3d_pair(sa, mA, fb, kb * BK, I * TM + (int)rank * 128, b);
+            if (kb >= ka) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                tma_load_3d_pair(sa + q * 8192, mAt, fb, I * TM + (int)rank * 128 + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d_pair(sa, mA, fb, kb * BK, I * TM + (int)rank * 128, b);
+            }
             if (ph.mode == kApply) {
 #pragma unroll
               for (int q = 0; q < 2; ++q)
                 tma_load_3d_pair(sb + q * 8192, mB, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
+            } else if (kb >= kbt) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                tma_load_3d_pair(sb + q * 8192, mBt, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
             } else {
               tma_load_3d_pair(sb, mB, fb, kb * BK, J * BN + (int)rank * 128, b);
             }
           } else {
-            tma_load_3d(sa, mA, fb, kb * BK, I * TM, b);
+            if (kb >= ka) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q) tma_load_3d(sa + q * 8192, mAt, fb, I * TM + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d(sa, mA, fb, kb * BK, I * TM, b);
+            }
             if (ph.mode == kApply) {
 #pragma unroll
               for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mB, fb, J * BN + q * 64, kb * BK, b);
+            } else if (kb >= kbt) {
+#pragma unroll
+              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mBt, fb, J * BN + q * 64, kb * BK, b);
             } else {
 #pragma unroll
               for (int h = 0; h < 2; ++h) tma_load_3d(sb + h * 16384, mB, fb, kb * BK, J * BN + h * 128, b);
@@ -1302,6 +1325,7 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
       const uint64_t b_desc0_k = sdesc_sw128(smem_u32(smem) + A_BYTES, 16, 1024);
       const uint64_t b_desc0_mn = sdesc_sw128(smem_u32(smem) + A_BYTES, 8192, 1024);
+      const uint64_t a_desc0_mn = sdesc_sw128(smem_u32(smem), 8192, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -1317,8 +1341,14 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
         const PhaseDesc& ph = P.ph[find_phase(P, t)];
         const bool mn = ph.mode == kApply;
         const uint32_t idesc = mn ? idesc_mn : idesc_k;
-        const uint64_t b_desc0 = mn ? b_desc0_mn : b_desc0_k;
-        const uint64_t b_step = mn ? (uint64_t)(UK * 128 / 16) : (uint64_t)(UK * 2 / 16);
+        // the k-blocks from which a lower-stored symmetric operand is read transposed
+        int ka = 0x7fffffff, kbt = 0x7fffffff;
+        if (ph.a.sym) {
+          int b, I, J;
+          decode_phase_tile(ph, t, b, I, J);
+          ka = upper_kb(ph.a.sym & 1, I * TM);
+          kbt = upper_kb(ph.mode == kPoly && (ph.a.sym & 2), J * BN);
+        }
         const int num_kb = (ph.a.k + BK - 1) / BK;
         if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, status)) break;
         tc_fence_after();
@@ -1330,10 +1360,15 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
           }
           tc_fence_after();
           const uint64_t soff = (uint64_t)((stage * STAGE_BYTES) >> 4);
+          const bool at = kb >= ka, bt = kb >= kbt;
+          const uint64_t a0 = (at ? a_desc0_mn : a_desc0) + soff;
+          const uint64_t b0 = ((mn || bt) ? b_desc0_mn : b_desc0_k) + soff;
+          const uint32_t astep = at ? UK * 128 / 16 : UK * 2 / 16;
+          const uint32_t bstep = (mn || bt) ? UK * 128 / 16 : UK * 2 / 16;
+          const uint32_t id = idesc | (at ? kIdescAMn : 0u) | (bt ? kIdescBMn : 0u);
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k)
-            tc_mma<G>(d, a_desc0 + soff + (uint64_t)(k * (UK * 2 / 16)), b_desc0 + soff + (uint64_t)k * b_step, idesc,
-                      (kb | k) != 0 ? 1u : 0u);
+            tc_mma<G>(d, a0 + (uint64_t)(k * astep), b0 + (uint64_t)(k * bstep), id, (kb | k) != 0 ? 1u : 0u);
           if constexpr (G == 2)
             tc_commit_pair(B.empty0 + 8 * stage, 0x3);
           else
@@ -1766,7 +1801,12 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
     e = make_map(&P->maps[kMapS0 + i], buf.slot[i] ? buf.slot[i] : buf.slot[0], m, m, batch, ldm, BK, 128);
   if (e == cudaSuccess) e = make_map(&P->maps[kMapX0mn], buf.x[0], n, m, batch, ldn, 64, BK);
   if (e == cudaSuccess) e = make_map(&P->maps[kMapX1mn], buf.x[1], n, m, batch, ldn, 64, BK);
+  for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+    e = make_map(&P->maps[kMapS0t + i], buf.slot[i] ? buf.slot[i] : buf.slot[0], m, m, batch, ldm, 64, BK);
   if (e != cudaSuccess) return e;
+  // the symmetric matrices are stored as their lower 256-column blocks, as in
+  // the per-product launches (DMUON_LOWER_STORE=0: in full)
+  const bool low = !(std::getenv("DMUON_LOWER_STORE") && std::getenv("DMUON_LOWER_STORE")[0] == '0');
 
   int j = 0;
   int64_t tiles = 0, per_matrix = 0;
@@ -1777,6 +1817,12 @@ cudaError_t tc_chain(const ChainBuffers& buf, int batch, int m, int n, int64_t l
     ph.upd = u;
     ph.mapA = mapA;
     ph.mapB = mapB;
+    // operands from the S slots are symmetric; gram and poly outputs too
+    const bool sa = mapA >= kMapS0 && mapA < kMapS0 + 5, sb = mapB >= kMapS0 && mapB < kMapS0 + 5;
+    ph.mapAt = sa ? mapA - kMapS0 + kMapS0t : mapA;
+    ph.mapBt = sb ? mapB - kMapS0 + kMapS0t : mapB;
+    ph.a.lower = low && mode != kApply ? 1 : 0;
+    ph.a.sym = low ? (sa ? 1 : 0) | (sb && mode == kPoly ? 2 : 0) : 0;
     ph.tile_start = (int)tiles;
     ph.dep = (uint32_t)(EPI * G * per_matrix);  // every epilogue warp of every CTA of a tile adds 1
     tiles += a.total_tiles;

@@ -225,15 +225,16 @@ def test_two_chain_streams_give_the_same_bits(name, idx, cap, monkeypatch):
         assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("fused", ["0", "1"])
 @pytest.mark.parametrize("shape", [(4096, 4096), (1408, 2048), (2048, 1408), (1024, 2816), (300, 700), (520, 1300),
                                    (768, 768)], ids=lambda s: f"{s[0]}x{s[1]}")
-def test_lower_stored_symmetric_matrices_give_the_same_bits(shape, monkeypatch):
-    # the per-product chain stores G, p(G) and the Gram-space products as
+def test_lower_stored_symmetric_matrices_give_the_same_bits(shape, fused, monkeypatch):
+    # the chain stores G, p(G) and the Gram-space products as
     # their lower 256-column blocks and reads the upper part of each operand
     # as the transposed lower block; storing them in full must give the same
     # bits (same operand values, same products), in Newton-Schulz and in a
-    # step with the fused update
-    monkeypatch.setenv("DMUON_FUSED_CHAIN", "0")
+    # step with the fused update; per-product launches and the fused chain
+    monkeypatch.setenv("DMUON_FUSED_CHAIN", fused)
     X = seeded(shape, 5 * shape[0] + shape[1])
     p0 = seeded(shape, 17 + shape[0], 0.02)
     g = seeded(shape, 19 + shape[1])

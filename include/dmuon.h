@@ -149,9 +149,10 @@ DMUON_API dmuon_status_t dmuon_ns_ex(const void* X, void* out, int64_t rows, int
  * DMUON_FUSED_UPDATE=0 runs it as a separate pass, with the same bits).  With
  * several chunks the momentum stage (and any separate update) runs on an
  * internal least-priority stream underneath the Newton-Schulz chains, which
- * run on an internal greatest-priority stream; both fork from `stream` and are
- * joined back into it before the call returns, on error paths too.  The
- * results do not depend on that schedule.
+ * run on internal greatest-priority streams (two chunks whose chains are one
+ * launch each may run at once); all fork from `stream` and are joined back
+ * into it before the call returns, on error paths too.  The results do not
+ * depend on that schedule.
  *
  * Routing by shape (m = min(R, C), n = max(R, C)), all in one call: fp32
  * matrices run an FFMA chain with fp32 X, G and p(G); bf16 matrices with

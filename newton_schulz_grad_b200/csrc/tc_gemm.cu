@@ -50,6 +50,7 @@
 #include <cstring>
 #include <memory>
 #include <mutex>
+#include <type_traits>
 
 #include "bounds.cuh"
 #include "internal.h"
@@ -644,6 +645,74 @@ __device__ __forceinline__ Bars bar_layout(uint64_t* bars) {
   return b;
 }
 
+// MMAs of k-blocks [k0, k1) of one tile into accumulator d, with descriptors
+// that do not change inside the range and compile-time k-steps (AT / BT:
+// operand A / B is MN-major, 2048 bytes per 16-row k-step, else K-major, 32
+// bytes): the single issuing thread must keep up with the tensor pipe, so
+// its loop carries nothing but the stage wait, the MMAs and the release.
+// Returns false if a wait ran out.
+template <int G, int STAGES, int STAGE_BYTES, bool AT, bool BT>
+__device__ __forceinline__ bool mma_range(int k0, int k1, uint32_t d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, const Bars& B, int& stage, uint32_t& phase, int* status) {
+  constexpr uint32_t astep = AT ? UK * 128 / 16 : UK * 2 / 16;
+  constexpr uint32_t bstep = BT ? UK * 128 / 16 : UK * 2 / 16;
+  for (int kb = k0; kb < k1; ++kb) {
+    if (!wait_bar(B.full0 + 8 * stage, phase, status)) return false;
+    tc_fence_after();
+    // descriptors of this stage: the bases plus the stage offset (16-byte units)
+    const uint64_t soff = (uint64_t)((stage * STAGE_BYTES) >> 4);
+#pragma unroll
+    for (int k = 0; k < BK / UK; ++k)
+      tc_mma<G>(d, adesc + soff + (uint64_t)(k * astep), bdesc + soff + (uint64_t)(k * bstep), idesc,
+                (kb | k) != 0 ? 1u : 0u);
+    if constexpr (G == 2)
+      tc_commit_pair(B.empty0 + 8 * stage, 0x3);
+    else
+      tc_commit<1>(B.empty0 + 8 * stage);
+    if (++stage == STAGES) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+  return true;
+}
+
+// The k-block ranges of one tile: operand A is read transposed (MN-major,
+// from its lower-stored copy) from k-block ka on, B from kb_t on (never when
+// beyond num_kb), so a tile is at most three ranges in which neither changes.
+// Calls f(A transposed, B transposed, k0, k1) per range, as std::bool_constant
+// tags so that each range's loop is compiled with a fixed pattern (a branch
+// per k-block in the producer's or the MMA thread's loop costs several per
+// cent of the kernel); stops when f returns false.
+template <typename F>
+__device__ __forceinline__ bool for_each_kb_range(int num_kb, int ka, int kb_t, F&& f) {
+  using T = std::true_type;
+  using N = std::false_type;
+  const int x = ka < num_kb ? ka : num_kb, y = kb_t < num_kb ? kb_t : num_kb;
+  const int k1 = x < y ? x : y, k2 = x < y ? y : x;
+  if (!f(N{}, N{}, 0, k1)) return false;
+  if (k1 == num_kb) return true;
+  if (x <= k1 && y <= k1) return f(T{}, T{}, k1, num_kb);
+  const bool ok = x <= k1 ? f(T{}, N{}, k1, k2) : f(N{}, T{}, k1, k2);
+  if (!ok || k2 == num_kb) return ok;
+  return f(T{}, T{}, k2, num_kb);
+}
+
+// All k-blocks of one tile.  a, b: the untransposed base descriptors (b is
+// MN-major when BMN, the apply's X); a_t, b_t: the MN-major ones; idesc: the
+// untransposed instruction descriptor.
+template <int G, int STAGES, int STAGE_BYTES, bool BMN>
+__device__ __forceinline__ bool mma_tile(int num_kb, int ka, int kb_t, uint32_t d, uint64_t a, uint64_t a_t,
+                                         uint64_t b, uint64_t b_t, uint32_t idesc, const Bars& B, int& stage,
+                                         uint32_t& phase, int* status) {
+  return for_each_kb_range(num_kb, ka, kb_t, [&](auto at, auto bt, int k0, int k1) {
+    constexpr bool AT = decltype(at)::value, BT = decltype(bt)::value;
+    return mma_range<G, STAGES, STAGE_BYTES, AT, BT || BMN>(
+        k0, k1, d, AT ? a_t : a, BT ? b_t : b, idesc | (AT ? kIdescAMn : 0u) | (BT ? kIdescBMn : 0u), B, stage,
+        phase, status);
+  });
+}
+
 // ================================================================ one CTA
 template <int MODE, bool UPD, int EPI>
 __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
@@ -693,36 +762,38 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
       for (int t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
         int b, I, J;
         decode_tile<MODE>(a, t, b, I, J);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, a.status)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = B.full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, STAGE1_BYTES);
-          const uint32_t sa = smem_u32(smem + stage * STAGE1_BYTES);
-          const uint32_t sb = sa + A1_BYTES;
-          if (kb >= upper_kb(MODE != kGram && (a.sym & 1), I * BM1)) {
+        const int ka = upper_kb(MODE != kGram && (a.sym & 1), I * BM1);
+        const int kbt = upper_kb(MODE == kPoly && (a.sym & 2), J * BN);
+        ok = for_each_kb_range(num_kb, ka, kbt, [&](auto at, auto bt, int k0, int k1) {
+          for (int kb = k0; kb < k1; ++kb) {
+            if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, a.status)) return false;
+            const uint32_t fb = B.full0 + 8 * stage;
+            mbar_arrive_expect_tx(fb, STAGE1_BYTES);
+            const uint32_t sa = smem_u32(smem + stage * STAGE1_BYTES);
+            const uint32_t sb = sa + A1_BYTES;
+            if constexpr (decltype(at)::value) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) tma_load_3d(sa + q * 8192, &tmAt, fb, I * BM1 + q * 64, kb * BK, b);
-          } else {
-            tma_load_3d(sa, &tmA, fb, kb * BK, I * BM1, b);
-          }
-          if (MODE == kApply) {
+              for (int q = 0; q < 2; ++q) tma_load_3d(sa + q * 8192, &tmAt, fb, I * BM1 + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d(sa, &tmA, fb, kb * BK, I * BM1, b);
+            }
+            if constexpr (MODE == kApply) {
 #pragma unroll
-            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmB, fb, J * BN + q * 64, kb * BK, b);
-          } else if (kb >= upper_kb(MODE == kPoly && (a.sym & 2), J * BN)) {
+              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmB, fb, J * BN + q * 64, kb * BK, b);
+            } else if constexpr (decltype(bt)::value) {
 #pragma unroll
-            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmBt, fb, J * BN + q * 64, kb * BK, b);
-          } else {
-            tma_load_3d(sb, &tmB, fb, kb * BK, J * BN, b);
+              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &tmBt, fb, J * BN + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d(sb, &tmB, fb, kb * BK, J * BN, b);
+            }
+            ++issued;
+            if (++stage == STAGES1) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          ++issued;
-          if (++stage == STAGES1) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+          return true;
+        });
       }
       // wait for the copies still in flight (all have landed on the normal path)
       const int64_t first = issued > STAGES1 ? issued - STAGES1 : 0;
@@ -759,29 +830,8 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1)
         if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(B.full0 + 8 * stage, phase, a.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // descriptors of this stage: the bases plus the stage offset (16-byte units)
-          const uint64_t soff = (uint64_t)((stage * STAGE1_BYTES) >> 4);
-          const bool at = kb >= ka, bt = kb >= kbt;
-          const uint64_t a0 = (at ? a_desc0_t : a_desc0) + soff;
-          const uint64_t b0 = (bt ? b_desc0_t : b_desc0) + soff;
-          const uint32_t astep = at ? UK * 128 / 16 : UK * 2 / 16;
-          const uint32_t bstep = (MODE == kApply || bt) ? UK * 128 / 16 : UK * 2 / 16;
-          const uint32_t id = idesc | (at ? kIdescAMn : 0u) | (bt ? kIdescBMn : 0u);
-#pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
-            tc_mma<1>(d, a0 + (uint64_t)(k * astep), b0 + (uint64_t)(k * bstep), id, (kb | k) != 0 ? 1u : 0u);
-          tc_commit<1>(B.empty0 + 8 * stage);
-          if (++stage == STAGES1) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+        ok = mma_tile<1, STAGES1, STAGE1_BYTES, MODE == kApply>(num_kb, ka, kbt, d, a_desc0, a_desc0_t, b_desc0,
+                                                                 b_desc0_t, idesc, B, stage, phase, a.status);
         if (!ok) break;
         tc_commit<1>(B.tfull0 + 8 * acc);
         if (++acc == 2) {
@@ -879,39 +929,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
       for (int t = pair; ok && t < a.total_tiles; t += npairs) {
         int b, I, J;
         decode_tile<MODE>(a, t, b, I, J);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, a.status)) {
-            ok = false;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(B.full0 + 8 * stage, 2 * STAGE2_BYTES);
-          const uint32_t fb = full_leader0 + 8 * stage;
-          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
-          const uint32_t sb = sa + A2_BYTES;
-          if (kb >= upper_kb(MODE != kGram && (a.sym & 1), I * BM2)) {
+        const int ka = upper_kb(MODE != kGram && (a.sym & 1), I * BM2);
+        const int kbt = upper_kb(MODE == kPoly && (a.sym & 2), J * BN);
+        const int r0 = I * BM2 + (int)rank * 128, n0 = J * BN + (int)rank * 128;
+        ok = for_each_kb_range(num_kb, ka, kbt, [&](auto at, auto bt, int k0, int k1) {
+          for (int kb = k0; kb < k1; ++kb) {
+            if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, a.status)) return false;
+            if (leader) mbar_arrive_expect_tx(B.full0 + 8 * stage, 2 * STAGE2_BYTES);
+            const uint32_t fb = full_leader0 + 8 * stage;
+            const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
+            const uint32_t sb = sa + A2_BYTES;
+            if constexpr (decltype(at)::value) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-              tma_load_3d_pair(sa + q * 8192, &tmAt, fb, I * BM2 + (int)rank * 128 + q * 64, kb * BK, b);
-          } else {
-            tma_load_3d_pair(sa, &tmA, fb, kb * BK, I * BM2 + (int)rank * 128, b);
-          }
-          if (MODE == kApply) {
+              for (int q = 0; q < 2; ++q) tma_load_3d_pair(sa + q * 8192, &tmAt, fb, r0 + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d_pair(sa, &tmA, fb, kb * BK, r0, b);
+            }
+            if constexpr (MODE == kApply) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-              tma_load_3d_pair(sb + q * 8192, &tmB, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
-          } else if (kb >= upper_kb(MODE == kPoly && (a.sym & 2), J * BN)) {
+              for (int q = 0; q < 2; ++q) tma_load_3d_pair(sb + q * 8192, &tmB, fb, n0 + q * 64, kb * BK, b);
+            } else if constexpr (decltype(bt)::value) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-              tma_load_3d_pair(sb + q * 8192, &tmBt, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
-          } else {
-            tma_load_3d_pair(sb, &tmB, fb, kb * BK, J * BN + (int)rank * 128, b);
+              for (int q = 0; q < 2; ++q) tma_load_3d_pair(sb + q * 8192, &tmBt, fb, n0 + q * 64, kb * BK, b);
+            } else {
+              tma_load_3d_pair(sb, &tmB, fb, kb * BK, n0, b);
+            }
+            ++issued;
+            if (++stage == STAGES2) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          ++issued;
-          if (++stage == STAGES2) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+          return true;
+        });
       }
       // the leader sees both CTAs' copies land on its full barriers
       if (leader) {
@@ -951,29 +1001,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Epi<EPI>::kThreads, 
         if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, a.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(B.full0 + 8 * stage, phase, a.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // descriptors of this stage: the bases plus the stage offset (16-byte units)
-          const uint64_t soff = (uint64_t)((stage * STAGE2_BYTES) >> 4);
-          const bool at = kb >= ka, bt = kb >= kbt;
-          const uint64_t a0 = (at ? a_desc0_t : a_desc0) + soff;
-          const uint64_t b0 = (bt ? b_desc0_t : b_desc0) + soff;
-          const uint32_t astep = at ? UK * 128 / 16 : UK * 2 / 16;
-          const uint32_t bstep = (MODE == kApply || bt) ? UK * 128 / 16 : UK * 2 / 16;
-          const uint32_t id = idesc | (at ? kIdescAMn : 0u) | (bt ? kIdescBMn : 0u);
-#pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
-            tc_mma<2>(d, a0 + (uint64_t)(k * astep), b0 + (uint64_t)(k * bstep), id, (kb | k) != 0 ? 1u : 0u);
-          tc_commit_pair(B.empty0 + 8 * stage, 0x3);
-          if (++stage == STAGES2) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+        ok = mma_tile<2, STAGES2, STAGE2_BYTES, MODE == kApply>(num_kb, ka, kbt, d, a_desc0, a_desc0_t, b_desc0,
+                                                                 b_desc0_t, idesc, B, stage, phase, a.status);
         if (!ok) break;
         tc_commit_pair(B.tfull0 + 8 * acc, 0x3);
         if (++acc == 2) {
@@ -1256,58 +1285,54 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
         const int ka = upper_kb(ph.a.sym & 1, I * TM);
         const int kbt = upper_kb(ph.mode == kPoly && (ph.a.sym & 2), J * BN);
         const int num_kb = (ph.a.k + BK - 1) / BK;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, status)) {
-            ok = false;
-            break;
+        const bool apply_b = ph.mode == kApply;  // B is X, MN-major
+        ok = for_each_kb_range(num_kb, ka, kbt, [&](auto at, auto bt, int k0, int k1) {
+          for (int kb = k0; kb < k1; ++kb) {
+            if (!wait_bar(B.empty0 + 8 * stage, phase ^ 1u, status)) return false;
+            if (leader) mbar_arrive_expect_tx(B.full0 + 8 * stage, G * STAGE_BYTES);
+            const uint32_t fb = full_base + 8 * stage;
+            const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+            const uint32_t sb = sa + A_BYTES;
+            if constexpr (G == 2) {
+              const int r0 = I * TM + (int)rank * 128, n0 = J * BN + (int)rank * 128;
+              if constexpr (decltype(at)::value) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) tma_load_3d_pair(sa + q * 8192, mAt, fb, r0 + q * 64, kb * BK, b);
+              } else {
+                tma_load_3d_pair(sa, mA, fb, kb * BK, r0, b);
+              }
+              if (apply_b || decltype(bt)::value) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                  tma_load_3d_pair(sb + q * 8192, apply_b ? mB : mBt, fb, n0 + q * 64, kb * BK, b);
+              } else {
+                tma_load_3d_pair(sb, mB, fb, kb * BK, n0, b);
+              }
+            } else {
+              if constexpr (decltype(at)::value) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) tma_load_3d(sa + q * 8192, mAt, fb, I * TM + q * 64, kb * BK, b);
+              } else {
+                tma_load_3d(sa, mA, fb, kb * BK, I * TM, b);
+              }
+              if (apply_b || decltype(bt)::value) {
+#pragma unroll
+                for (int q = 0; q < BN / 64; ++q)
+                  tma_load_3d(sb + q * 8192, apply_b ? mB : mBt, fb, J * BN + q * 64, kb * BK, b);
+              } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) tma_load_3d(sb + h * 16384, mB, fb, kb * BK, J * BN + h * 128, b);
+              }
+            }
+            ++issued;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          if (leader) mbar_arrive_expect_tx(B.full0 + 8 * stage, G * STAGE_BYTES);
-          const uint32_t fb = full_base + 8 * stage;
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
-          if constexpr (G == 2) {
-            if (kb >= ka) {
-#pragma unroll
-              for (int q = 0; q < 2; ++q)
-                tma_load_3d_pair(sa + q * 8192, mAt, fb, I * TM + (int)rank * 128 + q * 64, kb * BK, b);
-            } else {
-              tma_load_3d_pair(sa, mA, fb, kb * BK, I * TM + (int)rank * 128, b);
-            }
-            if (ph.mode == kApply) {
-#pragma unroll
-              for (int q = 0; q < 2; ++q)
-                tma_load_3d_pair(sb + q * 8192, mB, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
-            } else if (kb >= kbt) {
-#pragma unroll
-              for (int q = 0; q < 2; ++q)
-                tma_load_3d_pair(sb + q * 8192, mBt, fb, J * BN + (int)rank * 128 + q * 64, kb * BK, b);
-            } else {
-              tma_load_3d_pair(sb, mB, fb, kb * BK, J * BN + (int)rank * 128, b);
-            }
-          } else {
-            if (kb >= ka) {
-#pragma unroll
-              for (int q = 0; q < 2; ++q) tma_load_3d(sa + q * 8192, mAt, fb, I * TM + q * 64, kb * BK, b);
-            } else {
-              tma_load_3d(sa, mA, fb, kb * BK, I * TM, b);
-            }
-            if (ph.mode == kApply) {
-#pragma unroll
-              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mB, fb, J * BN + q * 64, kb * BK, b);
-            } else if (kb >= kbt) {
-#pragma unroll
-              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mBt, fb, J * BN + q * 64, kb * BK, b);
-            } else {
-#pragma unroll
-              for (int h = 0; h < 2; ++h) tma_load_3d(sb + h * 16384, mB, fb, kb * BK, J * BN + h * 128, b);
-            }
-          }
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+          return true;
+        });
+        if (!ok) break;
       }
       if (leader) {
         const int64_t first = issued > STAGES ? issued - STAGES : 0;
@@ -1353,31 +1378,10 @@ __global__ void __launch_bounds__(Epi<EPI>::kThreads, 1) k_chain(const __grid_co
         if (!wait_bar(B.tempty0 + 8 * acc, acc_phase ^ 1u, status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait_bar(B.full0 + 8 * stage, phase, status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t soff = (uint64_t)((stage * STAGE_BYTES) >> 4);
-          const bool at = kb >= ka, bt = kb >= kbt;
-          const uint64_t a0 = (at ? a_desc0_mn : a_desc0) + soff;
-          const uint64_t b0 = ((mn || bt) ? b_desc0_mn : b_desc0_k) + soff;
-          const uint32_t astep = at ? UK * 128 / 16 : UK * 2 / 16;
-          const uint32_t bstep = (mn || bt) ? UK * 128 / 16 : UK * 2 / 16;
-          const uint32_t id = idesc | (at ? kIdescAMn : 0u) | (bt ? kIdescBMn : 0u);
-#pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
-            tc_mma<G>(d, a0 + (uint64_t)(k * astep), b0 + (uint64_t)(k * bstep), id, (kb | k) != 0 ? 1u : 0u);
-          if constexpr (G == 2)
-            tc_commit_pair(B.empty0 + 8 * stage, 0x3);
-          else
-            tc_commit<1>(B.empty0 + 8 * stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+        ok = mn ? mma_tile<G, STAGES, STAGE_BYTES, true>(num_kb, ka, kbt, d, a_desc0, a_desc0_mn, b_desc0_mn,
+                                                         b_desc0_mn, idesc, B, stage, phase, status)
+                : mma_tile<G, STAGES, STAGE_BYTES, false>(num_kb, ka, kbt, d, a_desc0, a_desc0_mn, b_desc0_k,
+                                                          b_desc0_mn, idesc, B, stage, phase, status);
         if (!ok) break;
         if constexpr (G == 2)
           tc_commit_pair(B.tfull0 + 8 * acc, 0x3);

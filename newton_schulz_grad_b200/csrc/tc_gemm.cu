@@ -8,9 +8,10 @@
 //                                                  one triangle again)
 // The poly kernel is the general symmetric product C = p1 (A B) + p0 E + p2 I
 // for symmetric, commuting A and B (so A B is symmetric and B's rows are its
-// columns): the Gram-space form of the chain multiplies polynomials of one
-// Gram matrix this way.
-//   apply: Y = alpha (a X + P X)  m x n, K = m   (X is the MN-major operand)
+// columns): the chain stores p(G) = a I + b G + c G G this way, and its
+// Gram-space form multiplies polynomials of one Gram matrix.
+//   apply: Y = alpha (a X + P X)  m x n, K = m   (X is the MN-major operand;
+//                                                  the chain passes a = 0)
 //
 // Two kernels share the tile decode and the epilogue:
 //
@@ -31,10 +32,13 @@
 // thread, warps 2-5 epilogue, 2-9 for reductions up to 2048), with two TMEM
 // accumulators (2 x 256 fp32 columns) so the epilogue of one tile overlaps
 // the MMAs of the next.  The
-// polynomial terms (alpha, b G, a X) are fused into the epilogue.  For gram
-// and poly only tiles that touch the lower triangle are computed; every
-// element r >= c is stored, and r > c also at its mirror (c, r), so each
-// element is written exactly once and G, P are exactly symmetric.
+// polynomial terms (alpha, b G, a I, a X) are fused into the epilogue.  For
+// gram and poly only tiles that touch the lower triangle are computed; every
+// element r >= c is stored, and r > c also at its mirror (c, r), so G and P
+// are exactly symmetric.  Inside a chain the mirror is written only within
+// the diagonal 256 x 256 blocks (lower-stored matrices, see TcArgs::lower):
+// the consumers read an operand's blocks right of its own 256-row block as
+// the transposed lower block.
 //
 // Every mbarrier wait is bounded (%globaltimer); a wait that runs out records
 // DMUON_ERR_TIMEOUT in the status word, the CTA waits (bounded) for its own

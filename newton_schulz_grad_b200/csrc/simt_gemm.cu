@@ -6,15 +6,20 @@
 // exceeds the error budget there.  The three kernels are the three products
 // of one iteration (Gram Newton-Schulz, as the DMuon FAQ's related-work
 // entry names the default "gram" backend):
-//   gram:  G = alpha * X X^T           (one triangle of 64x64 tiles, mirrored)
+//   gram:  G = alpha * X X^T           (one triangle of tiles, mirrored)
 //   poly:  P = b G + c G G             (G symmetric, so G G = G G^T)
 //   apply: Y = alpha * (a X + P X)
-// 64x64 output tiles, k-slices of 16 staged in shared memory, 256 threads
-// with a 4x4 register tile each; fp32 accumulation in a fixed order, blocked:
-// each run of 256 k is summed on its own and then added to the total, so the
-// rounding error grows with 256 + k / 256 rather than k (a 1 x 2^20 fp32
-// vector: 6e-4 relative error unblocked, well inside 1e-4 blocked).  For
-// k <= 256 the result is the plain running sum.
+// Output tiles of 64 x 64 (256 threads, a 4 x 4 register tile each, k in
+// slices of 32) or, for chains too small to fill the GPU with those, 32 x 32
+// (128 threads, 2 x 4 each, slices of 64: four times the tiles).  fp32
+// accumulation in a fixed order, blocked: each run of 256 k is summed on its
+// own and then added to the total, so the rounding error grows with
+// 256 + k / 256 rather than k (a 1 x 2^20 fp32 vector: 6e-4 relative error
+// unblocked, well inside 1e-4 blocked).  For k <= 256 the result is the plain
+// running sum.  Every output element is the same sum in the same order
+// whatever the tile shape, so both shapes give the same bits.
+#include <algorithm>
+#include <cstdlib>
 #include <memory>
 
 #include "common.cuh"
@@ -23,10 +28,23 @@
 namespace dmuon {
 namespace {
 
-constexpr int SB = 64;
-constexpr int SK = 32;
-constexpr int kBlockSlices = 8;  // k-slices per accumulation block (256 k)
-constexpr int kThreads = 256;
+// BM x BM output tiles, THREADS threads with an RM x 4 register tile each,
+// k in slices of SK.  Operands move from global memory in runs of 16 bytes
+// (4 fp32 or 8 bf16 elements) along their contiguous dimension; run s of a
+// thread is number tid + THREADS * s of the slice, so a warp reads whole
+// 64- to 256-byte row segments.
+template <int BM_, int THREADS_, int RM_, int SK_>
+struct SimtCfg {
+  static constexpr int BM = BM_, kThreads = THREADS_, RM = RM_, RN = 4, SK = SK_;
+  static constexpr int TX = BM / RN;               // threads across a tile's columns
+  static constexpr int kBlockSlices = 256 / SK;    // slices per accumulation block (256 k)
+  static constexpr int kPerThread = BM * SK / kThreads;  // elements of each operand per slice
+  static constexpr int kPitch = BM + 4;            // floats per shared-memory row
+  static_assert((kThreads / TX) * RM == BM, "register tiles cover the output tile");
+  static_assert(256 % SK == 0 && BM % 4 == 0, "slices divide the accumulation block");
+};
+using Wide = SimtCfg<64, 256, 4, 32>;
+using Narrow = SimtCfg<32, 128, 2, 64>;
 
 enum { kGram = 0, kPoly = 1, kApply = 2 };
 
@@ -36,12 +54,13 @@ struct SimtArgs {
   const void* E;    // epilogue operand (G for poly, X for apply)
   void* C;          // output
   int64_t sA, sB, sE, sC;  // batch strides (elements)
-  int64_t lda, ldb, lde, ldc;
+  int64_t lda, ldb, ldc, lde;
   int m, n, k;      // output m x n, reduction length k
   float p0, p1;     // gram: alpha; poly: b, c; apply: a, alpha
   const float* scale;
   int tiles_n, tiles_per_mat;
   int batch;
+  int vec;          // bit 0: A, bit 1: B start every 16-byte run on a 16-byte boundary
   int* status;      // device status word (bounds errors of debug builds)
 };
 
@@ -59,6 +78,57 @@ __device__ __forceinline__ float ld(const T* p, int64_t i) {
   }
 }
 
+// One 16-byte run (4 fp32 or 8 bf16 elements) at p, 16-byte aligned, as fp32.
+template <typename T, bool COH>
+__device__ __forceinline__ void ld_run(const T* p, float* v) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 f = COH ? __ldcg(reinterpret_cast<const float4*>(p)) : *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+  } else {
+    const uint4 u = COH ? __ldcg(reinterpret_cast<const uint4*>(p)) : *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+}
+
+// Fetches this thread's runs of the NR x NC region at (r0, c0) of the
+// row-major operand M (leading dimension ldm, rows x cols valid; base and
+// extent locate M inside its buffer for the bounds checks of debug builds)
+// into v; elements outside the valid extent read as 0.  Run s is number
+// u = tid + THREADS * s of the region, at row u / (NC / R), column
+// (u % (NC / R)) * R.  vec: every run may be read as one aligned 16-byte load.
+template <typename T, bool COH, int NR, int NC, int THREADS>
+__device__ __forceinline__ void fetch_runs(const T* M, int64_t ldm, int rows, int cols, int r0, int c0, bool vec,
+                                           float* v, int* status, int64_t base, int64_t extent) {
+  constexpr int R = 16 / (int)sizeof(T);
+  constexpr int kRowRuns = NC / R;
+  constexpr int kRuns = NR * NC / (R * THREADS);
+  static_assert(kRuns * R * THREADS == NR * NC, "runs cover the region");
+#pragma unroll
+  for (int s = 0; s < kRuns; ++s) {
+    const int u = threadIdx.x + THREADS * s;
+    const int gr = r0 + u / kRowRuns, gc = c0 + (u % kRowRuns) * R;
+    float* w = v + s * R;
+    const int64_t off = (int64_t)gr * ldm + gc;
+    if (vec && gr < rows && gc + R <= cols && DMUON_IN(status, base + off, R, extent) &&
+        DMUON_IN(status, gc, R, ldm)) {
+      ld_run<T, COH>(M + off, w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < R; ++e)
+        w[e] = (gr < rows && gc + e < cols && DMUON_IN(status, base + off + e, 1, extent) &&
+                DMUON_IN(status, gc + e, 1, ldm))
+                   ? ld<T, COH>(M, off + e)
+                   : 0.f;
+    }
+  }
+}
+
 // linear triangle index l -> (ti, tj) with tj <= ti
 __device__ __forceinline__ void tri_decode(int l, int& ti, int& tj) {
   int t = (int)((sqrtf(8.f * (float)l + 1.f) - 1.f) * 0.5f);
@@ -68,14 +138,43 @@ __device__ __forceinline__ void tri_decode(int l, int& ti, int& tj) {
   tj = l - t * (t + 1) / 2;
 }
 
-// One 64 x 64 output tile `tile` of matrix b (all 256 threads).  The k loop
-// runs over slices of 32 in two shared-memory buffers: the next slice's
-// global loads are issued before the current slice is multiplied, so their
-// latency overlaps the arithmetic (one barrier per slice).  Each thread keeps
-// a 4 x 4 register tile and adds k in ascending order, in blocks of 256.
-template <typename TA, typename TB, typename TE, typename TC, int MODE, bool COH>
-__device__ __forceinline__ void simt_tile(const SimtArgs& a, int tile, int b, float (&As)[2][SK][SB + 4],
-                                          float (&Bs)[2][SK][SB + 4]) {
+// Shared-memory column of tile row (or column) r in k row kk of a transposed
+// (k-major) operand slice: groups of 4 consecutive rows are permuted by an
+// XOR with kk / 4, so that the transposing stores of a warp spread over the
+// banks while each thread's 4 (or 2) rows stay contiguous for vector reads.
+template <class CFG>
+__device__ __forceinline__ int swz(int kk, int r) {
+  return ((((r >> 2) ^ (kk >> 2)) & (CFG::BM / 4 - 1)) << 2) | (r & 3);
+}
+
+template <class CFG>
+struct SimtSmem {
+  float As[2][CFG::SK][CFG::kPitch];
+  float Bs[2][CFG::SK][CFG::kPitch];
+};
+
+// Transposing store of this thread's runs of a k-contiguous BM x SK slice
+// (fetched by fetch_runs with runs of R elements): element (row r, k kk)
+// goes to [kk][swz(kk, r)].
+template <class CFG, int R>
+__device__ __forceinline__ void stash_t(float (*S)[CFG::kPitch], const float* v) {
+  constexpr int kRowRuns = CFG::SK / R;
+#pragma unroll
+  for (int e = 0; e < CFG::kPerThread; ++e) {
+    const int u = threadIdx.x + CFG::kThreads * (e / R);
+    const int r = u / kRowRuns, kk = (u % kRowRuns) * R + e % R;
+    S[kk][swz<CFG>(kk, r)] = v[e];
+  }
+}
+
+// One BM x BM output tile `tile` of matrix b (all threads of the CTA).  The k
+// loop runs over slices in two shared-memory buffers: the next slice's global
+// loads are issued before the current slice is multiplied, so their latency
+// overlaps the arithmetic (one barrier per slice).  Each thread keeps an
+// RM x 4 register tile and adds k in ascending order, in blocks of 256.
+template <class CFG, typename TA, typename TB, typename TE, typename TC, int MODE, bool COH>
+__device__ __forceinline__ void simt_tile(const SimtArgs& a, int tile, int b, SimtSmem<CFG>& sm) {
+  constexpr int BM = CFG::BM, SK = CFG::SK, RM = CFG::RM, T = CFG::kThreads, PT = CFG::kPerThread;
   int ti, tj;
   if (MODE == kApply) {
     ti = tile / a.tiles_n;
@@ -83,63 +182,44 @@ __device__ __forceinline__ void simt_tile(const SimtArgs& a, int tile, int b, fl
   } else {
     tri_decode(tile, ti, tj);
   }
-  const int i0 = ti * SB, j0 = tj * SB;
+  const int i0 = ti * BM, j0 = tj * BM;
   const TA* A = static_cast<const TA*>(a.A) + (int64_t)b * a.sA;
   const TB* B = static_cast<const TB*>(a.B) + (int64_t)b * a.sB;
   const int tid = threadIdx.x;
-  const int ty = tid / 16, tx = tid % 16;
-  float acc[4][4], part[4][4];
+  const int ty = tid / CFG::TX, tx = tid % CFG::TX;
+  float acc[RM][4], part[RM][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < RM; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = part[i][j] = 0.f;
 
-  // per slice each thread moves 8 elements of A (row tid/4, k (tid%4)*8..+7)
-  // and 8 of B: k-major rows like A, or (apply) row k tid/8, columns (tid%8)*8..+7
-  const int arow = tid / 4, akq = (tid % 4) * 8;
-  const int bkk = tid / 8, bjq = (tid % 8) * 8;
-  float ra[8], rb[8];
+  // A: rows i0.. of a row-major m x k operand (k contiguous); B: rows j0.. of
+  // the same kind (gram, poly), or (apply) a k x n row-major operand
+  const bool vecA = a.vec & 1, vecB = (a.vec >> 1) & 1;
+  const int arows = a.m, brows = MODE == kApply ? a.k : a.n;
+  float ra[PT], rb[PT];
   auto fetch = [&](int k0) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int gr = i0 + arow, gk = k0 + akq + e;
-      ra[e] = (gr < a.m && gk < a.k &&
-               DMUON_IN(a.status, (int64_t)b * a.sA + (int64_t)gr * a.lda + gk, 1, a.batch * a.sA) &&
-               DMUON_IN(a.status, gk, 1, a.lda))
-                  ? ld<TA, COH>(A, (int64_t)gr * a.lda + gk)
-                  : 0.f;
-    }
-    if (MODE == kApply) {  // B is k x n row-major
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int gk = k0 + bkk, gj = j0 + bjq + e;
-        rb[e] = (gk < a.k && gj < a.n &&
-                 DMUON_IN(a.status, (int64_t)b * a.sB + (int64_t)gk * a.ldb + gj, 1, a.batch * a.sB) &&
-                 DMUON_IN(a.status, gj, 1, a.ldb))
-                    ? ld<TB, COH>(B, (int64_t)gk * a.ldb + gj)
-                    : 0.f;
-      }
-    } else {  // B rows j0.. (k-major, like A)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int gr = j0 + arow, gk = k0 + akq + e;
-        rb[e] = (gr < a.n && gk < a.k &&
-                 DMUON_IN(a.status, (int64_t)b * a.sB + (int64_t)gr * a.ldb + gk, 1, a.batch * a.sB) &&
-                 DMUON_IN(a.status, gk, 1, a.ldb))
-                    ? ld<TB, COH>(B, (int64_t)gr * a.ldb + gk)
-                    : 0.f;
-      }
-    }
+    fetch_runs<TA, COH, BM, SK, T>(A, a.lda, arows, a.k, i0, k0, vecA, ra, a.status, (int64_t)b * a.sA,
+                                   (int64_t)a.batch * a.sA);
+    if (MODE == kApply)
+      fetch_runs<TB, COH, SK, BM, T>(B, a.ldb, brows, a.n, k0, j0, vecB, rb, a.status, (int64_t)b * a.sB,
+                                     (int64_t)a.batch * a.sB);
+    else
+      fetch_runs<TB, COH, BM, SK, T>(B, a.ldb, brows, a.k, j0, k0, vecB, rb, a.status, (int64_t)b * a.sB,
+                                     (int64_t)a.batch * a.sB);
   };
   auto stash = [&](int buf) {
+    stash_t<CFG, 16 / (int)sizeof(TA)>(sm.As[buf], ra);
+    if (MODE == kApply) {  // already k-major: 16-byte stores of whole runs
+      constexpr int R = 16 / (int)sizeof(TB);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) As[buf][akq + e][arow] = ra[e];
-    if (MODE == kApply) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) Bs[buf][bkk][bjq + e] = rb[e];
+      for (int e = 0; e < PT; e += 4) {
+        const int u = tid + T * (e / R);
+        const int kk = u / (BM / R), c = (u % (BM / R)) * R + e % R;
+        *reinterpret_cast<float4*>(&sm.Bs[buf][kk][c]) = make_float4(rb[e], rb[e + 1], rb[e + 2], rb[e + 3]);
+      }
     } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) Bs[buf][akq + e][arow] = rb[e];
+      stash_t<CFG, 16 / (int)sizeof(TB)>(sm.Bs[buf], rb);
     }
   };
 
@@ -152,19 +232,25 @@ __device__ __forceinline__ void simt_tile(const SimtArgs& a, int tile, int b, fl
     if (more) fetch(k0 + SK);  // in flight while this slice is multiplied
 #pragma unroll
     for (int kk = 0; kk < SK; ++kk) {
-      // 16-byte shared-memory loads (rows of 68 floats keep them aligned)
-      const float4 a4 = *reinterpret_cast<const float4*>(&As[cur][kk][ty * 4]);
-      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[cur][kk][tx * 4]);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-      const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+      float av[RM], bv[4];
+      if constexpr (RM == 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(&sm.As[cur][kk][swz<CFG>(kk, ty * 4)]);
+        av[0] = a4.x; av[1] = a4.y; av[2] = a4.z; av[3] = a4.w;
+      } else {
+        const float2 a2 = *reinterpret_cast<const float2*>(&sm.As[cur][kk][swz<CFG>(kk, ty * 2)]);
+        av[0] = a2.x; av[1] = a2.y;
+      }
+      const float4 b4 = *reinterpret_cast<const float4*>(
+          &sm.Bs[cur][kk][MODE == kApply ? tx * 4 : swz<CFG>(kk, tx * 4)]);
+      bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < RM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
     }
-    if (++slices == kBlockSlices || !more) {
+    if (++slices == CFG::kBlockSlices || !more) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < RM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           acc[i][j] += part[i][j];
@@ -188,8 +274,8 @@ __device__ __forceinline__ void simt_tile(const SimtArgs& a, int tile, int b, fl
     alpha = 1.f;
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = i0 + ty * 4 + i;
+  for (int i = 0; i < RM; ++i) {
+    const int r = i0 + ty * RM + i;
     if (r >= a.m) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -221,10 +307,9 @@ __device__ __forceinline__ void simt_tile(const SimtArgs& a, int tile, int b, fl
 }
 
 template <typename TA, typename TB, typename TE, typename TC, int MODE>
-__global__ void __launch_bounds__(kThreads) k_simt(const SimtArgs a) {
-  __shared__ __align__(16) float As[2][SK][SB + 4];
-  __shared__ __align__(16) float Bs[2][SK][SB + 4];
-  simt_tile<TA, TB, TE, TC, MODE, false>(a, blockIdx.x, blockIdx.y, As, Bs);
+__global__ void __launch_bounds__(Wide::kThreads) k_simt(const SimtArgs a) {
+  __shared__ __align__(16) SimtSmem<Wide> sm;
+  simt_tile<Wide, TA, TB, TE, TC, MODE, false>(a, blockIdx.x, blockIdx.y, sm);
 }
 
 // ------------------------------------------------------------ fused chain
@@ -281,11 +366,10 @@ __device__ __noinline__ bool wait_count(const unsigned* c, uint32_t target, int*
   }
 }
 
-// XT: element type of X (fp32, or bf16 for thin bf16 matrices)
-template <typename XT>
-__global__ void __launch_bounds__(kThreads) k_simt_chain(const __grid_constant__ SimtChain P) {
-  __shared__ __align__(16) float As[2][SK][SB + 4];
-  __shared__ __align__(16) float Bs[2][SK][SB + 4];
+// XT: element type of X (fp32, or bf16 for thin bf16 matrices); CFG: tile shape
+template <typename XT, class CFG>
+__global__ void __launch_bounds__(CFG::kThreads) k_simt_chain(const __grid_constant__ SimtChain P) {
+  __shared__ __align__(16) SimtSmem<CFG> sm;
   __shared__ int s_tile;
   unsigned* next = P.counters + P.batch;
   while (true) {
@@ -312,11 +396,11 @@ __global__ void __launch_bounds__(kThreads) k_simt_chain(const __grid_constant__
     const int b = local / a.tiles_per_mat;
     const int tile = local - b * a.tiles_per_mat;
     if (mode == kGram)
-      simt_tile<XT, XT, float, float, kGram, true>(a, tile, b, As, Bs);
+      simt_tile<CFG, XT, XT, float, float, kGram, true>(a, tile, b, sm);
     else if (mode == kPoly)
-      simt_tile<float, float, float, float, kPoly, true>(a, tile, b, As, Bs);
+      simt_tile<CFG, float, float, float, float, kPoly, true>(a, tile, b, sm);
     else
-      simt_tile<float, XT, XT, XT, kApply, true>(a, tile, b, As, Bs);
+      simt_tile<CFG, float, XT, XT, XT, kApply, true>(a, tile, b, sm);
     __syncthreads();  // every store of the tile issued
     if (threadIdx.x == 0) {
       __threadfence();
@@ -325,13 +409,20 @@ __global__ void __launch_bounds__(kThreads) k_simt_chain(const __grid_constant__
   }
 }
 
-int tri_tiles(int m) {
-  const int t = (m + SB - 1) / SB;
+int tri_tiles(int m, int bm) {
+  const int t = (m + bm - 1) / bm;
   return t * (t + 1) / 2;
 }
 
+// Every 16-byte run of an operand (element size sz, leading dimension ld,
+// batch stride st, runs starting at multiples of 16 bytes within a row)
+// starts on a 16-byte boundary.
+bool runs_aligned(const void* p, int64_t ld, int64_t st, int64_t sz) {
+  return reinterpret_cast<uintptr_t>(p) % 16 == 0 && (ld * sz) % 16 == 0 && (st * sz) % 16 == 0;
+}
+
 SimtArgs gram_sargs(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg, float alpha,
-                    const float* scale, int* status) {
+                    const float* scale, int64_t xsz, int bm, int* status) {
   SimtArgs a{};
   a.batch = batch; a.status = status;
   a.A = X; a.B = X; a.E = nullptr; a.C = G;
@@ -339,12 +430,13 @@ SimtArgs gram_sargs(const void* X, void* G, int batch, int m, int n, int64_t ldx
   a.lda = a.ldb = ldx; a.ldc = ldg;
   a.m = m; a.n = m; a.k = n;
   a.p0 = alpha; a.scale = scale;
-  a.tiles_per_mat = tri_tiles(m);
+  a.tiles_per_mat = tri_tiles(m, bm);
+  a.vec = runs_aligned(X, ldx, a.sA, xsz) ? 3 : 0;
   return a;
 }
 
 SimtArgs poly_sargs(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b, float c,
-                    int* status) {
+                    int bm, int* status) {
   SimtArgs a{};
   a.batch = batch; a.status = status;
   a.A = G; a.B = G; a.E = G; a.C = P;
@@ -352,12 +444,14 @@ SimtArgs poly_sargs(const void* G, void* P, int batch, int m, int64_t ldg, int64
   a.lda = a.ldb = a.lde = ldg; a.ldc = ldp;
   a.m = m; a.n = m; a.k = m;
   a.p0 = b; a.p1 = c;
-  a.tiles_per_mat = tri_tiles(m);
+  a.tiles_per_mat = tri_tiles(m, bm);
+  a.vec = runs_aligned(G, ldg, a.sA, 4) ? 3 : 0;
   return a;
 }
 
 SimtArgs apply_sargs(const void* P, const void* X, void* Y, int batch, int m, int n, int64_t ldp, int64_t ldx,
-                     int64_t ldy, float a_coef, float alpha, const float* scale, int* status) {
+                     int64_t ldy, float a_coef, float alpha, const float* scale, int64_t xsz, int bm,
+                     int* status) {
   SimtArgs a{};
   a.batch = batch; a.status = status;
   a.A = P; a.B = X; a.E = X; a.C = Y;
@@ -365,9 +459,36 @@ SimtArgs apply_sargs(const void* P, const void* X, void* Y, int batch, int m, in
   a.lda = ldp; a.ldb = a.lde = ldx; a.ldc = ldy;
   a.m = m; a.n = n; a.k = m;
   a.p0 = a_coef; a.p1 = alpha; a.scale = scale;
-  a.tiles_n = (n + SB - 1) / SB;
-  a.tiles_per_mat = ((m + SB - 1) / SB) * a.tiles_n;
+  a.tiles_n = (n + bm - 1) / bm;
+  a.tiles_per_mat = ((m + bm - 1) / bm) * a.tiles_n;
+  a.vec = (runs_aligned(P, ldp, a.sA, 4) ? 1 : 0) | (runs_aligned(X, ldx, a.sB, xsz) ? 2 : 0);
   return a;
+}
+
+// Chains whose widest product has fewer 64 x 64 tiles than the GPU has SMs
+// run 32 x 32 tiles (DMUON_FFMA_TILE=64 or =32 forces one shape).
+bool narrow_chain(int batch, int m, int n, int num_sms) {
+  if (const char* v = std::getenv("DMUON_FFMA_TILE")) {
+    if (v[0] == '6') return false;
+    if (v[0] == '3') return true;
+  }
+  const int64_t t = (m + Wide::BM - 1) / Wide::BM, u = (n + Wide::BM - 1) / Wide::BM;
+  return t * u * batch < num_sms;
+}
+
+template <class CFG, typename XT>
+cudaError_t launch_chain(const SimtChain& C, int64_t widest, int num_sms, cudaStream_t st) {
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_simt_chain<XT, CFG>, CFG::kThreads, 0);
+  if (e != cudaSuccess || per_sm <= 0) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  // no more CTAs than the largest product has tiles: the rest would only wait
+  const int64_t most = (int64_t)num_sms * per_sm;
+  const int grid = (int)(widest < most ? widest : most);
+  k_simt_chain<XT, CFG><<<grid, CFG::kThreads, 0, st>>>(C);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -375,21 +496,21 @@ SimtArgs apply_sargs(const void* P, const void* X, void* Y, int batch, int m, in
 cudaError_t simt_gram(const void* X, void* G, int batch, int m, int n, int64_t ldx, int64_t ldg,
                       float alpha, const float* scale, bool xbf16, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
-  const SimtArgs a = gram_sargs(X, G, batch, m, n, ldx, ldg, alpha, scale, status);
+  const SimtArgs a = gram_sargs(X, G, batch, m, n, ldx, ldg, alpha, scale, xbf16 ? 2 : 4, Wide::BM, status);
   dim3 grid(a.tiles_per_mat, batch);
   if (xbf16)
-    k_simt<__nv_bfloat16, __nv_bfloat16, float, float, kGram><<<grid, kThreads, 0, st>>>(a);
+    k_simt<__nv_bfloat16, __nv_bfloat16, float, float, kGram><<<grid, Wide::kThreads, 0, st>>>(a);
   else
-    k_simt<float, float, float, float, kGram><<<grid, kThreads, 0, st>>>(a);
+    k_simt<float, float, float, float, kGram><<<grid, Wide::kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t simt_poly(const void* G, void* P, int batch, int m, int64_t ldg, int64_t ldp, float b,
                       float c, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
-  const SimtArgs a = poly_sargs(G, P, batch, m, ldg, ldp, b, c, status);
+  const SimtArgs a = poly_sargs(G, P, batch, m, ldg, ldp, b, c, Wide::BM, status);
   dim3 grid(a.tiles_per_mat, batch);
-  k_simt<float, float, float, float, kPoly><<<grid, kThreads, 0, st>>>(a);
+  k_simt<float, float, float, float, kPoly><<<grid, Wide::kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -397,12 +518,13 @@ cudaError_t simt_apply(const void* P, const void* X, void* Y, int batch, int m, 
                        int64_t ldx, int64_t ldy, float a_coef, float alpha, const float* scale,
                        bool xbf16, cudaStream_t st, int* status) {
   if (batch == 0) return cudaSuccess;
-  const SimtArgs a = apply_sargs(P, X, Y, batch, m, n, ldp, ldx, ldy, a_coef, alpha, scale, status);
+  const SimtArgs a =
+      apply_sargs(P, X, Y, batch, m, n, ldp, ldx, ldy, a_coef, alpha, scale, xbf16 ? 2 : 4, Wide::BM, status);
   dim3 grid(a.tiles_per_mat, batch);
   if (xbf16)
-    k_simt<float, __nv_bfloat16, __nv_bfloat16, __nv_bfloat16, kApply><<<grid, kThreads, 0, st>>>(a);
+    k_simt<float, __nv_bfloat16, __nv_bfloat16, __nv_bfloat16, kApply><<<grid, Wide::kThreads, 0, st>>>(a);
   else
-    k_simt<float, float, float, float, kApply><<<grid, kThreads, 0, st>>>(a);
+    k_simt<float, float, float, float, kApply><<<grid, Wide::kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -412,9 +534,12 @@ cudaError_t simt_chain(void* const* x, void* G, void* P, int batch, int m, int n
   *result_x = 0;
   if (batch == 0 || steps == 0) return cudaSuccess;
   if (3 * steps > kMaxSimtPhases || !counters) return cudaErrorNotSupported;
+  const bool narrow = narrow_chain(batch, m, n, num_sms);
+  const int bm = narrow ? Narrow::BM : Wide::BM;
+  const int64_t xsz = xbf16 ? 2 : 4;
   std::unique_ptr<SimtChain> C(new SimtChain());
   int j = 0;
-  int64_t tiles = 0, per_matrix = 0;
+  int64_t tiles = 0, per_matrix = 0, widest = 0;
   auto add = [&](const SimtArgs& a, int mode) {
     SimtPhase& ph = C->ph[j++];
     ph.a = a;
@@ -423,14 +548,15 @@ cudaError_t simt_chain(void* const* x, void* G, void* P, int batch, int m, int n
     ph.dep = (uint32_t)per_matrix;  // one increment per finished tile
     tiles += (int64_t)a.tiles_per_mat * batch;
     per_matrix += a.tiles_per_mat;
+    widest = std::max(widest, (int64_t)a.tiles_per_mat * batch);
   };
   int cur = 0;
   for (int k = 0; k < steps; ++k) {
     const float* sc = k == 0 ? scale : nullptr;
     const float* c = sched + 3 * k;
-    add(gram_sargs(x[cur], G, batch, m, n, ldx, ldg, 1.f, sc, status), kGram);
-    add(poly_sargs(G, P, batch, m, ldg, ldg, c[1], c[2], status), kPoly);
-    add(apply_sargs(P, x[cur], x[1 - cur], batch, m, n, ldg, ldx, ldx, c[0], 1.f, sc, status), kApply);
+    add(gram_sargs(x[cur], G, batch, m, n, ldx, ldg, 1.f, sc, xsz, bm, status), kGram);
+    add(poly_sargs(G, P, batch, m, ldg, ldg, c[1], c[2], bm, status), kPoly);
+    add(apply_sargs(P, x[cur], x[1 - cur], batch, m, n, ldg, ldx, ldx, c[0], 1.f, sc, xsz, bm, status), kApply);
     cur = 1 - cur;
   }
   if (tiles > 0x7fffffff) return cudaErrorNotSupported;
@@ -447,26 +573,11 @@ cudaError_t simt_chain(void* const* x, void* G, void* P, int batch, int m, int n
   *result_x = cur;
   cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)(batch + 1) * sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = xbf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_simt_chain<__nv_bfloat16>, kThreads, 0)
-            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_simt_chain<float>, kThreads, 0);
-  if (e != cudaSuccess || per_sm <= 0) {
-    cudaGetLastError();
-    per_sm = 1;
-  }
-  // no more CTAs than the largest product has tiles: the rest would only wait
-  int64_t widest = 0;
-  for (int i = 0; i < j; ++i) {
-    const int64_t w = (int64_t)C->ph[i].a.tiles_per_mat * batch;
-    widest = w > widest ? w : widest;
-  }
-  const int64_t most = (int64_t)num_sms * per_sm;
-  const int grid = (int)(widest < most ? widest : most);
-  if (xbf16)
-    k_simt_chain<__nv_bfloat16><<<grid, kThreads, 0, st>>>(*C);
-  else
-    k_simt_chain<float><<<grid, kThreads, 0, st>>>(*C);
-  return cudaGetLastError();
+  if (narrow)
+    return xbf16 ? launch_chain<Narrow, __nv_bfloat16>(*C, widest, num_sms, st)
+                 : launch_chain<Narrow, float>(*C, widest, num_sms, st);
+  return xbf16 ? launch_chain<Wide, __nv_bfloat16>(*C, widest, num_sms, st)
+               : launch_chain<Wide, float>(*C, widest, num_sms, st);
 }
 
 }  // namespace dmuon

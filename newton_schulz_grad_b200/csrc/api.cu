@@ -864,7 +864,8 @@ const char* dmuon_get_last_error(void) { return g_last_error.c_str(); }
 
 const char* dmuon_build_info(void) {
   static std::string s = std::string("dmuon-b200 0.1.0; sm_100a; ") + tc_config_string() +
-                         "; FFMA chain for fp32 and min side <= 64; elementwise 64x64 tiles" +
+                         "; FFMA chain (64x64 or 32x32 tiles) for fp32, for bf16 with min side < 256 and max side < 3 x min,"
+                         " and for bf16 with min side <= 64 beyond the clustered kernel; elementwise 64x64 tiles" +
 #ifdef DMUON_DEBUG
                          "; debug bounds checks";
 #else

@@ -1,9 +1,11 @@
 // FFMA (CUDA-core) kernels of the Gram Newton-Schulz chain.
 //
 // Used for the fp32 dtype (the tensor cores have no fp32-exact product; tf32
-// would lose the 1e-4 budget) and for thin bf16 matrices (min side <= 64),
-// whose Gram matrices stay in fp32 because bf16 rounding of G and p(G) alone
-// exceeds the error budget there.  The three kernels are the three products
+// would lose the 1e-4 budget), for small near-square bf16 matrices (min side
+// < 256, max side < 3 x min), whose X, G and p(G) stay in fp32, and for thin
+// bf16 matrices (min side <= 64) too wide for the clustered kernel, whose G
+// and p(G) stay in fp32: bf16 rounding of G and p(G) alone exceeds the error
+// budget at those sizes.  The three kernels are the three products
 // of one iteration (Gram Newton-Schulz, as the DMuon FAQ's related-work
 // entry names the default "gram" backend):
 //   gram:  G = alpha * X X^T           (one triangle of tiles, mirrored)

@@ -91,6 +91,22 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def roofline_peak(kind: str, has_flops: bool, peaks: dict, sms: int, sm_max_mhz):
+    """(bound, unit, peak, basis) of the step's dominant kernel.  The FFMA
+    kernels (fp32 products on the CUDA cores: `*_ffma`, and the clustered
+    thin-matrix chain `chain_small`) are bound by the FMA issue rate: SMs x 128
+    fp32 lanes (4 schedulers x 32) x 2 flop per cycle at the maximum SM clock;
+    tensor-core kernels by the measured sustained bf16 peak; kernels counted
+    in bytes by the measured copy bandwidth.  basis is None unless derived here."""
+    if has_flops and (kind.endswith("_ffma") or kind == "chain_small"):
+        mhz = float(sm_max_mhz or 1965.0)
+        peak = sms * 128 * 2 * mhz * 1e6 / 1e12
+        return "alu", "TFLOP/s", round(peak, 1), f"{sms} SMs x 128 fp32 lanes x 2 flop x {mhz:.0f} MHz"
+    if has_flops:
+        return "tensor", "TFLOP/s", float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))), None
+    return "hbm", "GB/s", float(peaks["hbm_gbs"]), None
+
+
 def launches_per_matrix(kernel: str, m: int, n: int, dtype: str, steps: int):
     """How many launches of `kernel` one matrix of oriented shape m x n sees in
     a step (the library's default schedule: bf16 matrices with m <= 64, or
@@ -411,14 +427,13 @@ def run_ours(args):
     dom = max(timed_kinds.items(), key=lambda kv: kv[1]["total_ms"])
     dname, d = dom
     avg_ms = d["total_ms"] / d["launches"]
+    bound, unit, peak, peak_basis = roofline_peak(dname, d["flops"] > 0, peaks,
+                                                  torch.cuda.get_device_properties(dev).multi_processor_count,
+                                                  (clk or {}).get("sm_max_mhz"))
     if d["flops"] > 0:
         achieved = (d["flops"] / d["launches"]) / (avg_ms / 1e3) / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-        bound, unit = "tensor", "TFLOP/s"
     else:
         achieved = (d["bytes"] / d["launches"]) / (avg_ms / 1e3) / 1e9
-        peak = float(peaks["hbm_gbs"])
-        bound, unit = "hbm", "GB/s"
     # kernels of the auxiliary stream (momentum, norm, separate update) run
     # underneath the chain: their event windows include time spent queued
     # behind it, so they carry no bandwidth figure here (see elementwise_isolated)
@@ -478,6 +493,7 @@ def run_ours(args):
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
         "roofline": {"kernel": dname, "bound": bound, "achieved": round(achieved, 1), "peak": peak,
                      "unit": unit, "frac": round(achieved / peak, 4),
+                     **({"peak_basis": peak_basis} if peak_basis else {}),
                      "traffic": traffic_record(dname, w, d["launches"] // max(1, args.steps)),
                      "per_launch": {"flops": d["flops"] / d["launches"],
                                     "bytes": d["bytes"] / d["launches"], "avg_ms": avg_ms}},
